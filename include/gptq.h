@@ -1,0 +1,207 @@
+/*
+ * gptq.h — C ABI of libgptq_b200, a B200 (sm_100a) implementation of GPTQ
+ * layer-wise weight quantization.
+ *
+ * Sources (web pages on GPTQ, cited by title and section):
+ *   [GPTQ-tool]  "GPTQ", ozercemkelahmet.com/tools/gptq — How it works,
+ *                Steps 1-9; Optional refinements; A minimal Python sketch;
+ *                Memory arithmetic; Glossary.
+ *   [GPTQ-guide] "GPTQ Quantization: Complete Technical Guide",
+ *                notes.jayaprakash.net — Quantization Equation; Computing the
+ *                Hessian; Configuration Deep Dive.
+ *   [GPTQ-breakdown] "GPTQ", ai360xpert.com/papers/gptq — How It Works.
+ *   [What-is-GPTQ] "What Is GPTQ? Classic 4-Bit LLM Quantization",
+ *                ai-tldr.dev — How it works, Step 3.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.   Every array argument is a DEVICE pointer (memory the caller
+ *             allocated with cudaMalloc or a caching allocator on the device
+ *             the call runs on) unless its comment says otherwise.  The
+ *             library allocates nothing and keeps no state between calls;
+ *             scratch memory is the caller's workspace `ws` of at least
+ *             gptq_workspace_size(...) bytes, 256-byte aligned.
+ * Layout.     Row-major.  W is (r, k): r = out-features (rows), k =
+ *             in-features (columns); X is (n, k): n calibration tokens.
+ *             Leading dimensions are in elements.
+ * Streams.    Every call enqueues its kernels on `stream` (0 = legacy
+ *             default stream) and returns without synchronising.
+ * Errors.     Argument errors are detected on the host and returned before
+ *             anything is enqueued.  GPTQ_ERR_CUDA means a launch failed
+ *             (the CUDA error is left for cudaGetLastError to report).
+ *             Failures that only the device can see are written to device
+ *             status words (`d_info`, `d_status`) that the caller reads after
+ *             synchronising; no kernel traps, asserts or waits without bound.
+ * Inputs.     W, X and H are never modified.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GPTQ_API __attribute__((visibility("default")))
+#else
+#define GPTQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* gptq_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, leading dimension, alignment */
+  GPTQ_ERR_NOT_PD = 2,      /* damped Hessian not positive definite (device: d_info) */
+  GPTQ_ERR_CUDA = 3,        /* a kernel launch failed */
+  GPTQ_ERR_UNSUPPORTED = 4, /* valid request this build does not implement (bits, dtype) */
+  GPTQ_ERR_WORKSPACE = 5,   /* workspace null, too small or misaligned */
+  GPTQ_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
+  GPTQ_ERR_NONFINITE = 7    /* NaN/Inf met in the weights being quantized (device: d_status) */
+} gptq_status;
+
+typedef enum { GPTQ_F32 = 0, GPTQ_F16 = 1, GPTQ_BF16 = 2 } gptq_dtype;
+
+/* Quantization settings ([GPTQ-guide] Configuration Deep Dive; [GPTQ-tool]
+ * Optional refinements).
+ *   bits        2, 3, 4 or 8: codes are 0 .. 2^bits-1 on an asymmetric grid.
+ *   group_size  columns (in processing order) sharing one scale/zero per row;
+ *               -1 = one group per row.  Must divide block_size or be a
+ *               multiple of it, so a group never straddles a lazy block.
+ *   block_size  lazy-batch width B ([GPTQ-tool] Step 7), 16..128, multiple of 16.
+ *   percdamp    damping fraction of mean(diag H) ([GPTQ-tool] Step 4), >= 0.
+ *   act_order   nonzero: process columns by descending diag(H).
+ *   sym         reserved, must be 0 (asymmetric grid only). */
+typedef struct {
+  int bits;
+  int group_size;
+  int block_size;
+  float percdamp;
+  int act_order;
+  int sym;
+} gptq_config;
+
+typedef enum {
+  GPTQ_OP_HESSIAN = 0,
+  GPTQ_OP_PREPARE_HINV = 1,
+  GPTQ_OP_QUANTIZE = 2
+} gptq_op;
+
+/* Bytes of workspace `op` needs for the given sizes (n is ignored except by
+ * GPTQ_OP_HESSIAN; cfg may be NULL for GPTQ_OP_HESSIAN).  0 means none. */
+GPTQ_API size_t gptq_workspace_size(int op, int64_t r, int64_t k, int64_t n, const gptq_config* cfg);
+
+/* Human-readable name of a status code (static storage). */
+GPTQ_API const char* gptq_status_string(gptq_status s);
+
+/* Hessian accumulation: H += alpha * X^T X.
+ * [GPTQ-tool] Step 3 and A minimal Python sketch (H = 2 X^T X / n);
+ * [GPTQ-guide] Computing the Hessian.  Call once per chunk of calibration
+ * tokens with alpha = 2 / n_total (n_total = tokens over all chunks).
+ *   X      (n, k) row-major, dtype `dt`, leading dimension ldx >= k.
+ *          F16 / BF16 are accumulated on the tensor cores (exact products,
+ *          fp32 accumulation over short token runs, re-accumulated in fp32);
+ *          F32 on the CUDA cores in fp32.  F16/BF16 need k % 8 == 0,
+ *          ldx % 8 == 0 and a 16-byte aligned X.
+ *   H      (k, k) fp32, symmetric on entry (zero it before the first chunk);
+ *          both triangles are updated.  Must not alias X.
+ *   ws     GPTQ_OP_HESSIAN workspace (may be NULL when that size is 0).
+ * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_WORKSPACE, GPTQ_ERR_CUDA.
+ * n == 0 or k == 0 is a no-op. */
+GPTQ_API gptq_status gptq_hessian_accumulate(const void* X, gptq_dtype dt, int64_t n, int64_t k,
+                                    int64_t ldx, float alpha, float* H, void* ws,
+                                    size_t ws_bytes, gptq_stream_t stream);
+
+/* Inverse-Hessian factor with dead columns, act-order and damping.
+ * [GPTQ-tool] Steps 4 and 6, Optional refinements (act-order), and the
+ * sketch's factor cholesky(cholesky_inverse(cholesky(H)), upper=True).
+ *   H       (k, k) fp32 undamped Hessian (read only).
+ *   Steps:  dead = {i : H_ii == 0} (those get H_ii := 1; the sweep zeroes
+ *           their weights); perm = stable sort of columns by descending
+ *           diag(H) if cfg->act_order, else identity; Hp = H[perm][:, perm];
+ *           Hp += percdamp * mean(diag Hp) * I; U = upper Cholesky factor of
+ *           Hp^-1 (U^T U = Hp^-1), computed as U = V^-1 with Hp = V V^T,
+ *           V upper (a bottom-up Cholesky), never forming Hp^-1.
+ *   U       (k, k) fp32 out, row-major, in PROCESSING order; lower triangle
+ *           written as 0.
+ *   perm    int32[k] out: perm[j] = original column processed j-th.
+ *   invperm int32[k] out: invperm[perm[j]] = j.
+ *   dead    uint8[k] out (original column order): 1 = dead column.
+ *   d_info  int32 device scalar out: 0, or 1 + the processing-order index
+ *           of the first pivot found non-positive or non-finite (then U is
+ *           unspecified; retry with a larger percdamp).
+ *   ws      GPTQ_OP_PREPARE_HINV workspace.
+ * Returns GPTQ_OK (the device may still report NOT_PD in d_info),
+ * GPTQ_ERR_INVALID_ARG, GPTQ_ERR_WORKSPACE, GPTQ_ERR_CUDA. */
+GPTQ_API gptq_status gptq_prepare_hinv(const float* H, int64_t k, const gptq_config* cfg, float* U,
+                              int32_t* perm, int32_t* invperm, uint8_t* dead,
+                              int32_t* d_info, void* ws, size_t ws_bytes,
+                              gptq_stream_t stream);
+
+/* Lazy-blocked GPTQ column sweep of one layer.
+ * [GPTQ-tool] Steps 5, 7 and 8, A minimal Python sketch; [What-is-GPTQ]
+ * Step 3 (groups); [GPTQ-breakdown] How It Works (lazy batching).
+ * Per block of B = cfg->block_size processing-order columns [s, e): at each
+ * group start the row's grid is taken from the current weights of the group
+ * (lo = min(0, min w), hi = max(0, max w), scale = max(hi-lo, 1e-8)/maxq,
+ * zero = rint(-lo/scale)); each column is coded c = clamp(rint(w/scale) +
+ * zero, 0, maxq) (fp32 decisions, ties to even), err = (w - q)/U[i,i] with
+ * q = scale*(c - zero), later in-block columns get w_j -= err*U[i,j], and at
+ * the block end W[:, e:] -= Err * U[s:e, e:].
+ *   W       (r, k) dtype `dt` (F32/F16/BF16), leading dimension ldw >= k,
+ *           ORIGINAL column order (read only).
+ *   U, perm, dead  as produced by gptq_prepare_hinv for this layer.
+ *   H0      (k, k) fp32 undamped Hessian for the layer loss, or NULL.
+ *   codes   uint8 (r, k) out, ORIGINAL column order.
+ *   scales  fp32 (r, ngroups) out, group index in processing order;
+ *           ngroups = ceil(k / group_size) (1 when group_size == -1).
+ *   zeros   int32 (r, ngroups) out.
+ *   g_idx   int32[k] out: group of each ORIGINAL column.
+ *   loss    fp64 device array of r+1 out (may be NULL; ignored when H0 is
+ *           NULL): loss[0..r-1] = per-row (w0-q) H0 (w0-q)^T, loss[r] = their
+ *           sum ([GPTQ-tool] Step 2 objective; Reading a quantization log).
+ *   d_status int32 device scalar out (may be NULL): 0, or GPTQ_ERR_NONFINITE
+ *           if a non-finite weight was met (its code is then the zero point).
+ *   ws      GPTQ_OP_QUANTIZE workspace (holds the fp32 working copy of W).
+ * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_UNSUPPORTED,
+ * GPTQ_ERR_WORKSPACE, GPTQ_ERR_CUDA. */
+GPTQ_API gptq_status gptq_quantize_layer(const void* W, gptq_dtype dt, int64_t r, int64_t k,
+                                int64_t ldw, const float* U, const int32_t* perm,
+                                const uint8_t* dead, const float* H0,
+                                const gptq_config* cfg, uint8_t* codes, float* scales,
+                                int32_t* zeros, int32_t* g_idx, double* loss,
+                                int32_t* d_status, void* ws, size_t ws_bytes,
+                                gptq_stream_t stream);
+
+/* Pack codes into 32-bit words ([GPTQ-tool] Step 8: eight 4-bit codes per
+ * 32-bit word).  Each row's codes form an LSB-first bit stream: code j
+ * occupies stream bits [j*bits, (j+1)*bits), stream bit m is bit m%32 of
+ * word m/32 (3-bit codes straddle words).
+ *   codes   uint8 (r, k), values < 2^bits (higher bits are masked off),
+ *           16-byte aligned.
+ *   qweight int32 (r, k*bits/32) out.  Needs k % 32 == 0 (then every row
+ *           is a whole number of 32-code runs of `bits` words each).
+ * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_UNSUPPORTED, GPTQ_ERR_CUDA. */
+GPTQ_API gptq_status gptq_pack(const uint8_t* codes, int64_t r, int64_t k, int bits, int32_t* qweight,
+                      gptq_stream_t stream);
+
+/* Dequantize packed codes: out[i, c] = scales[i, g] * (code - zeros[i, g]),
+ * g = g_idx[c] ([GPTQ-tool] sketch dequantization; [What-is-GPTQ] Step 3).
+ * The product is formed in fp32 and rounded to out_dt (F32/F16/BF16).
+ *   qweight int32 (r, k*bits/32); scales fp32 / zeros int32 (r, ngroups);
+ *   g_idx int32[k] with 0 <= g_idx[c] < ngroups; out (r, k) row-major.
+ *   Needs k % 32 == 0.
+ * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_UNSUPPORTED, GPTQ_ERR_CUDA. */
+GPTQ_API gptq_status gptq_dequant(const int32_t* qweight, const float* scales, const int32_t* zeros,
+                         const int32_t* g_idx, int64_t r, int64_t k, int bits,
+                         int64_t ngroups, gptq_dtype out_dt, void* out,
+                         gptq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_H */

@@ -101,12 +101,33 @@ def fix_dead_columns(H, W):
     return H, W, dead
 
 
-def act_order_perm(H):
+def act_order_perm(H, force_perm=None, tau_rel=1e-5):
     """[GPTQ-tool] *Optional refinements*, Act-order: process columns in
     descending order of the Hessian diagonal.  READING R3: stable, so equal
-    diagonal values keep ascending column index."""
+    diagonal values keep ascending column index.
+
+    The order is an integer result decided by floating-point values: two
+    diagonals that agree within the Hessian's tolerance may come out in
+    either order from an fp32 Hessian.  ``force_perm`` (a candidate order)
+    is accepted when it is a permutation whose every out-of-order pair lies
+    within ``tau_rel`` (relative) of a tie, i.e. d[perm[j]] >=
+    (1 - tau_rel) * max_{m > j} d[perm[m]] for all j; otherwise ValueError.
+    """
     d = np.diag(np.asarray(H, dtype=F64))
-    return np.argsort(-d, kind="stable").astype(np.int64)
+    if force_perm is None:
+        return np.argsort(-d, kind="stable").astype(np.int64)
+    p = np.asarray(force_perm, dtype=np.int64)
+    k = d.shape[0]
+    if p.shape != (k,) or not np.array_equal(np.sort(p), np.arange(k)):
+        raise ValueError("candidate order is not a permutation")
+    dp = d[p]
+    suffix_max = np.maximum.accumulate(dp[::-1])[::-1]
+    later = np.append(suffix_max[1:], -np.inf)
+    bad = dp < (1.0 - tau_rel) * later
+    if bad.any():
+        j = int(np.flatnonzero(bad)[0])
+        raise ValueError(f"candidate order breaks descending diag at position {j}")
+    return p
 
 
 def damp(H, percdamp):
@@ -446,7 +467,7 @@ def layer_loss(W0, qhat, H0):
 
 def gptq(W, H, bits=4, group_size=128, block_size=128, percdamp=0.01,
          act_order=False, include_zero=True, decide_dtype=F32, blocked=True,
-         force_codes=None, force_zeros=None, tau=1e-3):
+         force_codes=None, force_zeros=None, tau=1e-3, force_perm=None, tau_perm=1e-5):
     """GPTQ for one linear layer, given W (r, k) and the undamped Hessian H.
 
     Order of steps ([GPTQ-tool] *How it works* Steps 3-8): dead columns
@@ -457,13 +478,18 @@ def gptq(W, H, bits=4, group_size=128, block_size=128, percdamp=0.01,
     layer loss against the undamped H (READING R11).
 
     ``force_codes`` / ``force_zeros`` (original column order) request the
-    tie-aware replay (``sweep_replay``).
+    tie-aware replay (``sweep_replay``); ``force_perm`` a candidate act-order
+    permutation, accepted only where it is a valid order within ``tau_perm``
+    (see ``act_order_perm``).
     """
     W0 = np.asarray(W, dtype=F64)
     H0 = np.asarray(H, dtype=F64)
     r, k = W0.shape
     Hf, Wf, dead = fix_dead_columns(H0, W0)
-    perm = act_order_perm(Hf) if act_order else np.arange(k, dtype=np.int64)
+    if act_order:
+        perm = act_order_perm(Hf, force_perm, tau_perm)
+    else:
+        perm = np.arange(k, dtype=np.int64)
     Wp = Wf[:, perm]
     Hp = Hf[np.ix_(perm, perm)]
     Hd = damp(Hp, percdamp)

@@ -1,0 +1,47 @@
+// Shared device helpers for libgptq_b200 (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/gptq.h"
+
+#define GPTQ_CHECK_LAUNCH()                              \
+  do {                                                   \
+    cudaError_t e_ = cudaPeekAtLastError();              \
+    if (e_ != cudaSuccess) return GPTQ_ERR_CUDA;         \
+  } while (0)
+
+namespace gptq {
+
+constexpr int kWarp = 32;
+
+__host__ __device__ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+// The quantization decision of the grid: c = clamp(rint(w / scale) + zero, 0, maxq),
+// with an IEEE fp32 division and round-half-to-even, as the fp32 reference does.
+__device__ __forceinline__ float quant_code(float w, float scale, float zero, float maxq) {
+  float c = rintf(__fdiv_rn(w, scale)) + zero;
+  return fminf(fmaxf(c, 0.0f), maxq);
+}
+
+// Grid parameters of one group from its min and max:
+// lo = min(0, min), hi = max(0, max), scale = max(hi - lo, 1e-8) / maxq, zero = rint(-lo / scale).
+__device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, float& scale,
+                                                float& zero) {
+  float lo = fminf(mn, 0.0f), hi = fmaxf(mx, 0.0f);
+  scale = __fdiv_rn(fmaxf(__fsub_rn(hi, lo), 1e-8f), maxq);
+  zero = rintf(__fdiv_rn(-lo, scale));
+}
+
+}  // namespace gptq

@@ -380,6 +380,19 @@ def test_act_order_permutation_and_gidx():
     assert list(res2["g_idx"]) == [0, 0, 0, 0, 1, 1, 1, 1]
 
 
+def test_act_order_candidate_accepted_only_at_ties():
+    # a candidate order may swap columns whose diagonals agree within the
+    # tolerance, nothing else
+    d = np.array([1.0, 5.0, 5.0 * (1 + 1e-7), 2.0, 9.0])
+    H = np.diag(d)
+    assert list(O.act_order_perm(H)) == [4, 2, 1, 3, 0]
+    assert list(O.act_order_perm(H, [4, 1, 2, 3, 0], 1e-5)) == [4, 1, 2, 3, 0]
+    with pytest.raises(ValueError):
+        O.act_order_perm(H, [4, 1, 2, 0, 3], 1e-5)
+    with pytest.raises(ValueError):
+        O.act_order_perm(H, [4, 1, 1, 3, 0], 1e-5)
+
+
 # ---------------------------------------------------------------- the sketch
 
 def _sketch_in_my_words(W, X, bits, damp_frac):
