@@ -1,0 +1,455 @@
+"""GPTQ layer quantization throughput on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--config q_proj] [--no-e2e] [--no-cpu-baseline]
+
+A step is one pass of the whole hot path over one layer: Hessian
+accumulation over all calibration tokens, inverse factor (dead columns,
+damping, act-order if set), lazy-blocked sweep with the layer loss, pack and
+dequant.  The default workload is the Llama-7B-shaped q_proj layer: W 4096 x
+4096 fp16, X 262144 x 4096 fp16 (2.15 GB, larger than L2, so no flush is
+needed between steps), int4 asymmetric, group 128, block 128, damp 0.01.
+
+value  = weights quantized per second over all ranks (Mweights/s), inputs
+         resident in HBM, device time (CUDA events), max over ranks.
+e2e    = the same metric through the host-buffer API (pinned X and W copied in,
+         packed result and loss copied out, inside the timed region).
+N > 1  = weak scaling: every rank quantizes its own independent layer (a
+         different seed); no collective is on the data path.
+--impl reference runs the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only) and prints the same line with "impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "GPTQ layer quantize Mweights/s end-to-end"
+UNIT = "Mweights/s"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.lines = []
+        self.dev = str(device_index)
+        try:
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            if bus:
+                self.dev = bus
+        except Exception:
+            pass
+
+    def start(self):
+        """Start sampling every 100 ms; returns once the first sample is in."""
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.dev], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.first = self.proc.stdout.readline()
+        except Exception:
+            self.proc = None
+            self.first = ""
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        out = (self.first or "") + (out or "")
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(spec, seed, n_tokens, n_rows):
+    """Time the fp64 oracle on a bounded sample of the workload and
+    extrapolate to the whole layer: Hessian over ``n_tokens`` tokens (scaled by
+    n / n_tokens), the inverse factor at full k, the sweep, pack and dequant
+    over ``n_rows`` rows (scaled by r / n_rows)."""
+    import oracle as O
+    X = synth.make_x(spec, seed, t0=0, t1=n_tokens)
+    W = synth.make_w(spec, seed)[:n_rows]
+    Xn = X.float().numpy() if X.dtype == torch.bfloat16 else X.numpy()
+    Wn = W.float().numpy() if W.dtype == torch.bfloat16 else W.numpy()
+    t0 = time.perf_counter()
+    H = O.hessian(Xn, n_total=n_tokens)
+    t1 = time.perf_counter()
+    Hf, Wf, dead = O.fix_dead_columns(H, Wn)
+    perm = O.act_order_perm(Hf) if spec.act_order else np.arange(spec.k)
+    Hd = O.damp(Hf[np.ix_(perm, perm)], spec.percdamp)
+    U = O.hinv_upper_factor(Hd)
+    t2 = time.perf_counter()
+    res = O.sweep_blocked(Wf[:, perm], U, spec.bits, spec.group_size, spec.block_size)
+    codes = np.zeros_like(res["codes"], dtype=np.int64)
+    codes[:, perm] = res["codes"]
+    qhat = np.zeros_like(res["qhat"])
+    qhat[:, perm] = res["qhat"]
+    O.layer_loss(Wn, qhat, H)
+    t3 = time.perf_counter()
+    G = spec.k if spec.group_size == -1 else spec.group_size
+    g_idx = np.zeros(spec.k, dtype=np.int64)
+    g_idx[perm] = np.arange(spec.k) // G
+    qw = O.pack(codes, spec.bits)
+    O.dequant(O.unpack(qw, spec.k, spec.bits), res["scales"], res["zeros"], g_idx, np.float16)
+    t4 = time.perf_counter()
+    t_full = ((t1 - t0) * spec.n / n_tokens + (t2 - t1) + (t3 - t2) * spec.r / n_rows
+              + (t4 - t3) * spec.r / n_rows)
+    sample = (f"Hessian over {n_tokens} of {spec.n} tokens (x{spec.n / n_tokens:g}); inverse "
+              f"factor at full k={spec.k}; sweep+loss, pack, dequant over {n_rows} of {spec.r} rows "
+              f"(x{spec.r / n_rows:g}); phases {t1 - t0:.2f}/{t2 - t1:.2f}/{t3 - t2:.2f}/"
+              f"{t4 - t3:.2f} s")
+    return t_full, t4 - t0, sample
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def reference_arm(args, spec, world, rank):
+    if rank != 0:
+        return 0
+    n_tok, n_rows = args.ref_tokens, args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(spec, args.seed, n_tok, n_rows)
+    ts, wall, sample = [], 0.0, ""
+    for _ in range(args.steps):
+        t_full, w, sample = oracle_sample(spec, args.seed, n_tok, n_rows)
+        ts.append(t_full)
+        wall += w
+    t = statistics.median(ts)
+    value = spec.r * spec.k / t / 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(spec),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(spec):
+    G = "per-row" if spec.group_size == -1 else f"g{spec.group_size}"
+    return {
+        "workload": (f"{spec.name}: W {spec.r}x{spec.k} {spec.w_dtype}, X {spec.n}x{spec.k} "
+                     f"{spec.x_dtype} ({spec.x_kind}), int{spec.bits} asym {G} B{spec.block_size} "
+                     f"damp {spec.percdamp}{' act-order' if spec.act_order else ''}"),
+        "l2": f"inputs larger than L2 (X {spec.n * spec.k * 2 / 1e9:.2f} GB), no flush",
+    }
+
+
+# --------------------------------------------------------------------------- native arm
+
+def native_arm(args, spec, world, rank, local):
+    from post_weight_quantization_23_b200 import GptqPlan, QuantConfig
+    from post_weight_quantization_23_b200.api import HostPipeline
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    seed = args.seed + rank  # independent layer per rank (weak scaling)
+    cfg = QuantConfig(spec.bits, spec.group_size, spec.block_size, spec.percdamp, spec.act_order)
+    xdt = synth.dtype_of(spec.x_dtype)
+    X_host = torch.empty(spec.n, spec.k, dtype=xdt, pin_memory=True)
+    synth.make_x(spec, seed, out=X_host)
+    W_host = synth.make_w(spec, seed).pin_memory()
+    Xd = X_host.to(dev)
+    Wd = W_host.to(dev)
+    plan = GptqPlan(spec.r, spec.k, cfg, dev, want_loss=True, deq_dtype=torch.float16,
+                    hessian_tokens_hint=spec.n)
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+
+    def lib_calls():
+        plan.hessian_add(Xd, spec.n)
+        plan.prepare()
+        plan.quantize(Wd)
+        plan.pack()
+        plan.dequant()
+
+    def step(record=False):
+        if record:
+            ev[0].record(stream)
+        plan.hessian_reset()
+        plan.hessian_add(Xd, spec.n)
+        if record:
+            ev[1].record(stream)
+        plan.prepare()
+        if record:
+            ev[2].record(stream)
+        plan.quantize(Wd)
+        if record:
+            ev[3].record(stream)
+        plan.pack()
+        if record:
+            ev[4].record(stream)
+        plan.dequant()
+        if record:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    plan.check()
+
+    # per-phase device times (separate pass, events between phases)
+    phase = np.zeros(5)
+    n_phase = max(2, min(args.steps, 5))
+    for _ in range(n_phase):
+        step(record=True)
+        torch.cuda.synchronize(dev)
+        phase += [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
+    phase /= n_phase
+
+    launches = count_launches(lib_calls, dev)  # the H reset is a torch memset, not ours
+    plan.check()
+
+    clocks = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    plan.check()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    ms = max_over_ranks(ms, world)
+    value = world * spec.r * spec.k / (ms / 1e3) / 1e6
+
+    e2e = None
+    if not args.no_e2e:
+        pipe = HostPipeline(plan, args.e2e_chunk, xdt, W_host.dtype)
+        for _ in range(2):
+            pipe.run(X_host, W_host)
+            pipe.wait()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        k_e2e = max(1, min(args.steps, args.e2e_steps))
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(k_e2e):
+            pipe.run(X_host, W_host)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        pipe.wait()
+        barrier(world)
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / k_e2e, world)
+        e2e = {"value": world * spec.r * spec.k / (ms_e2e / 1e3) / 1e6, "unit": UNIT,
+               "ms_per_step": ms_e2e, "steps": k_e2e,
+               "h2d_bytes_per_step": pipe.h2d_bytes(X_host, W_host),
+               "d2h_bytes_per_step": pipe.d2h_bytes()}
+
+    peaks = _peaks()
+    flops = float(spec.n) * spec.k * (spec.k + 1)  # symmetric triangle, algorithmic
+    t_h = phase[0] / 1e3
+    achieved = flops / t_h / 1e12
+    roofline = {"bound": "tensor", "kernel": "gptq_hessian_accumulate (X^T X)",
+                "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_sustained"], "traffic": args.traffic,
+                "peak_kind": f"bf16 dense sustained ({peaks['source']}); f16 has the same nominal rate",
+                "algorithmic": f"n*k*(k+1) = {flops:.4g} flop per launch"}
+    sweep_bytes = sweep_model_bytes(spec)
+    phases = {
+        "hessian_ms": phase[0], "prepare_ms": phase[1], "quantize_ms": phase[2],
+        "pack_ms": phase[3], "dequant_ms": phase[4],
+        "hessian_tflops": achieved,
+        "hessian_x_gbs": spec.n * spec.k * 2 / t_h / 1e9,
+        "sweep_model_gbs": sweep_bytes / (phase[2] / 1e3) / 1e9,
+        "sweep_frac_hbm": sweep_bytes / (phase[2] / 1e3) / 1e9 / peaks["hbm"],
+    }
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": dict(workload_config(spec), parallelism=f"{world} independent layers"),
+        "roofline": roofline, "phases": phases,
+        "gpu_launches": launches * args.steps if launches is not None else None,
+        "gpu_launches_per_step": launches, "clocks": clk, "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_full, wall, sample = oracle_sample(spec, args.seed, args.ref_tokens, args.ref_rows)
+        line["cpu_baseline"] = {"value": spec.r * spec.k / t_full / 1e6, "unit": UNIT,
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": sample + f"; wall {wall:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def sweep_model_bytes(spec):
+    """Algorithmic bytes of the lazy-blocked sweep: per block the trailing fp32
+    slice of W in and out (8 r (k-e)), the U panel (4 B (k-e)), plus the W
+    read (input dtype), the fp32 working copy in and out, the error block, and
+    the codes written."""
+    r, k, B = spec.r, spec.k, spec.block_size
+    nb = -(-k // B)
+    sigma = sum(k - min((b + 1) * B, k) for b in range(nb))
+    wbytes = 2 if spec.w_dtype in ("f16", "bf16") else 4
+    return 8 * r * sigma + 4 * B * sigma + 16 * r * k + r * k + wbytes * r * k
+
+
+def count_launches(step, dev):
+    """Kernel launches of one step, counted from a CUDA-graph capture of it."""
+    try:
+        from cuda.bindings import runtime as cudart
+    except Exception:
+        try:
+            from cuda import cudart  # type: ignore
+        except Exception:
+            return None
+    try:
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+    except TypeError:
+        g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        g.capture_begin()
+        step()
+        g.capture_end()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    try:
+        raw = g.raw_cuda_graph()
+        handle = raw if isinstance(raw, cudart.cudaGraph_t) else cudart.cudaGraph_t(int(raw))
+        err, nodes, num = cudart.cudaGraphGetNodes(handle, 0)
+        err, nodes, num = cudart.cudaGraphGetNodes(handle, num)
+        n = 0
+        for nd in nodes:
+            err, ty = cudart.cudaGraphNodeGetType(nd)
+            if ty == cudart.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                n += 1
+        return n
+    except Exception as e:  # report, but do not fail the bench over the count
+        print(f"launch count unavailable: {e!r}", file=sys.stderr)
+        return None
+    finally:
+        del g
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--config", default="q_proj", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-chunk", type=int, default=32768)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=8192)
+    ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per Hessian launch from an ncu capture of this kernel")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    spec = synth.CONFIGS[args.config]
+    if args.impl == "reference":
+        # CPU only: rank 0 runs the oracle, other ranks exit without work
+        return reference_arm(args, spec, int(os.environ.get("WORLD_SIZE", "1")),
+                             int(os.environ.get("RANK", "0")))
+    world, rank, local = dist_setup(args)
+    try:
+        return native_arm(args, spec, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -152,3 +152,79 @@ def quantize_layer(W: torch.Tensor, X=None, cfg: QuantConfig | None = None, H=No
     plan.run_after_hessian(W)
     plan.check()
     return plan.result()
+
+
+class HostPipeline:
+    """End-to-end layer quantization from HOST buffers (pinned memory):
+    X is streamed to the device in chunks on a copy stream while the Hessian
+    accumulates the previous chunk on the compute stream (two device staging
+    buffers, event-ordered), W is copied once, and the packed result (qweight,
+    scales, zeros, g_idx) plus the layer loss are copied back to pinned host
+    buffers.  ``run`` enqueues everything and returns; ``wait`` synchronises."""
+
+    def __init__(self, plan: GptqPlan, chunk_tokens: int, x_dtype: torch.dtype,
+                 w_dtype: torch.dtype):
+        self.plan = plan
+        self.chunk = int(chunk_tokens)
+        dev = plan.device
+        self.stage = [torch.empty(self.chunk, plan.k, dtype=x_dtype, device=dev) for _ in range(2)]
+        self.Wd = torch.empty(plan.r, plan.k, dtype=w_dtype, device=dev)
+        self.copy_stream = torch.cuda.Stream(dev)
+        self.compute_stream = torch.cuda.Stream(dev)
+        self.copied = [torch.cuda.Event() for _ in range(2)]
+        self.consumed = [torch.cuda.Event() for _ in range(2)]
+        pin = dict(pin_memory=True)
+        self.out_qweight = torch.empty(plan.qweight.shape, dtype=plan.qweight.dtype, **pin)
+        self.out_scales = torch.empty(plan.scales.shape, dtype=plan.scales.dtype, **pin)
+        self.out_zeros = torch.empty(plan.zeros.shape, dtype=plan.zeros.dtype, **pin)
+        self.out_gidx = torch.empty(plan.g_idx.shape, dtype=plan.g_idx.dtype, **pin)
+        self.out_loss = torch.empty(1, dtype=torch.float64, **pin)
+        self.out_status = torch.empty(2, dtype=torch.int32, **pin)
+
+    def h2d_bytes(self, X_host, W_host) -> int:
+        return X_host.numel() * X_host.element_size() + W_host.numel() * W_host.element_size()
+
+    def d2h_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (
+            self.out_qweight, self.out_scales, self.out_zeros, self.out_gidx, self.out_loss,
+            self.out_status))
+
+    def run(self, X_host: torch.Tensor, W_host: torch.Tensor):
+        plan, cs, ks = self.plan, self.copy_stream, self.compute_stream
+        n = X_host.shape[0]
+        ks.wait_stream(torch.cuda.current_stream(plan.device))
+        cs.wait_stream(ks)  # staging buffers and Wd are free once the last run's compute is done
+        with torch.cuda.stream(ks):
+            plan.hessian_reset()
+        with torch.cuda.stream(cs):
+            self.Wd.copy_(W_host, non_blocking=True)
+        for i, a in enumerate(range(0, n, self.chunk)):
+            b = i % 2
+            rows = min(self.chunk, n - a)
+            with torch.cuda.stream(cs):
+                if i >= 2:
+                    cs.wait_event(self.consumed[b])
+                self.stage[b][:rows].copy_(X_host[a:a + rows], non_blocking=True)
+                self.copied[b].record(cs)
+            ks.wait_event(self.copied[b])
+            plan.hessian_add(self.stage[b][:rows], n, stream=ks)
+            self.consumed[b].record(ks)
+        ks.wait_stream(cs)
+        plan.run_after_hessian(self.Wd, stream=ks)
+        with torch.cuda.stream(ks):
+            self.out_qweight.copy_(plan.qweight, non_blocking=True)
+            self.out_scales.copy_(plan.scales, non_blocking=True)
+            self.out_zeros.copy_(plan.zeros, non_blocking=True)
+            self.out_gidx.copy_(plan.g_idx, non_blocking=True)
+            if plan.loss is not None:
+                self.out_loss.copy_(plan.loss[-1:], non_blocking=True)
+            self.out_status[0:1].copy_(plan.d_info, non_blocking=True)
+            self.out_status[1:2].copy_(plan.d_status, non_blocking=True)
+        torch.cuda.current_stream(plan.device).wait_stream(ks)
+
+    def wait(self):
+        self.compute_stream.synchronize()
+        if int(self.out_status[0]) != 0:
+            raise NotPositiveDefinite(_lib.GPTQ_ERR_NOT_PD, "gptq_prepare_hinv")
+        if int(self.out_status[1]) != 0:
+            raise GptqError(int(self.out_status[1]), "gptq_quantize_layer")

@@ -78,10 +78,16 @@ hessian_simt_kernel(const T* __restrict__ X, int64_t n, int k, int64_t ldx, floa
   }
 }
 
-// H[j][i] = H[i][j] for j > i.
-__global__ void mirror_upper_kernel(float* __restrict__ H, int k) {
+// H[j][i] = H[i][j] for j > i.  A nonzero *poison_flag (a device-side wait
+// of the tensor-core pass gave up) writes NaN into H[0][0] instead, so the
+// Cholesky of the next stage reports the failure.
+__global__ void mirror_upper_kernel(float* __restrict__ H, int k, const int32_t* poison_flag) {
   __shared__ float tile[32][33];
   int bi = blockIdx.y, bj = blockIdx.x;
+  if (poison_flag != nullptr && *poison_flag != 0) {
+    if (bi == 0 && bj == 0 && threadIdx.x == 0 && threadIdx.y == 0) H[0] = __int_as_float(0x7fc00000);
+    return;
+  }
   if (bj < bi) return;
   int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
   for (int r = ty; r < 32; r += 8) {
@@ -119,7 +125,7 @@ gptq_status hessian_simt(const void* X, gptq_dtype dt, int64_t n, int64_t k, int
   }
   GPTQ_CHECK_LAUNCH();
   int nb = (int)cdiv(k, 32);
-  mirror_upper_kernel<<<dim3(nb, nb), dim3(32, 8), 0, s>>>(H, (int)k);
+  mirror_upper_kernel<<<dim3(nb, nb), dim3(32, 8), 0, s>>>(H, (int)k, nullptr);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
 }

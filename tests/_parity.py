@@ -68,10 +68,12 @@ class Agreement:
         assert self.loss_rel <= TOL_LOSS_REL, self
 
 
-def compare(gpu, W_np, X_np, cfg, rows=None):
+def compare(gpu, W_np, X_np, cfg, rows=None, H=None):
     """Oracle on the same inputs; ``rows`` restricts the sweep comparison to a
-    sample of rows (rows are independent given U)."""
-    H = O.hessian(X_np)
+    sample of rows (rows are independent given U).  ``H`` may carry the
+    oracle's own Hessian of X when it was computed in chunks beforehand."""
+    if H is None:
+        H = O.hessian(X_np)
     Hg = gpu["H"].double().numpy()
     h_rel = float(np.linalg.norm(Hg - H) / np.linalg.norm(H))
     Wc = W_np if rows is None else W_np[rows]
