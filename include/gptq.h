@@ -141,6 +141,31 @@ GPTQ_API gptq_status gptq_prepare_hinv(const float* H, int64_t k, const gptq_con
                               int32_t* d_info, void* ws, size_t ws_bytes,
                               gptq_stream_t stream);
 
+/* gptq_prepare_hinv without a workspace, for callers that cannot allocate
+ * device memory (the pages have no counterpart: this is an interface
+ * convenience, not part of the method).
+ * Some callers cannot call cudaMalloc or hand over a workspace: a plugin
+ * whose host passes it only its input and output buffers, a process that has
+ * carved all device memory into its own arena, or a runtime that forbids
+ * allocation after start-up.  This call computes exactly what
+ * gptq_prepare_hinv computes (same arguments minus ws / ws_bytes) with its
+ * scratch in a 4 MiB array of the library's device code, which every device
+ * that loads the library holds until the process exits.
+ *   k        1 .. 12288; a larger k returns GPTQ_ERR_WORKSPACE (the built-in
+ *            scratch is too small) before anything is enqueued.
+ *   Setup.   The first call on a device, with that device current, looks up
+ *            the array's device address (cudaGetSymbolAddress); make that
+ *            first call before any stream capture.
+ *   Sharing. All calls share the array and it keeps the last call's
+ *            contents (every word is written before it is read, nothing needs
+ *            clearing).  Calls whose work overlaps on the GPU (other streams,
+ *            other host threads) race on it: serialise them.
+ * Returns as gptq_prepare_hinv, with GPTQ_ERR_WORKSPACE for k > 12288. */
+GPTQ_API gptq_status gptq_prepare_hinv_noalloc(const float* H, int64_t k, const gptq_config* cfg,
+                                               float* U, int32_t* perm, int32_t* invperm,
+                                               uint8_t* dead, int32_t* d_info,
+                                               gptq_stream_t stream);
+
 /* Lazy-blocked GPTQ column sweep of one layer.
  * [GPTQ-tool] Steps 5, 7 and 8, A minimal Python sketch; [What-is-GPTQ]
  * Step 3 (groups); [GPTQ-breakdown] How It Works (lazy batching).

@@ -34,6 +34,7 @@ EXPORTED = (
     "gptq_status_string",
     "gptq_hessian_accumulate",
     "gptq_prepare_hinv",
+    "gptq_prepare_hinv_noalloc",
     "gptq_quantize_layer",
     "gptq_pack",
     "gptq_dequant",
@@ -91,6 +92,8 @@ def load(path: str = LIB_PATH):
     lib.gptq_hessian_accumulate.argtypes = [vp, i32, i64, i64, i64, ctypes.c_float, vp, vp, sz, vp]
     lib.gptq_prepare_hinv.restype = i32
     lib.gptq_prepare_hinv.argtypes = [vp, i64, cfgp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gptq_prepare_hinv_noalloc.restype = i32
+    lib.gptq_prepare_hinv_noalloc.argtypes = [vp, i64, cfgp, vp, vp, vp, vp, vp, vp]
     lib.gptq_quantize_layer.restype = i32
     lib.gptq_quantize_layer.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, cfgp, vp, vp, vp,
                                         vp, vp, vp, vp, sz, vp]
@@ -155,6 +158,15 @@ def prepare_hinv(H, cfg, U, perm, invperm, dead, d_info, ws, stream=None):
                                   _ptr(dead), _ptr(d_info), _ptr(ws), ws.numel() * ws.element_size(),
                                   _stream(stream))
     _check(st, "gptq_prepare_hinv")
+
+
+def prepare_hinv_noalloc(H, cfg, U, perm, invperm, dead, d_info, stream=None):
+    """gptq_prepare_hinv without a workspace (scratch in the library's own
+    device array; see include/gptq.h)."""
+    k = H.shape[0]
+    st = load().gptq_prepare_hinv_noalloc(_ptr(H), k, ctypes.byref(cfg), _ptr(U), _ptr(perm),
+                                          _ptr(invperm), _ptr(dead), _ptr(d_info), _stream(stream))
+    _check(st, "gptq_prepare_hinv_noalloc")
 
 
 def quantize_layer(W, U, perm, dead, H0, cfg, codes, scales, zeros, g_idx, loss, d_status, ws,
