@@ -433,12 +433,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=8192)
     ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the calibration token count (smaller cases for profiling)")
+    ap.add_argument("--rows", type=int, default=None, help="override the row count of W")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per Hessian launch from an ncu capture of this kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     spec = synth.CONFIGS[args.config]
+    if args.tokens or args.rows:
+        spec = spec.scaled(r=args.rows, n=args.tokens)
     if args.impl == "reference":
         # CPU only: rank 0 runs the oracle, other ranks exit without work
         return reference_arm(args, spec, int(os.environ.get("WORLD_SIZE", "1")),
