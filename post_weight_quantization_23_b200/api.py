@@ -109,6 +109,26 @@ class GptqPlan:
         self.pack(stream)
         self.dequant(stream)
 
+    def capture(self, fn) -> "torch.cuda.CUDAGraph":
+        """Record the library calls that ``fn()`` issues (with this plan's
+        fixed buffers) into a CUDA graph; ``graph.replay()`` then re-runs them
+        without per-kernel launch cost.  Inputs must stay at the same
+        addresses between replays (copy new data into them)."""
+        dev = self.device
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            fn()  # first calls on a stream outside capture: lazy set-up happens here
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize(dev)
+        try:
+            g = torch.cuda.CUDAGraph(keep_graph=True)
+        except TypeError:
+            g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+        return g
+
     def check(self):
         """Synchronise and raise on a device-reported failure."""
         torch.cuda.synchronize(self.device)

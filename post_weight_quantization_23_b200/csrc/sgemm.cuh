@@ -1,11 +1,13 @@
 // FP32 CUDA-core GEMM used by the inverse-factor and loss stages:
-//   C = beta * C + alpha * A * op(B)
-// A row-major (M x K, lda); B row-major (K x N, ldb), or, with TRANS_B, the
-// transpose of a row-major (N x K) matrix.  TRI_A: A is upper triangular
-// (A[i][m] == 0 for m < i), so a row tile's K loop starts at its first row.
-// UPPER_ONLY: tiles that lie entirely below the diagonal are skipped (the
-// caller only reads C's upper triangle).  A nonzero *abort_flag (device)
-// makes every CTA return at once; it carries an earlier stage's failure.
+//   C = beta * C + alpha * op(A) * op(B)
+// A row-major (M x K, lda), or with TRANS_A the transpose of a row-major
+// (K x M) matrix; B row-major (K x N, ldb), or with TRANS_B the transpose of a
+// row-major (N x K) matrix.  TRI_A: only the upper triangle of op(A) is used
+// (entries below the diagonal are read as 0, whatever memory holds there), so
+// a row tile's K loop starts at its first row.  TRI_B: only the upper triangle
+// of op(B) is used, so a column tile's K loop ends at its last column.  UPPER_ONLY: tiles that lie entirely below the diagonal are
+// skipped (the caller only reads C's upper triangle).  A nonzero *abort_flag
+// (device) makes every CTA return at once; it carries an earlier failure.
 #pragma once
 
 #include "common.cuh"
@@ -14,7 +16,7 @@ namespace gptq {
 
 constexpr int SG_BM = 128, SG_BN = 128, SG_BK = 8, SG_THREADS = 256;
 
-template <bool TRANS_B, bool TRI_A, bool UPPER_ONLY>
+template <bool TRANS_A, bool TRANS_B, bool TRI_A, bool TRI_B, bool UPPER_ONLY>
 __global__ void __launch_bounds__(SG_THREADS)
 sgemm_kernel(int M, int N, int K, float alpha, const float* __restrict__ A, int64_t lda,
              const float* __restrict__ B, int64_t ldb, float beta, float* __restrict__ C,
@@ -35,6 +37,7 @@ sgemm_kernel(int M, int N, int K, float alpha, const float* __restrict__ A, int6
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
   const int kbeg = TRI_A ? (m0 / SG_BK) * SG_BK : 0;
+  const int kend = TRI_B ? min(K, n0 + SG_BN) : K;
   // A tile: 128 rows x 8 k; thread loads rows (tid/2) and k (tid%2)*4 .. +3
   const int a_row = tid / 2, a_k = (tid % 2) * 4;
   // B tile (no trans): 8 k x 128 n; thread loads k = tid/32, n = (tid%32)*4 .. +3
@@ -42,30 +45,50 @@ sgemm_kernel(int M, int N, int K, float alpha, const float* __restrict__ A, int6
   float ra[4], rb[4];
 
   auto load_tile = [&](int k0) {
+    if (!TRANS_A) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      int gm = m0 + a_row, gk = k0 + a_k + q;
-      ra[q] = (gm < M && gk < K) ? A[(int64_t)gm * lda + gk] : 0.f;
+      for (int q = 0; q < 4; ++q) {
+        int gm = m0 + a_row, gk = k0 + a_k + q;
+        bool ok = gm < M && gk < kend && (!TRI_A || gk >= gm);
+        ra[q] = ok ? A[(int64_t)gm * lda + gk] : 0.f;
+      }
+    } else {
+      // element (m, kk) = A[kk * lda + m]: thread loads kk = tid / 32, m = (tid % 32) * 4 .. +3
+      int kk = tid / 32, mm = (tid % 32) * 4;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        int gk = k0 + kk, gm = m0 + mm + q;
+        bool ok = gk < kend && gm < M && (!TRI_A || gk >= gm);
+        ra[q] = ok ? A[(int64_t)gk * lda + gm] : 0.f;
+      }
     }
     if (!TRANS_B) {
       int kk = tid / 32, nn = (tid % 32) * 4;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         int gk = k0 + kk, gn = n0 + nn + q;
-        rb[q] = (gk < K && gn < N) ? B[(int64_t)gk * ldb + gn] : 0.f;
+        bool ok = gk < kend && gn < N && (!TRI_B || gk <= gn);
+        rb[q] = ok ? B[(int64_t)gk * ldb + gn] : 0.f;
       }
     } else {
       int nn = tid / 2, kk = (tid % 2) * 4;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         int gk = k0 + kk + q, gn = n0 + nn;
-        rb[q] = (gk < K && gn < N) ? B[(int64_t)gn * ldb + gk] : 0.f;
+        bool ok = gk < kend && gn < N && (!TRI_B || gk <= gn);
+        rb[q] = ok ? B[(int64_t)gn * ldb + gk] : 0.f;
       }
     }
   };
   auto store_tile = [&](int buf) {
+    if (!TRANS_A) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) sA[buf][a_k + q][a_row] = ra[q];
+      for (int q = 0; q < 4; ++q) sA[buf][a_k + q][a_row] = ra[q];
+    } else {
+      int kk = tid / 32, mm = (tid % 32) * 4;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sA[buf][kk][mm + q] = ra[q];
+    }
     if (!TRANS_B) {
       int kk = tid / 32, nn = (tid % 32) * 4;
 #pragma unroll
@@ -78,13 +101,13 @@ sgemm_kernel(int M, int N, int K, float alpha, const float* __restrict__ A, int6
   };
 
   int buf = 0;
-  if (kbeg < K) {
+  if (kbeg < kend) {
     load_tile(kbeg);
     store_tile(0);
   }
   __syncthreads();
-  for (int k0 = kbeg; k0 < K; k0 += SG_BK) {
-    const bool more = k0 + SG_BK < K;
+  for (int k0 = kbeg; k0 < kend; k0 += SG_BK) {
+    const bool more = k0 + SG_BK < kend;
     if (more) load_tile(k0 + SG_BK);
 #pragma unroll
     for (int kk = 0; kk < SG_BK; ++kk) {
@@ -121,13 +144,13 @@ sgemm_kernel(int M, int N, int K, float alpha, const float* __restrict__ A, int6
   }
 }
 
-template <bool TRANS_B, bool TRI_A, bool UPPER_ONLY>
+template <bool TRANS_A, bool TRANS_B, bool TRI_A, bool TRI_B, bool UPPER_ONLY>
 inline void sgemm(int M, int N, int K, float alpha, const float* A, int64_t lda, const float* B,
                   int64_t ldb, float beta, float* C, int64_t ldc, const int32_t* abort_flag,
                   cudaStream_t s) {
   if (M <= 0 || N <= 0) return;
   dim3 grid((unsigned)cdiv(N, SG_BN), (unsigned)cdiv(M, SG_BM));
-  sgemm_kernel<TRANS_B, TRI_A, UPPER_ONLY>
+  sgemm_kernel<TRANS_A, TRANS_B, TRI_A, TRI_B, UPPER_ONLY>
       <<<grid, SG_THREADS, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, abort_flag);
 }
 

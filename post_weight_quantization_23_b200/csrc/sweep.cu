@@ -211,14 +211,14 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     GPTQ_CHECK_LAUNCH();
     int e0 = s0 + bw;
     if (e0 < k) {
-      sgemm<false, false, false>(r, k - e0, bw, -1.0f, sc.Err, B, U + (int64_t)s0 * k + e0, k,
+      sgemm<false, false, false, false, false>(r, k - e0, bw, -1.0f, sc.Err, B, U + (int64_t)s0 * k + e0, k,
                                  1.0f, sc.Wt + e0, k, nullptr, s);
       GPTQ_CHECK_LAUNCH();
     }
   }
   if (want_loss) {
     // Y = D * H0 into the (now free) working copy, then per-row dot with D.
-    sgemm<false, false, false>(r, k, k, 1.0f, sc.D, k, H0, k, 0.0f, sc.Wt, k, nullptr, s);
+    sgemm<false, false, false, false, false>(r, k, k, 1.0f, sc.D, k, H0, k, 0.0f, sc.Wt, k, nullptr, s);
     GPTQ_CHECK_LAUNCH();
     rowdot_kernel<<<(unsigned)cdiv((int64_t)r * kWarp, 256), 256, 0, s>>>(sc.Wt, sc.D, r, k, loss);
     GPTQ_CHECK_LAUNCH();
