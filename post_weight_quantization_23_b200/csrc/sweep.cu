@@ -5,10 +5,18 @@
 // sequential over columns.  Per lazy block [s, e) of processing-order columns:
 //   (group kernel)  when a group starts at s and is wider than the block, its
 //                   per-row grid comes from the row's current weights;
-//   (block kernel)  one lane per row, the block's slice of the row in shared
-//                   memory: group grids that start inside the block, codes,
-//                   err = (w - q) / U[i][i], in-block compensation, Err out;
+//   (block kernel)  four threads per row: the block's slice of 32 rows and the
+//                   block's U tile (transposed) sit in shared memory; columns
+//                   are taken in sub-blocks of SB held in registers (in-sub-
+//                   block compensation immediately), and the remaining columns
+//                   of the block get the sub-block's errors as one rank-SB
+//                   update, each thread of the row taking every fourth column;
 //   (trailing)      W[:, e:] -= Err * U[s:e, e:]  (fp32 GEMM).
+// The layer loss is accumulated inside the block kernel through the Optimal
+// Brain Surgeon accounting: fixing column i and compensating the later ones
+// raises (w - q) Hd (w - q)^T by err_i^2, so per row
+//   (w0 - q) H0 (w0 - q)^T = sum_i err_i^2 - lambda * sum_i (w0_i - q_i)^2
+// (H0 = Hd - lambda I, dead columns count with w0 = 0); no k x k product.
 // The fp32 working copy Wt (processing order) lives in the workspace.
 #include "common.cuh"
 #include "sgemm.cuh"
@@ -16,16 +24,22 @@
 namespace gptq {
 
 constexpr int SW_MAX_B = 128;
+constexpr int SW_ROWS = 32;           // rows per CTA (4 warps x 8 rows)
+constexpr int SW_THREADS = 128;
+constexpr int SW_LDW = 40;            // sW column stride: 32 rows + 8 pad (conflict-free quads)
+constexpr int SW_LDU = SW_MAX_B + 4;  // UtS column stride
+constexpr size_t SW_SMEM = sizeof(float) * ((size_t)SW_MAX_B * SW_LDU + (size_t)SW_MAX_B * SW_LDW +
+                                            SW_MAX_B);
 
 struct SweepScratch {
-  float* Wt;   // [r * k] working weights, processing order
-  float* Err;  // [r * B]
-  float* D;    // [r * k] w0 - q in original order (loss)
+  float* Wt;      // [r * k] working weights, processing order
+  float* Err;     // [r * B]
+  float* lambda;  // [1] damping added to the Hessian diagonal (for the loss)
 };
 
 size_t sweep_workspace_bytes(int64_t r, int64_t k, int B) {
   return align256(sizeof(float) * (size_t)r * k) + align256(sizeof(float) * (size_t)r * B) +
-         align256(sizeof(float) * (size_t)r * k);
+         align256(sizeof(float));
 }
 
 static SweepScratch carve_sweep(void* ws, int64_t r, int64_t k, int B) {
@@ -33,16 +47,16 @@ static SweepScratch carve_sweep(void* ws, int64_t r, int64_t k, int B) {
   SweepScratch s;
   s.Wt = (float*)p; p += align256(sizeof(float) * (size_t)r * k);
   s.Err = (float*)p; p += align256(sizeof(float) * (size_t)r * B);
-  s.D = (float*)p;
+  s.lambda = (float*)p;
   return s;
 }
 
-// Wt[row][j] = dead[perm[j]] ? 0 : W[row][perm[j]];  g_idx[perm[j]] = j / G.
 template <typename T>
 __global__ void sweep_init_kernel(const T* __restrict__ W, int64_t ldw, int r, int k,
                                   const int32_t* __restrict__ perm,
                                   const uint8_t* __restrict__ dead, int G, float* __restrict__ Wt,
-                                  int32_t* __restrict__ g_idx, int32_t* __restrict__ d_status) {
+                                  int32_t* __restrict__ g_idx, double* __restrict__ loss,
+                                  int32_t* __restrict__ d_status) {
   int row = blockIdx.y;
   for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < k; j += gridDim.x * blockDim.x) {
     int c = perm[j];
@@ -50,7 +64,33 @@ __global__ void sweep_init_kernel(const T* __restrict__ W, int64_t ldw, int r, i
     Wt[(int64_t)row * k + j] = v;
     if (row == 0) g_idx[c] = j / G;
   }
-  if (row == 0 && blockIdx.x == 0 && threadIdx.x == 0 && d_status != nullptr) *d_status = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (loss != nullptr) {
+      loss[row] = 0.0;
+      if (row == 0) loss[r] = 0.0;
+    }
+    if (row == 0 && d_status != nullptr) *d_status = 0;
+  }
+}
+
+// lambda = percdamp * mean(diag H0), dead diagonal entries (0) counted as 1,
+// exactly as the inverse factor damped the Hessian.  One CTA.
+__global__ void sweep_lambda_kernel(const float* __restrict__ H0, int k, float percdamp,
+                                    float* __restrict__ lambda) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    float d = H0[(int64_t)i * k + i];
+    acc += (double)(d == 0.0f ? 1.0f : d);
+  }
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double sm = 0.0;
+    for (int w = 0; w < (int)(blockDim.x / 32); ++w) sm += red[w];
+    *lambda = (float)((double)percdamp * (sm / (double)k));
+  }
 }
 
 // Per-row grid of a group [s, s+gw) wider than the lazy block: one warp per row.
@@ -79,91 +119,132 @@ __global__ void group_grid_kernel(const float* __restrict__ Wt, int r, int k, in
   }
 }
 
-// One lazy block for 32 rows (one warp per CTA).
-template <typename T>
-__global__ void __launch_bounds__(32)
-sweep_block_kernel(float* __restrict__ Wt, float* __restrict__ Err, const float* __restrict__ U,
-                   const int32_t* __restrict__ perm, const T* __restrict__ W0, int64_t ldw, int r,
+// One lazy block [s, s + bw) for 32 rows.  Thread (rr = row in CTA, q = lane
+// % 4): all four threads of a row run the column chain (identical values, so
+// SIMT issues it once); the rank-SB updates of the rest of the block and the
+// outputs are split by q.  SB divides the group size when groups are smaller
+// than the block, so a group always starts at a sub-block boundary.
+template <int SB, typename T>
+__global__ void __launch_bounds__(SW_THREADS)
+sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
+                   const float* __restrict__ U, const int32_t* __restrict__ perm,
+                   const uint8_t* __restrict__ dead, const T* __restrict__ W0, int64_t ldw, int r,
                    int k, int s, int bw, int B, int G, int ngroups, float maxq,
-                   float* __restrict__ scales, int32_t* __restrict__ zeros,
-                   uint8_t* __restrict__ codes, float* __restrict__ D,
-                   int32_t* __restrict__ d_status) {
-  __shared__ float sW[SW_MAX_B][33];
-  __shared__ float sE[SW_MAX_B][33];
-  const int lane = threadIdx.x;
-  const int r0 = blockIdx.x * 32;
-  const int row = r0 + lane;
+                   const float* __restrict__ lambda, float* __restrict__ scales,
+                   int32_t* __restrict__ zeros, uint8_t* __restrict__ codes,
+                   double* __restrict__ loss, int32_t* __restrict__ d_status) {
+  extern __shared__ float sm_sweep[];
+  float* UtS = sm_sweep;                           // UtS[j * LDU + i] = U[s+i][s+j], i <= j
+  float* sW = UtS + SW_MAX_B * SW_LDU;             // sW[j * LDW + rr] = W[r0+rr][s+j]
+  float* rdg = sW + SW_MAX_B * SW_LDW;             // 1 / U[s+i][s+i]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q = lane & 3;
+  const int rr = warp * 8 + (lane >> 2);
+  const int r0 = blockIdx.x * SW_ROWS;
+  const int row = r0 + rr;
   const bool valid = row < r;
-  // cooperative, row-contiguous load of the block slice
-  for (int rr = 0; rr < 32; ++rr) {
-    int gr = r0 + rr;
-    for (int j = lane; j < bw; j += 32) sW[j][rr] = (gr < r) ? Wt[(int64_t)gr * k + s + j] : 0.f;
+  for (int e = tid; e < bw * bw; e += SW_THREADS) {
+    const int i = e / bw, j = e % bw;
+    UtS[j * SW_LDU + i] = (j >= i) ? U[(int64_t)(s + i) * k + s + j] : 0.f;
   }
-  __syncwarp();
+  for (int e = tid; e < SW_ROWS * bw; e += SW_THREADS) {
+    const int r2 = e / bw, j = e % bw;
+    const int gr = r0 + r2;
+    sW[j * SW_LDW + r2] = (gr < r) ? Wt[(int64_t)gr * k + s + j] : 0.f;
+  }
+  for (int i = tid; i < bw; i += SW_THREADS) rdg[i] = 1.0f / U[(int64_t)(s + i) * k + s + i];
+  __syncthreads();
+
   float scale = 1.f, zero = 0.f;
-  bool nonfinite = false;
-  if (G > B) {  // group started at or before s and spans the block
-    int g = s / G;
-    if (valid) {
-      scale = scales[(int64_t)row * ngroups + g];
-      zero = (float)zeros[(int64_t)row * ngroups + g];
-    }
+  if (G > B && valid) {  // the group started at or before s and spans the block
+    const int g = s / G;
+    scale = scales[(int64_t)row * ngroups + g];
+    zero = (float)zeros[(int64_t)row * ngroups + g];
   }
-  for (int i = 0; i < bw; ++i) {
-    const int gi = s + i;
-    if (G <= B && gi % G == 0) {
-      int gw = min(G, bw - i);
+  const float lam = (lambda != nullptr) ? *lambda : 0.f;
+  double e2 = 0.0, d2 = 0.0;
+  bool nonfinite = false;
+
+  for (int c0 = 0; c0 < bw; c0 += SB) {
+    float w[SB];
+#pragma unroll
+    for (int jj = 0; jj < SB; ++jj) w[jj] = (c0 + jj < bw) ? sW[(c0 + jj) * SW_LDW + rr] : 0.f;
+    if (G <= B && (s + c0) % G == 0) {
+      const int gw = min(G, bw - c0);
       float mn = INFINITY, mx = -INFINITY;
-      for (int j = 0; j < gw; ++j) {
-        float v = sW[i + j][lane];
+#pragma unroll
+      for (int jj = 0; jj < SB; ++jj)
+        if (jj < gw) mn = fminf(mn, w[jj]), mx = fmaxf(mx, w[jj]);
+      for (int j = c0 + SB + q; j < c0 + gw; j += 4) {
+        const float v = sW[j * SW_LDW + rr];
         mn = fminf(mn, v);
         mx = fmaxf(mx, v);
       }
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       grid_from_range(mn, mx, maxq, scale, zero);
-      if (valid) {
-        scales[(int64_t)row * ngroups + gi / G] = scale;
-        zeros[(int64_t)row * ngroups + gi / G] = (int32_t)zero;
+      if (valid && q == 0) {
+        scales[(int64_t)row * ngroups + (s + c0) / G] = scale;
+        zeros[(int64_t)row * ngroups + (s + c0) / G] = (int32_t)zero;
       }
     }
-    float w = sW[i][lane];
-    float c;
-    if (isfinite(w)) {
-      c = quant_code(w, scale, zero, maxq);
-    } else {
-      nonfinite = true;
-      c = zero;
+    float errs[SB];
+#pragma unroll
+    for (int ii = 0; ii < SB; ++ii) {
+      const int col = c0 + ii;
+      float err = 0.f;
+      if (col < bw) {
+        const float wv = w[ii];
+        float c;
+        if (isfinite(wv)) {
+          c = quant_code(wv, scale, zero, maxq);
+        } else {
+          nonfinite = true;
+          c = zero;
+        }
+        const float qv = scale * (c - zero);
+        err = (wv - qv) * rdg[col];
+        if (valid && (ii & 3) == q) {
+          const int oc = perm[s + col];
+          codes[(int64_t)row * k + oc] = (uint8_t)c;
+          if (loss != nullptr) {
+            const float w0 = dead[oc] ? 0.f : to_f32(W0[(int64_t)row * ldw + oc]);
+            const double dd = (double)w0 - (double)qv;
+            d2 += dd * dd;
+            e2 += (double)err * (double)err;
+          }
+        }
+      }
+      errs[ii] = err;
+#pragma unroll
+      for (int jj = ii + 1; jj < SB; ++jj)
+        w[jj] = fmaf(-err, UtS[(c0 + jj) * SW_LDU + col], w[jj]);
     }
-    float q = scale * (c - zero);
-    float err = (w - q) / U[(int64_t)gi * k + gi];
-    sE[i][lane] = err;
+    // rank-SB update of the block's remaining columns
+    for (int j = c0 + SB + q; j < bw; j += 4) {
+      float v = sW[j * SW_LDW + rr];
+      const float* ucol = UtS + j * SW_LDU + c0;
+#pragma unroll
+      for (int ii = 0; ii < SB; ++ii) v = fmaf(-errs[ii], ucol[ii], v);
+      sW[j * SW_LDW + rr] = v;
+    }
     if (valid) {
-      int oc = perm[gi];
-      codes[(int64_t)row * k + oc] = (uint8_t)c;
-      if (D != nullptr) D[(int64_t)row * k + oc] = to_f32(W0[(int64_t)row * ldw + oc]) - q;
+#pragma unroll
+      for (int ii = 0; ii < SB; ++ii)
+        if ((ii & 3) == q && c0 + ii < bw) Err[(int64_t)row * B + c0 + ii] = errs[ii];
     }
-    const float* urow = U + (int64_t)gi * k + s;
-    for (int j = i + 1; j < bw; ++j) sW[j][lane] = fmaf(-err, __ldg(urow + j), sW[j][lane]);
+    __syncwarp();
   }
-  __syncwarp();
-  for (int rr = 0; rr < 32; ++rr) {
-    int gr = r0 + rr;
-    if (gr < r)
-      for (int j = lane; j < bw; j += 32) Err[(int64_t)gr * B + j] = sE[j][rr];
+  if (loss != nullptr) {
+    e2 += __shfl_xor_sync(0xffffffffu, e2, 1);
+    d2 += __shfl_xor_sync(0xffffffffu, d2, 1);
+    e2 += __shfl_xor_sync(0xffffffffu, e2, 2);
+    d2 += __shfl_xor_sync(0xffffffffu, d2, 2);
+    if (valid && q == 0) atomicAdd(&loss[row], e2 - (double)lam * d2);
   }
   if (nonfinite && valid && d_status != nullptr) atomicCAS(d_status, 0, (int32_t)GPTQ_ERR_NONFINITE);
-}
-
-// loss[row] = sum_c Y[row][c] * D[row][c] (fp64), one warp per row.
-__global__ void rowdot_kernel(const float* __restrict__ Y, const float* __restrict__ D, int r,
-                              int k, double* __restrict__ loss) {
-  int warp = (blockIdx.x * blockDim.x + threadIdx.x) / kWarp;
-  int lane = threadIdx.x % kWarp;
-  if (warp >= r) return;
-  double acc = 0.0;
-  for (int c = lane; c < k; c += kWarp)
-    acc += (double)Y[(int64_t)warp * k + c] * (double)D[(int64_t)warp * k + c];
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) loss[warp] = acc;
 }
 
 __global__ void loss_total_kernel(double* __restrict__ loss, int r) {
@@ -180,6 +261,23 @@ __global__ void loss_total_kernel(double* __restrict__ loss, int r) {
   }
 }
 
+template <int SB, typename T>
+static void launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* Err,
+                         const float* U, const int32_t* perm, const uint8_t* dead, const T* W0,
+                         int64_t ldw, int r, int k, int s0, int bw, int B, int G, int ngroups,
+                         float maxq, const float* lambda, float* scales, int32_t* zeros,
+                         uint8_t* codes, double* loss, int32_t* d_status) {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(sweep_block_kernel<SB, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)SW_SMEM);
+    attr = true;
+  }
+  sweep_block_kernel<SB, T><<<grid, SW_THREADS, SW_SMEM, s>>>(
+      Wt, Err, U, perm, dead, W0, ldw, r, k, s0, bw, B, G, ngroups, maxq, lambda, scales, zeros,
+      codes, loss, d_status);
+}
+
 template <typename T>
 static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const float* U,
                                   const int32_t* perm, const uint8_t* dead, const float* H0,
@@ -192,11 +290,24 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
   const float maxq = (float)((1 << cfg->bits) - 1);
   SweepScratch sc = carve_sweep(ws, r, k, B);
   const bool want_loss = (H0 != nullptr && loss != nullptr);
+  double* lossp = want_loss ? loss : nullptr;
   {
     dim3 grid((unsigned)cdiv(k, 1024), (unsigned)r);
-    sweep_init_kernel<T><<<grid, 256, 0, s>>>(W, ldw, r, k, perm, dead, G, sc.Wt, g_idx, d_status);
+    sweep_init_kernel<T><<<grid, 256, 0, s>>>(W, ldw, r, k, perm, dead, G, sc.Wt, g_idx, lossp,
+                                              d_status);
     GPTQ_CHECK_LAUNCH();
   }
+  if (want_loss) {
+    sweep_lambda_kernel<<<1, 1024, 0, s>>>(H0, k, cfg->percdamp, sc.lambda);
+    GPTQ_CHECK_LAUNCH();
+  }
+  // sub-block width: 16, or the largest power of two dividing a smaller group
+  int SB = 16;
+  if (G < B) {
+    SB = 1;
+    while (SB < 16 && G % (SB * 2) == 0) SB *= 2;
+  }
+  const unsigned grid = (unsigned)cdiv(r, SW_ROWS);
   for (int s0 = 0; s0 < k; s0 += B) {
     int bw = min(B, k - s0);
     if (G > B && s0 % G == 0) {
@@ -205,23 +316,28 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
           sc.Wt, r, k, s0, gw, s0 / G, ngroups, maxq, scales, zeros);
       GPTQ_CHECK_LAUNCH();
     }
-    sweep_block_kernel<T><<<(unsigned)cdiv(r, 32), 32, 0, s>>>(
-        sc.Wt, sc.Err, U, perm, W, ldw, r, k, s0, bw, B, G, ngroups, maxq, scales, zeros, codes,
-        want_loss ? sc.D : nullptr, d_status);
+    const float* lam = want_loss ? sc.lambda : nullptr;
+#define GPTQ_SWEEP_BLOCK(SBV)                                                                     \
+  launch_block<SBV, T>(grid, s, sc.Wt, sc.Err, U, perm, dead, W, ldw, r, k, s0, bw, B, G, ngroups, \
+                       maxq, lam, scales, zeros, codes, lossp, d_status)
+    switch (SB) {
+      case 16: GPTQ_SWEEP_BLOCK(16); break;
+      case 8: GPTQ_SWEEP_BLOCK(8); break;
+      case 4: GPTQ_SWEEP_BLOCK(4); break;
+      case 2: GPTQ_SWEEP_BLOCK(2); break;
+      default: GPTQ_SWEEP_BLOCK(1); break;
+    }
+#undef GPTQ_SWEEP_BLOCK
     GPTQ_CHECK_LAUNCH();
     int e0 = s0 + bw;
     if (e0 < k) {
-      sgemm<false, false, false, false, false>(r, k - e0, bw, -1.0f, sc.Err, B, U + (int64_t)s0 * k + e0, k,
-                                 1.0f, sc.Wt + e0, k, nullptr, s);
+      sgemm<false, false, false, false, false>(r, k - e0, bw, -1.0f, sc.Err, B,
+                                               U + (int64_t)s0 * k + e0, k, 1.0f, sc.Wt + e0, k,
+                                               nullptr, s);
       GPTQ_CHECK_LAUNCH();
     }
   }
   if (want_loss) {
-    // Y = D * H0 into the (now free) working copy, then per-row dot with D.
-    sgemm<false, false, false, false, false>(r, k, k, 1.0f, sc.D, k, H0, k, 0.0f, sc.Wt, k, nullptr, s);
-    GPTQ_CHECK_LAUNCH();
-    rowdot_kernel<<<(unsigned)cdiv((int64_t)r * kWarp, 256), 256, 0, s>>>(sc.Wt, sc.D, r, k, loss);
-    GPTQ_CHECK_LAUNCH();
     loss_total_kernel<<<1, 1024, 0, s>>>(loss, r);
     GPTQ_CHECK_LAUNCH();
   }

@@ -304,6 +304,30 @@ def test_layer_loss_equals_direct_output_error():
     assert np.allclose(res["loss_rows"], 2.0 / X.shape[0] * np.sum((D @ X.T) ** 2, axis=1))
 
 
+@pytest.mark.parametrize("gs,bs,act,bits", [(32, 32, False, 4), (128, 128, True, 3),
+                                             (-1, 64, False, 2), (16, 64, True, 8)])
+def test_loss_equals_obs_error_sum(gs, bs, act, bits):
+    # Optimal Brain Surgeon accounting ("GPTQ" page, Where it came from; the
+    # guide's Detailed Algorithm): fixing column i and compensating the rest
+    # raises (w - q)^T Hd (w - q) by err_i^2 = (w_i - q_i)^2 / U_ii^2, so the
+    # damped layer error is the sum of err^2 and the undamped one subtracts
+    # lambda * ||W0 - Q||^2.  Holds row by row, with groups, act-order and dead
+    # columns (whose original weights count as 0).
+    spec = synth.CONFIGS["q_proj"].scaled(r=24, k=192, n=3000)
+    W = synth.make_w(spec, bits).numpy().astype(np.float64)
+    X = synth.make_x(spec, bits).numpy()
+    X[:, [5, 77]] = 0
+    H = O.hessian(X)
+    res = O.gptq(W, H, bits, gs, bs, 0.01, act)
+    Hf, Wf, dead = O.fix_dead_columns(H, W)
+    perm = res["perm"]
+    lam = 0.01 * np.mean(np.diag(Hf))
+    sw = O.sweep_blocked(Wf[:, perm], res["U"], bits, gs, bs)
+    e2 = (sw["err"] ** 2).sum(axis=1)
+    d2 = ((Wf[:, perm] - sw["qhat"]) ** 2).sum(axis=1)
+    assert np.allclose(e2 - lam * d2, res["loss_rows"], rtol=1e-10, atol=0)
+
+
 @pytest.mark.parametrize("seed", range(5))
 def test_gptq_beats_rtn_on_tiny_layer(seed):
     # "GPTQ" (ozercemkelahmet.com), sketch remark: compare the output error with
