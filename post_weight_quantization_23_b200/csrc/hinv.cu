@@ -10,20 +10,20 @@
 // about half its flops.  fp32 throughout.
 //
 // One k x k work matrix (the output U) holds both factors: L grows in the
-// LOWER triangle while U is built in the UPPER one, so the inverse never
-// reads what it writes.
-// Factor, blocks of HV_B = 64 indices from the last one up, step J = [j0, j1):
+// LOWER triangle; the UPPER triangle first holds Y = V[0:e, e:] U[e:, e:]
+// (rows above the processed part) and turns into U row block by row block.
+// Blocks of HV_B = 64 indices, from the last one up; step J = [j0, j1), e = j1:
 //   K1 diag    L_JJ from the Schur-updated diagonal block (lower part) and
 //              U_JJ = (L_JJ^T)^-1, written to A[J, J] (upper) and the scratch.
-//   K2 panel   L[J, 0:j0] = U_JJ * Hp[J, 0:j0]   (in place, lower part).
-//   K3 update  A[0:j0, 0:j0] (lower) -= L[J, 0:j0]^T L[J, 0:j0].
-// Inverse, recursively over halves of the block range (leaves = the U_JJ):
-//   with V = [[V11, V12], [0, V22]], U12 = -U11 V12 U22 and V12 = L21^T:
-//   S = U11 * L21^T into the free upper-right block, then U12 = -S * U22 in
-//   place (row by row, columns right to left).
+//   K2 panel   P = L[J, 0:j0] = U_JJ * Hp[J, 0:j0]   (in place, lower part),
+//      and     U[J, e:] = -U_JJ * Y[J, e:]          (in place, upper part):
+//              V = [[V_JJ, V_J*], [0, V_**]] gives U_J* = -V_JJ^-1 V_J* U_**.
+//   K3 one rank-64 update of rows [0, j0) (K = the 64 rows of block J):
+//              A[0:j0, 0:j0] (lower) -= P^T P        (Schur complement)
+//              Y[0:j0, j0:]          += P^T U[J, j0:] (V[0:j0, J] = P^T)
+// so every step's large work is a short-K product with a big output.
 // A final pass zeroes the strict lower triangle.
 #include "common.cuh"
-#include "sgemm.cuh"
 
 namespace gptq {
 
@@ -114,7 +114,7 @@ __global__ void hinv_rank_kernel(const float* __restrict__ diag, int k, int act_
 }
 
 // A[a][b] = H[perm[a]][perm[b]] for b <= a (lower part), the diagonal replaced
-// by diag (dead fix) + lambda.
+// by diag (dead fix) + lambda; the strict upper part (Y) starts at 0.
 __global__ void hinv_gather_lower_kernel(const float* __restrict__ H, int k,
                                          const int32_t* __restrict__ perm,
                                          const float* __restrict__ diag,
@@ -123,8 +123,8 @@ __global__ void hinv_gather_lower_kernel(const float* __restrict__ H, int k,
   int pa = perm[a];
   float lam = *lambda;
   const float* hrow = H + (int64_t)pa * k;
-  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b <= a; b += gridDim.x * blockDim.x) {
-    float v = (b == a) ? diag[pa] + lam : hrow[perm[b]];
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < k; b += gridDim.x * blockDim.x) {
+    float v = (b == a) ? diag[pa] + lam : (b < a ? hrow[perm[b]] : 0.f);
     A[(int64_t)a * k + b] = v;
   }
 }
@@ -133,27 +133,31 @@ __device__ __forceinline__ void set_info(int32_t* d_info, int idx) { atomicCAS(d
 
 // K1: factor the diagonal block (lower storage, A_JJ = L^T L with L lower)
 // and invert V = L^T: U_JJ = V^-1 (upper), written to the scratch and to the
-// upper part of A[J, J] (the block was read into shared memory first).  One
-// CTA of 256 threads.
+// upper part of A[J, J].  One CTA of 256 threads.
 //   factor, c = b-1 .. 0:  a_ij -= a_ci a_cj / a_cc  (j <= i < c), then
 //   L_cj = a_cj / sqrt(a_cc) (j < c), L_cc = sqrt(a_cc);
-//   inverse, i = b-1 .. 0: U_ii = 1 / V_ii, U_ic = -(sum_{m=i+1..c} V_im U_mc) / V_ii,
-//   with V_im = L_mi.
+//   inverse, i = b-1 .. 0: U_ii = 1 / L_ii, U_ic = -(sum_{m=i+1..c} L_mi U_mc) / L_ii.
+// Factor: thread (ri = t / 4, jq = t % 4) keeps a[ri][jq + 4q] (q < 16) in
+// registers and writes them through to shared memory, where step c reads the
+// pivot row c; one barrier per step.  Inverse: thread (c = t / 4, part = t % 4)
+// keeps U[part + 4u][c] (u < 16) in registers; the four threads of a column
+// combine their partial sums with shuffles, so the inverse needs no barrier.
 __global__ void __launch_bounds__(256)
 chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
                      float* __restrict__ ujj, int32_t* __restrict__ d_info) {
   if (*d_info != 0) return;
   __shared__ float S[HV_B][HV_B + 1];
-  __shared__ float Y[HV_B][HV_B + 1];
-  __shared__ float dg[HV_B];
+  __shared__ float rdg[HV_B];
   const int t = threadIdx.x;
-  for (int e = t; e < HV_B * HV_B; e += 256) {
-    int i = e / HV_B, j = e % HV_B;
-    S[i][j] = (i < b && j <= i) ? A[(int64_t)(j0 + i) * k + j0 + j] : 0.f;
-    Y[i][j] = 0.f;
+  const int ri = t >> 2, jq = t & 3;
+  float r[HV_B / 4];
+#pragma unroll
+  for (int q = 0; q < HV_B / 4; ++q) {
+    const int j = jq + 4 * q;
+    r[q] = (ri < b && j <= ri) ? A[(int64_t)(j0 + ri) * k + j0 + j] : 0.f;
+    S[ri][j] = r[q];
   }
   __syncthreads();
-  const int ri = t >> 2, jq = t & 3;  // row ri, columns jq, jq+4, ...
   int fail = -1;
   for (int c = b - 1; c >= 0; --c) {
     const float p = S[c][c];
@@ -162,11 +166,17 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
       break;
     }
     if (ri < c) {
-      const float f = S[c][ri] / p;
+      const float f = S[c][ri] * __frcp_rn(p);
+      float cv[HV_B / 4];
+#pragma unroll
+      for (int q = 0; q < HV_B / 4; ++q) cv[q] = S[c][jq + 4 * q];
 #pragma unroll
       for (int q = 0; q < HV_B / 4; ++q) {
         const int j = jq + 4 * q;
-        if (j <= ri) S[ri][j] = fmaf(-f, S[c][j], S[ri][j]);
+        if (j <= ri) {
+          r[q] = fmaf(-f, cv[q], r[q]);
+          S[ri][j] = r[q];
+        }
       }
     }
     __syncthreads();
@@ -175,57 +185,78 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
     if (t == 0) set_info(d_info, j0 + fail);
     return;
   }
-  if (t < b) dg[t] = sqrtf(S[t][t]);
-  __syncthreads();
-  // scale to L: L_ij = a_ij / sqrt(a_ii) below the diagonal, L_ii = sqrt(a_ii)
+  // L: scale each row by 1 / sqrt(a_ii); S then holds L
   if (ri < b) {
-    const float rd = 1.0f / dg[ri];
+    const float d = sqrtf(S[ri][ri]);
+    const float rd = __frcp_rn(d);
 #pragma unroll
     for (int q = 0; q < HV_B / 4; ++q) {
       const int j = jq + 4 * q;
-      if (j < ri) S[ri][j] *= rd;
+      if (j < ri) r[q] *= rd;
+      else if (j == ri) r[q] = d;
     }
+    if (jq == 0) rdg[ri] = rd;
   }
   __syncthreads();
-  if (t < b) S[t][t] = dg[t];
+#pragma unroll
+  for (int q = 0; q < HV_B / 4; ++q) {
+    const int j = jq + 4 * q;
+    if (j <= ri) S[ri][j] = r[q];
+  }
   __syncthreads();
-  // inverse of V = L^T, rows from the bottom; thread (c = t / 4, part = t % 4)
+  // inverse of V = L^T by rows from the bottom; y[u] = U[part + 4u][c]
   const int c = t >> 2, part = t & 3;
-  for (int i = b - 1; i >= 0; --i) {
-    float s = 0.f;
-    if (c > i && c < b)
-      for (int m = i + 1 + part; m <= c; m += 4) s = fmaf(S[m][i], Y[m][c], s);
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
-    if (part == 0 && c < b) {
-      const float rv = 1.0f / S[i][i];
-      if (c == i) Y[i][i] = rv;
-      else if (c > i) Y[i][c] = -s * rv;
+  float y[HV_B / 4];
+#pragma unroll
+  for (int u = 0; u < HV_B / 4; ++u) y[u] = 0.f;
+#pragma unroll
+  for (int i = HV_B - 1; i >= 0; --i) {
+    if (i < b) {  // uniform
+      float sum = 0.f;
+#pragma unroll
+      for (int u = 0; u < HV_B / 4; ++u) {
+        const int m = part + 4 * u;
+        if (m > i && m <= c && m < b) sum = fmaf(S[m][i], y[u], sum);
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      if ((i & 3) == part && c < b) {
+        const float rv = rdg[i];
+        if (c == i) y[i >> 2] = rv;
+        else if (c > i) y[i >> 2] = -sum * rv;
+      }
     }
-    __syncthreads();
   }
-  for (int e = t; e < HV_B * HV_B; e += 256) {
-    const int i = e / HV_B, j = e % HV_B;
-    const float y = Y[i][j];
-    ujj[e] = y;
-    if (i < b && j < b && j >= i) A[(int64_t)(j0 + i) * k + j0 + j] = y;
+#pragma unroll
+  for (int u = 0; u < HV_B / 4; ++u) {
+    const int i = part + 4 * u;
+    ujj[i * HV_B + c] = y[u];
+    if (i < b && c < b && c >= i) A[(int64_t)(j0 + i) * k + j0 + c] = y[u];
   }
 }
 
-// K2: L[J, c] = U_JJ * A[J, c] for columns c in [c0, c0 + 64) of [0, j0), in
-// place.  Thread (r = t / 4, cq = t % 4) computes row r, columns cq + 4q.
+// K2, one launch, two independent roles:
+//   CTAs [0, n_pan): 64-column tiles c0 of [0, j0): P[:, c] = U_JJ * A[J, c]
+//     (lower part of row block J, in place).
+//   CTAs [n_pan, ...): 64-column tiles c0 of [e, k): U[J, c] = -U_JJ * Y[J, c]
+//     (upper part of row block J, in place).
+// Each CTA reads its whole 64 x 64 tile before writing it.  Thread
+// (r = t / 4, cq = t % 4) computes row r, columns cq + 4q.
 __global__ void __launch_bounds__(256)
-chol_panel_kernel(float* __restrict__ A, int k, int j0, int b, const float* __restrict__ ujj,
-                  const int32_t* __restrict__ d_info) {
+panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* __restrict__ ujj,
+                      int n_pan, const int32_t* __restrict__ d_info) {
   if (*d_info != 0) return;
   __shared__ float Us[HV_B][HV_B + 1];
   __shared__ float Hs[HV_B][HV_B + 1];
   const int t = threadIdx.x;
-  const int c0 = blockIdx.x * HV_B;
+  const bool pan = (int)blockIdx.x < n_pan;
+  const int c0 = pan ? blockIdx.x * HV_B : j0 + b + (blockIdx.x - n_pan) * HV_B;
+  const int cend = pan ? j0 : k;
+  const float sign = pan ? 1.0f : -1.0f;
   for (int e = t; e < HV_B * HV_B; e += 256) {
     int i = e / HV_B, j = e % HV_B;
     Us[i][j] = ujj[e];
-    Hs[i][j] = (i < b && c0 + j < j0) ? A[(int64_t)(j0 + i) * k + c0 + j] : 0.f;
+    Hs[i][j] = (i < b && c0 + j < cend) ? A[(int64_t)(j0 + i) * k + c0 + j] : 0.f;
   }
   __syncthreads();
   const int r = t >> 2, cq = t & 3;
@@ -241,115 +272,122 @@ chol_panel_kernel(float* __restrict__ A, int k, int j0, int b, const float* __re
 #pragma unroll
   for (int q = 0; q < HV_B / 4; ++q) {
     const int cc = c0 + cq + 4 * q;
-    if (cc < j0) A[(int64_t)(j0 + r) * k + cc] = acc[q];
+    if (cc < cend) A[(int64_t)(j0 + r) * k + cc] = sign * acc[q];
   }
 }
 
-// K3: A[0:n, 0:n] (lower) -= P^T P with P = A[j0:j0+b, 0:n] (b x n): 128 x 128
-// tiles on or below the diagonal, 256 threads with 8 x 8 outputs.
+// K3: rows [0, j0) += P^T Q with P = A[j0:j0+b, 0:j0] (the panel) and
+//   Q[m][c] = -P[m][c]            for c < j0 (lower-triangle tiles only),
+//   Q[m][c] = U[j0 + m][c]        for c >= j0 (U_JJ read as upper triangular).
+// 128 x 128 output tiles; the K = b rows are taken in chunks of 16, double
+// buffered; thread (ty = t / 16, tx = t % 16) owns 8 x 8 outputs.
+constexpr int RU_KC = 16, RU_LD = 128 + 4;
+
 __global__ void __launch_bounds__(256)
-syrk_lower_tn_kernel(float* __restrict__ A, int k, int n, int j0, int b,
-                     const int32_t* __restrict__ d_info) {
+rank_update_kernel(float* __restrict__ A, int k, int j0, int b, int n_low,
+                   const int32_t* __restrict__ d_info) {
   if (*d_info != 0) return;
-  const int bi = blockIdx.y, bj = blockIdx.x;
-  if (bj > bi) return;
-  const int i0 = bi * 128, jj0 = bj * 128;
-  __shared__ float Pi[16][128 + 4];
-  __shared__ float Pj[16][128 + 4];
+  __shared__ float Pi[2][RU_KC][RU_LD];
+  __shared__ float Qc[2][RU_KC][RU_LD];
+  const int x = blockIdx.x;
+  int bi, c0;
+  bool low;
+  if (x < n_low) {
+    low = true;
+    bi = (int)((sqrtf(8.0f * x + 1.0f) - 1.0f) * 0.5f);
+    while (bi * (bi + 1) / 2 > x) --bi;
+    while ((bi + 1) * (bi + 2) / 2 <= x) ++bi;
+    c0 = (x - bi * (bi + 1) / 2) * 128;
+  } else {
+    low = false;
+    const int nt = (j0 + 127) / 128;
+    const int y = x - n_low;
+    bi = y % nt;
+    c0 = j0 + (y / nt) * 128;
+  }
+  const int i0 = bi * 128;
+  const int j1 = j0 + b;
   const int t = threadIdx.x, tx = t % 16, ty = t / 16;
+  const int lm = t / 16, lc = (t % 16) * 8;
   float acc[8][8];
 #pragma unroll
   for (int p = 0; p < 8; ++p)
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[p][q] = 0.f;
-  for (int m0 = 0; m0 < b; m0 += 16) {
-    for (int e = t; e < 16 * 128; e += 256) {
-      int mm = e / 128, cc = e % 128;
-      const float* prow = A + (int64_t)(j0 + m0 + mm) * k;
-      bool okm = m0 + mm < b;
-      Pi[mm][cc] = (okm && i0 + cc < n) ? prow[i0 + cc] : 0.f;
-      Pj[mm][cc] = (okm && jj0 + cc < n) ? prow[jj0 + cc] : 0.f;
-    }
-    __syncthreads();
+  float ri[8], rq[8];
+  auto gload = [&](int m0) {
+    const int m = m0 + lm;
+    const bool okm = m < b;
+    const float* prow = A + (int64_t)(j0 + m) * k;
 #pragma unroll
-    for (int mm = 0; mm < 16; ++mm) {
+    for (int q = 0; q < 8; ++q) {
+      const int i = i0 + lc + q, c = c0 + lc + q;
+      ri[q] = (okm && i < j0) ? prow[i] : 0.f;
+      bool okq;
+      if (low) okq = okm && c < j0;
+      else okq = okm && c < k && (c >= j1 || m <= c - j0);
+      rq[q] = okq ? prow[c] : 0.f;
+    }
+  };
+  auto sstore = [&](int buf) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      Pi[buf][lm][lc + q] = ri[q];
+      Qc[buf][lm][lc + q] = rq[q];
+    }
+  };
+  gload(0);
+  sstore(0);
+  __syncthreads();
+  int buf = 0;
+  for (int m0 = 0; m0 < b; m0 += RU_KC) {
+    const bool more = m0 + RU_KC < b;
+    if (more) gload(m0 + RU_KC);
+#pragma unroll
+    for (int mm = 0; mm < RU_KC; ++mm) {
       float a[8], bb[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        a[q] = Pi[mm][ty * 4 + q];
-        a[q + 4] = Pi[mm][64 + ty * 4 + q];
-        bb[q] = Pj[mm][tx * 4 + q];
-        bb[q + 4] = Pj[mm][64 + tx * 4 + q];
+        a[q] = Pi[buf][mm][ty * 4 + q];
+        a[q + 4] = Pi[buf][mm][64 + ty * 4 + q];
+        bb[q] = Qc[buf][mm][tx * 4 + q];
+        bb[q + 4] = Qc[buf][mm][64 + tx * 4 + q];
       }
 #pragma unroll
       for (int p = 0; p < 8; ++p)
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[p][q] = fmaf(a[p], bb[q], acc[p][q]);
     }
+    if (more) sstore(buf ^ 1);
     __syncthreads();
+    buf ^= 1;
   }
+  const float sign = low ? -1.0f : 1.0f;
+  const int cend = low ? j0 : k;
+  const bool vec = (k % 4 == 0) && (!low || c0 + 127 < i0);
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
     const int gi = i0 + (p < 4 ? ty * 4 + p : 64 + ty * 4 + p - 4);
-    if (gi >= n) continue;
+    if (gi >= j0) continue;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int gj = jj0 + (q < 4 ? tx * 4 + q : 64 + tx * 4 + q - 4);
-      if (gj <= gi && gj < n) A[(int64_t)gi * k + gj] -= acc[p][q];
-    }
-  }
-}
-
-// C[0:M, 0:N] := alpha * C * Uu, Uu (N x N) upper triangular, in place.
-// Row a of the result needs only row a of C, and column c needs C[a][0..c]:
-// each CTA owns TM rows and walks column tiles from right to left, so the
-// entries it still has to read are never overwritten.  256 threads: thread
-// (ty = t / 64, tx = t % 64) owns rows 4ty..4ty+3 of the tile, column tx.
-constexpr int TR_TM = 16, TR_TN = 64, TR_KC = 32;
-__global__ void __launch_bounds__(256)
-trmm_right_upper_inplace_kernel(float* __restrict__ C, int64_t ldc, int M, int N,
-                                const float* __restrict__ Uu, int64_t ldu, float alpha,
-                                const int32_t* __restrict__ d_info) {
-  if (*d_info != 0) return;
-  __shared__ float Cs[TR_TM][TR_KC + 1];
-  __shared__ float Us[TR_KC][TR_TN + 4];
-  const int t = threadIdx.x, ty = t >> 6, tx = t & 63;
-  const int a0 = blockIdx.x * TR_TM;
-  if (a0 >= M) return;
-  const int ntiles = (N + TR_TN - 1) / TR_TN;
-  for (int tile = ntiles - 1; tile >= 0; --tile) {
-    const int c0 = tile * TR_TN;
-    const int kend = min(N, c0 + TR_TN);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int m0 = 0; m0 < kend; m0 += TR_KC) {
-      for (int q = t; q < TR_TM * TR_KC; q += 256) {
-        const int aa = q / TR_KC, mm = q % TR_KC;
-        const int gr = a0 + aa, gm = m0 + mm;
-        Cs[aa][mm] = (gr < M && gm < kend) ? C[(int64_t)gr * ldc + gm] : 0.f;
-      }
-      for (int q = t; q < TR_KC * TR_TN; q += 256) {
-        const int mm = q / TR_TN, cc = q % TR_TN;
-        const int gm = m0 + mm, gc = c0 + cc;
-        Us[mm][cc] = (gm < kend && gc < N && gm <= gc) ? Uu[(int64_t)gm * ldu + gc] : 0.f;
-      }
-      __syncthreads();
-#pragma unroll 8
-      for (int mm = 0; mm < TR_KC; ++mm) {
-        const float u = Us[mm][tx];
+    for (int h = 0; h < 2; ++h) {
+      const int gc = c0 + h * 64 + tx * 4;
+      float* dst = A + (int64_t)gi * k + gc;
+      if (vec && gc + 3 < cend) {
+        float4 v = *reinterpret_cast<float4*>(dst);
+        v.x = fmaf(sign, acc[p][h * 4 + 0], v.x);
+        v.y = fmaf(sign, acc[p][h * 4 + 1], v.y);
+        v.z = fmaf(sign, acc[p][h * 4 + 2], v.z);
+        v.w = fmaf(sign, acc[p][h * 4 + 3], v.w);
+        *reinterpret_cast<float4*>(dst) = v;
+      } else {
 #pragma unroll
-        for (int p = 0; p < 4; ++p) acc[p] = fmaf(Cs[4 * ty + p][mm], u, acc[p]);
-      }
-      __syncthreads();
-    }
-    const int gc = c0 + tx;
-    if (gc < N) {
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int gr = a0 + 4 * ty + p;
-        if (gr < M) C[(int64_t)gr * ldc + gc] = alpha * acc[p];
+        for (int q = 0; q < 4; ++q) {
+          const int c = gc + q;
+          if (c < cend && (!low || c <= gi)) dst[q] = fmaf(sign, acc[p][h * 4 + q], dst[q]);
+        }
       }
     }
-    __syncthreads();
   }
 }
 
@@ -359,37 +397,6 @@ __global__ void zero_lower_kernel(float* __restrict__ U, int k, const int32_t* _
   int i = blockIdx.y;
   for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < i; j += gridDim.x * blockDim.x)
     U[(int64_t)i * k + j] = 0.f;
-}
-
-// Start of block `blk` when blocks of HV_B are laid from the bottom (the
-// short block, if any, is block 0 at the top).
-static int block_start(int k, int blk) {
-  const int nb = (int)cdiv(k, HV_B);
-  return std::max(0, k - (nb - blk) * HV_B);
-}
-
-// Upper inverse of the blocks [lo, hi): both halves first, then the coupling
-// block U12 = -U11 * L21^T * U22.
-static gptq_status trtri_range(float* A, int k, int lo, int hi, const int32_t* d_info,
-                               cudaStream_t s) {
-  if (hi - lo <= 1) return GPTQ_OK;  // leaf: U_JJ written by the diagonal kernel
-  const int mid = (lo + hi) / 2;
-  gptq_status st = trtri_range(A, k, lo, mid, d_info, s);
-  if (st != GPTQ_OK) return st;
-  st = trtri_range(A, k, mid, hi, d_info, s);
-  if (st != GPTQ_OK) return st;
-  const int r1 = block_start(k, lo), r2 = block_start(k, mid);
-  const int e = (hi == (int)cdiv(k, HV_B)) ? k : block_start(k, hi);
-  const int k1 = r2 - r1, k2 = e - r2;
-  // S = U11 * L21^T  (U11 upper; L21 = A[r2:e, r1:r2]) into A[r1:r2, r2:e]
-  sgemm<false, true, true, false, false>(k1, k2, k1, 1.0f, A + (int64_t)r1 * k + r1, k,
-                                         A + (int64_t)r2 * k + r1, k, 0.0f,
-                                         A + (int64_t)r1 * k + r2, k, d_info, s);
-  GPTQ_CHECK_LAUNCH();
-  trmm_right_upper_inplace_kernel<<<(unsigned)cdiv(k1, TR_TM), 256, 0, s>>>(
-      A + (int64_t)r1 * k + r2, k, k1, k2, A + (int64_t)r2 * k + r2, k, -1.0f, d_info);
-  GPTQ_CHECK_LAUNCH();
-  return GPTQ_OK;
 }
 
 gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cfg, float* U,
@@ -414,17 +421,20 @@ gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cf
     const int b = j1 - j0;
     chol_inv_diag_kernel<<<1, 256, 0, s>>>(U, k, j0, b, sc.ujj, d_info);
     GPTQ_CHECK_LAUNCH();
-    if (j0 > 0) {
-      chol_panel_kernel<<<(unsigned)cdiv(j0, HV_B), 256, 0, s>>>(U, k, j0, b, sc.ujj, d_info);
-      GPTQ_CHECK_LAUNCH();
-      const int nt = (int)cdiv(j0, 128);
-      syrk_lower_tn_kernel<<<dim3(nt, nt), 256, 0, s>>>(U, k, j0, j0, b, d_info);
+    const int n_pan = (int)cdiv(j0, HV_B);
+    const int n_row = (int)cdiv(k - j1, HV_B);
+    if (n_pan + n_row > 0) {
+      panel_rowblock_kernel<<<(unsigned)(n_pan + n_row), 256, 0, s>>>(U, k, j0, b, sc.ujj, n_pan,
+                                                                       d_info);
       GPTQ_CHECK_LAUNCH();
     }
-  }
-  {
-    gptq_status st = trtri_range(U, k, 0, (int)cdiv(k, HV_B), d_info, s);
-    if (st != GPTQ_OK) return st;
+    if (j0 > 0) {
+      const int nt = (int)cdiv(j0, 128);
+      const int n_low = nt * (nt + 1) / 2;
+      const int n_right = nt * (int)cdiv(k - j0, 128);
+      rank_update_kernel<<<(unsigned)(n_low + n_right), 256, 0, s>>>(U, k, j0, b, n_low, d_info);
+      GPTQ_CHECK_LAUNCH();
+    }
   }
   {
     dim3 grid((unsigned)cdiv(k, 1024), (unsigned)k);
