@@ -53,32 +53,38 @@ def _peaks():
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """Samples SM clocks and throttle reasons with nvidia-smi every 100 ms while
+    the timed region runs (all GPUs are queried; the one on this process's
+    PCI bus is kept, or the only one)."""
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index):
         self.proc = None
-        self.lines = []
-        self.dev = str(device_index)
+        self.first = ""
+        self.bus = None
         try:
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
-            if bus:
-                self.dev = bus
+            self.bus = str(torch.cuda.get_device_properties(device_index).pci_bus_id).lower()
         except Exception:
             pass
 
     def start(self):
-        """Start sampling every 100 ms; returns once the first sample is in."""
+        """Start sampling; returns once the first sample is in."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", self.dev], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.first = self.proc.stdout.readline()
         except Exception:
             self.proc = None
-            self.first = ""
+
+    def _mine(self, bus_field, n_lines_seen):
+        if self.bus is None:
+            return True
+        a = bus_field.lower().split(":", 1)[-1]
+        b = self.bus.split(":", 1)[-1]
+        return a == b
 
     def stop(self):
         if self.proc is None:
@@ -90,12 +96,14 @@ class ClockSampler:
             self.proc.kill()
             out, _ = self.proc.communicate()
         out = (self.first or "") + (out or "")
+        rows = [[x.strip() for x in line.split(",")] for line in out.strip().splitlines()]
+        rows = [f for f in rows if len(f) >= 9]
+        buses = {f[0] for f in rows}
+        if len(buses) > 1:
+            rows = [f for f in rows if self._mine(f[0], 0)]
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
+        for f in rows:
             try:
                 sm.append(float(f[1]))
                 mx.append(float(f[2]))

@@ -13,7 +13,7 @@ size_t hessian_tc_workspace_bytes(int64_t k, int64_t n);
 size_t hinv_workspace_bytes(int64_t k);
 gptq_status prepare_hinv_impl(const float* H, int64_t k, const gptq_config* cfg, float* U,
                               int32_t* perm, int32_t* invperm, uint8_t* dead, int32_t* d_info,
-                              void* ws, cudaStream_t s);
+                              void* ws, size_t ws_bytes, cudaStream_t s);
 size_t sweep_workspace_bytes(int64_t r, int64_t k, int B);
 gptq_status quantize_layer_impl(const void* W, gptq_dtype dt, int64_t r, int64_t k, int64_t ldw,
                                 const float* U, const int32_t* perm, const uint8_t* dead,
@@ -119,7 +119,8 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t k, const gptq_config* cfg,
   if ((const void*)H == (const void*)U) return GPTQ_ERR_INVALID_ARG;
   size_t need = hinv_workspace_bytes(k);
   if (ws == nullptr || ws_bytes < need || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
-  return prepare_hinv_impl(H, k, cfg, U, perm, invperm, dead, d_info, ws, (cudaStream_t)stream);
+  return prepare_hinv_impl(H, k, cfg, U, perm, invperm, dead, d_info, ws, ws_bytes,
+                           (cudaStream_t)stream);
 }
 
 gptq_status gptq_quantize_layer(const void* W, gptq_dtype dt, int64_t r, int64_t k, int64_t ldw,

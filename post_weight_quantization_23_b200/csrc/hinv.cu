@@ -18,7 +18,9 @@
 //   K2 panel   P = L[J, 0:j0] = U_JJ * Hp[J, 0:j0]   (in place, lower part),
 //      and     U[J, e:] = -U_JJ * Y[J, e:]          (in place, upper part):
 //              V = [[V_JJ, V_J*], [0, V_**]] gives U_J* = -V_JJ^-1 V_J* U_**.
-//   K3 one rank-64 update of rows [0, j0) (K = the 64 rows of block J):
+//   K3 one rank-64 update of rows [0, j0) (K = the 64 rows of block J), on
+//      the tensor cores in fp32-accurate 3xTF32 when the workspace holds the
+//      operand splits (tf32x3.cu), else on the CUDA cores:
 //              A[0:j0, 0:j0] (lower) -= P^T P        (Schur complement)
 //              Y[0:j0, j0:]          += P^T U[J, j0:] (V[0:j0, J] = P^T)
 // so every step's large work is a short-K product with a big output.
@@ -29,14 +31,21 @@ namespace gptq {
 
 constexpr int HV_B = 64;  // block width
 
+bool tc_update_supported(int64_t k);
+gptq_status tc_rank_update(float* A, int k, int j0, int b, float* r_hi, float* r_lo,
+                           int32_t* d_info, cudaStream_t s);
+
 struct HinvScratch {
   double* sum_diag;  // [1]
   float* lambda;     // [1]
   float* diag;       // [k] diag(H) after the dead-column fix
   float* ujj;        // [HV_B * HV_B] U_JJ of the current step
+  float* r_hi;       // [HV_B * k] tf32 split of the current row block (tensor-core path)
+  float* r_lo;       // [HV_B * k]
 };
 
-size_t hinv_workspace_bytes(int64_t k) {
+// Scratch of the CUDA-core path.
+size_t hinv_workspace_min_bytes(int64_t k) {
   size_t b = 0;
   b += align256(sizeof(double));
   b += align256(sizeof(float));
@@ -45,13 +54,23 @@ size_t hinv_workspace_bytes(int64_t k) {
   return b;
 }
 
-static HinvScratch carve(void* ws, int64_t k) {
+// Scratch of the tensor-core path (the size gptq_workspace_size reports).
+size_t hinv_workspace_bytes(int64_t k) {
+  size_t b = hinv_workspace_min_bytes(k);
+  if (tc_update_supported(k)) b += 2 * align256(sizeof(float) * HV_B * (size_t)k);
+  return b;
+}
+
+static HinvScratch carve(void* ws, int64_t k, bool tc) {
   char* p = (char*)ws;
   HinvScratch s;
   s.sum_diag = (double*)p; p += align256(sizeof(double));
   s.lambda = (float*)p; p += align256(sizeof(float));
   s.diag = (float*)p; p += align256(sizeof(float) * (size_t)k);
-  s.ujj = (float*)p;
+  s.ujj = (float*)p; p += align256(sizeof(float) * HV_B * HV_B);
+  s.r_hi = tc ? (float*)p : nullptr;
+  if (tc) p += align256(sizeof(float) * HV_B * (size_t)k);
+  s.r_lo = tc ? (float*)p : nullptr;
   return s;
 }
 
@@ -401,9 +420,11 @@ __global__ void zero_lower_kernel(float* __restrict__ U, int k, const int32_t* _
 
 gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cfg, float* U,
                               int32_t* perm, int32_t* invperm, uint8_t* dead, int32_t* d_info,
-                              void* ws, cudaStream_t s) {
+                              void* ws, size_t ws_bytes, cudaStream_t s) {
   const int k = (int)k64;
-  HinvScratch sc = carve(ws, k);
+  // tensor-core rank updates when the workspace holds their operand splits
+  const bool tc = tc_update_supported(k) && ws_bytes >= hinv_workspace_bytes(k);
+  HinvScratch sc = carve(ws, k, tc);
   hinv_prep_kernel<<<1, 1024, 0, s>>>(H, k, cfg->percdamp, dead, sc.diag, sc.sum_diag, sc.lambda,
                                       d_info);
   GPTQ_CHECK_LAUNCH();
@@ -429,11 +450,17 @@ gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cf
       GPTQ_CHECK_LAUNCH();
     }
     if (j0 > 0) {
-      const int nt = (int)cdiv(j0, 128);
-      const int n_low = nt * (nt + 1) / 2;
-      const int n_right = nt * (int)cdiv(k - j0, 128);
-      rank_update_kernel<<<(unsigned)(n_low + n_right), 256, 0, s>>>(U, k, j0, b, n_low, d_info);
-      GPTQ_CHECK_LAUNCH();
+      if (tc) {
+        gptq_status st = tc_rank_update(U, k, j0, b, sc.r_hi, sc.r_lo, d_info, s);
+        if (st != GPTQ_OK) return st;
+      } else {
+        const int nt = (int)cdiv(j0, 128);
+        const int n_low = nt * (nt + 1) / 2;
+        const int n_right = nt * (int)cdiv(k - j0, 128);
+        rank_update_kernel<<<(unsigned)(n_low + n_right), 256, 0, s>>>(U, k, j0, b, n_low,
+                                                                       d_info);
+        GPTQ_CHECK_LAUNCH();
+      }
     }
   }
   {

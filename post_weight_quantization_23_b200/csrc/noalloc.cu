@@ -6,13 +6,14 @@
 // output buffers, a process that has carved all device memory into its own
 // arena up front (so a new allocation would fail or fragment it), or a
 // runtime that forbids allocation after start-up.  This entry point runs the
-// same kernels as gptq_prepare_hinv, but its scratch lives in a file-scope
+// same computation as gptq_prepare_hinv, but its scratch lives in a file-scope
 // __device__ array that the CUDA runtime creates when the library's device
 // code is loaded, so the call itself allocates nothing.
 //
 // The array is `kScratchBytes` (4 MiB) on every device that loads the
 // library and is held until the process exits; it covers k up to
-// kNoAllocMaxK = 12288.  All calls share it and it keeps the previous call's
+// kNoAllocMaxK = 12288 (when the tensor-core update's operand splits do not
+// fit as well, the CUDA-core update is used).  All calls share it and it keeps the previous call's
 // contents; the Cholesky stages write every scratch word before reading it,
 // so nothing needs clearing.  Calls whose work overlaps on the GPU (two
 // streams, or two host threads) race on the array: serialise them.
@@ -26,10 +27,10 @@
 #include "common.cuh"
 
 namespace gptq {
-size_t hinv_workspace_bytes(int64_t k);
+size_t hinv_workspace_min_bytes(int64_t k);
 gptq_status prepare_hinv_impl(const float* H, int64_t k, const gptq_config* cfg, float* U,
                               int32_t* perm, int32_t* invperm, uint8_t* dead, int32_t* d_info,
-                              void* ws, cudaStream_t s);
+                              void* ws, size_t ws_bytes, cudaStream_t s);
 }  // namespace gptq
 
 namespace {
@@ -71,10 +72,10 @@ extern "C" gptq_status gptq_prepare_hinv_noalloc(const float* H, int64_t k,
   if (!(cfg->percdamp >= 0.0f) || !isfinite(cfg->percdamp)) return GPTQ_ERR_INVALID_ARG;
   if ((const void*)H == (const void*)U) return GPTQ_ERR_INVALID_ARG;
   // sizes beyond the built-in scratch
-  if (k > kNoAllocMaxK || gptq::hinv_workspace_bytes(k) > kScratchBytes) return GPTQ_ERR_WORKSPACE;
+  if (k > kNoAllocMaxK || gptq::hinv_workspace_min_bytes(k) > kScratchBytes) return GPTQ_ERR_WORKSPACE;
   void* ws = nullptr;
   gptq_status st = scratch_address(&ws);
   if (st != GPTQ_OK) return st;
-  return gptq::prepare_hinv_impl(H, k, cfg, U, perm, invperm, dead, d_info, ws,
+  return gptq::prepare_hinv_impl(H, k, cfg, U, perm, invperm, dead, d_info, ws, kScratchBytes,
                                  (cudaStream_t)stream);
 }

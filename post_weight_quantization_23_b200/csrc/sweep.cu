@@ -11,7 +11,9 @@
 //                   block compensation immediately), and the remaining columns
 //                   of the block get the sub-block's errors as one rank-SB
 //                   update, each thread of the row taking every fourth column;
-//   (trailing)      W[:, e:] -= Err * U[s:e, e:]  (fp32 GEMM).
+//   (trailing)      W[:, e:] -= Err * U[s:e, e:]: on the tensor cores in
+//                   fp32-accurate 3xTF32 (tf32x3.cu) when k % 4 == 0, else an
+//                   fp32 CUDA-core GEMM.
 // The layer loss is accumulated inside the block kernel through the Optimal
 // Brain Surgeon accounting: fixing column i and compensating the later ones
 // raises (w - q) Hd (w - q)^T by err_i^2, so per row
@@ -29,26 +31,51 @@ constexpr int SW_THREADS = 128;
 constexpr int SW_LDW = 40;            // sW column stride: 32 rows + 8 pad (conflict-free quads)
 constexpr int SW_LDU = SW_MAX_B + 4;  // UtS column stride
 constexpr size_t SW_SMEM = sizeof(float) * ((size_t)SW_MAX_B * SW_LDU + (size_t)SW_MAX_B * SW_LDW +
-                                            SW_MAX_B);
+                                            SW_MAX_B) +
+                           sizeof(int32_t) * SW_MAX_B;
+
+bool tc_update_supported(int64_t k);
+gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float* hi,
+                               float* lo, int64_t ldo, cudaStream_t s);
+gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* u_hi,
+                              const float* u_lo, float* Wt, int r, int k, int s0, int e,
+                              int32_t* d_status, cudaStream_t s);
 
 struct SweepScratch {
   float* Wt;      // [r * k] working weights, processing order
-  float* Err;     // [r * B]
+  float* Err;     // [r * B] errors of the current block (tf32 high part on the tensor-core path)
+  float* Err_lo;  // [r * B] tf32 low part (tensor-core path)
+  float* U_hi;    // [k * k] tf32 split of U^T (tensor-core path)
+  float* U_lo;    // [k * k]
   float* lambda;  // [1] damping added to the Hessian diagonal (for the loss)
 };
 
 size_t sweep_workspace_bytes(int64_t r, int64_t k, int B) {
-  return align256(sizeof(float) * (size_t)r * k) + align256(sizeof(float) * (size_t)r * B) +
-         align256(sizeof(float));
+  size_t b = align256(sizeof(float) * (size_t)r * k) + 2 * align256(sizeof(float) * (size_t)r * B) +
+             align256(sizeof(float));
+  if (tc_update_supported(k)) b += 2 * align256(sizeof(float) * (size_t)k * k);
+  return b;
 }
 
-static SweepScratch carve_sweep(void* ws, int64_t r, int64_t k, int B) {
+static SweepScratch carve_sweep(void* ws, int64_t r, int64_t k, int B, bool tc) {
   char* p = (char*)ws;
   SweepScratch s;
   s.Wt = (float*)p; p += align256(sizeof(float) * (size_t)r * k);
   s.Err = (float*)p; p += align256(sizeof(float) * (size_t)r * B);
-  s.lambda = (float*)p;
+  s.Err_lo = (float*)p; p += align256(sizeof(float) * (size_t)r * B);
+  s.lambda = (float*)p; p += align256(sizeof(float));
+  s.U_hi = tc ? (float*)p : nullptr;
+  if (tc) p += align256(sizeof(float) * (size_t)k * k);
+  s.U_lo = tc ? (float*)p : nullptr;
   return s;
+}
+
+// hi = x rounded to tf32 (nearest, ties away), lo = x - hi
+__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
+  uint32_t h;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+  hi = __uint_as_float(h);
+  lo = x - hi;
 }
 
 template <typename T>
@@ -127,7 +154,8 @@ __global__ void group_grid_kernel(const float* __restrict__ Wt, int r, int k, in
 template <int SB, typename T>
 __global__ void __launch_bounds__(SW_THREADS)
 sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
-                   const float* __restrict__ U, const int32_t* __restrict__ perm,
+                   float* __restrict__ Err_lo, const float* __restrict__ U,
+                   const int32_t* __restrict__ perm,
                    const uint8_t* __restrict__ dead, const T* __restrict__ W0, int64_t ldw, int r,
                    int k, int s, int bw, int B, int G, int ngroups, float maxq,
                    const float* __restrict__ lambda, float* __restrict__ scales,
@@ -137,6 +165,7 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
   float* UtS = sm_sweep;                           // UtS[j * LDU + i] = U[s+i][s+j], i <= j
   float* sW = UtS + SW_MAX_B * SW_LDU;             // sW[j * LDW + rr] = W[r0+rr][s+j]
   float* rdg = sW + SW_MAX_B * SW_LDW;             // 1 / U[s+i][s+i]
+  int32_t* pcol = (int32_t*)(rdg + SW_MAX_B);      // perm[s + i]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int q = lane & 3;
   const int rr = warp * 8 + (lane >> 2);
@@ -152,7 +181,10 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
     const int gr = r0 + r2;
     sW[j * SW_LDW + r2] = (gr < r) ? Wt[(int64_t)gr * k + s + j] : 0.f;
   }
-  for (int i = tid; i < bw; i += SW_THREADS) rdg[i] = 1.0f / U[(int64_t)(s + i) * k + s + i];
+  for (int i = tid; i < bw; i += SW_THREADS) {
+    rdg[i] = 1.0f / U[(int64_t)(s + i) * k + s + i];
+    pcol[i] = perm[s + i];
+  }
   __syncthreads();
 
   float scale = 1.f, zero = 0.f;
@@ -190,6 +222,19 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
         zeros[(int64_t)row * ngroups + (s + c0) / G] = (int32_t)zero;
       }
     }
+    // original weights of the columns this thread reports (ii % 4 == q),
+    // fetched before the column chain so their latency overlaps it
+    constexpr int NQ = (SB + 3) / 4;
+    float w0r[NQ];
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+      const int ii = 4 * u + q;
+      w0r[u] = 0.f;
+      if (loss != nullptr && valid && ii < SB && c0 + ii < bw) {
+        const int oc = pcol[c0 + ii];
+        w0r[u] = dead[oc] ? 0.f : to_f32(W0[(int64_t)row * ldw + oc]);
+      }
+    }
     float errs[SB];
 #pragma unroll
     for (int ii = 0; ii < SB; ++ii) {
@@ -207,11 +252,10 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
         const float qv = scale * (c - zero);
         err = (wv - qv) * rdg[col];
         if (valid && (ii & 3) == q) {
-          const int oc = perm[s + col];
+          const int oc = pcol[col];
           codes[(int64_t)row * k + oc] = (uint8_t)c;
           if (loss != nullptr) {
-            const float w0 = dead[oc] ? 0.f : to_f32(W0[(int64_t)row * ldw + oc]);
-            const double dd = (double)w0 - (double)qv;
+            const double dd = (double)w0r[ii >> 2] - (double)qv;
             d2 += dd * dd;
             e2 += (double)err * (double)err;
           }
@@ -233,7 +277,16 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
     if (valid) {
 #pragma unroll
       for (int ii = 0; ii < SB; ++ii)
-        if ((ii & 3) == q && c0 + ii < bw) Err[(int64_t)row * B + c0 + ii] = errs[ii];
+        if ((ii & 3) == q && c0 + ii < bw) {
+          if (Err_lo != nullptr) {
+            float h, l;
+            split_tf32(errs[ii], h, l);
+            Err[(int64_t)row * B + c0 + ii] = h;
+            Err_lo[(int64_t)row * B + c0 + ii] = l;
+          } else {
+            Err[(int64_t)row * B + c0 + ii] = errs[ii];
+          }
+        }
     }
     __syncwarp();
   }
@@ -263,7 +316,7 @@ __global__ void loss_total_kernel(double* __restrict__ loss, int r) {
 
 template <int SB, typename T>
 static void launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* Err,
-                         const float* U, const int32_t* perm, const uint8_t* dead, const T* W0,
+                         float* Err_lo, const float* U, const int32_t* perm, const uint8_t* dead, const T* W0,
                          int64_t ldw, int r, int k, int s0, int bw, int B, int G, int ngroups,
                          float maxq, const float* lambda, float* scales, int32_t* zeros,
                          uint8_t* codes, double* loss, int32_t* d_status) {
@@ -274,7 +327,7 @@ static void launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* 
     attr = true;
   }
   sweep_block_kernel<SB, T><<<grid, SW_THREADS, SW_SMEM, s>>>(
-      Wt, Err, U, perm, dead, W0, ldw, r, k, s0, bw, B, G, ngroups, maxq, lambda, scales, zeros,
+      Wt, Err, Err_lo, U, perm, dead, W0, ldw, r, k, s0, bw, B, G, ngroups, maxq, lambda, scales, zeros,
       codes, loss, d_status);
 }
 
@@ -288,7 +341,8 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
   const int G = cfg->group_size == -1 ? k : cfg->group_size;
   const int ngroups = (int)cdiv(k, G);
   const float maxq = (float)((1 << cfg->bits) - 1);
-  SweepScratch sc = carve_sweep(ws, r, k, B);
+  const bool tc = tc_update_supported(k);
+  SweepScratch sc = carve_sweep(ws, r, k, B, tc);
   const bool want_loss = (H0 != nullptr && loss != nullptr);
   double* lossp = want_loss ? loss : nullptr;
   {
@@ -300,6 +354,10 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
   if (want_loss) {
     sweep_lambda_kernel<<<1, 1024, 0, s>>>(H0, k, cfg->percdamp, sc.lambda);
     GPTQ_CHECK_LAUNCH();
+  }
+  if (tc) {
+    gptq_status st = tc_split_transpose(U, k, k, k, sc.U_hi, sc.U_lo, k, s);
+    if (st != GPTQ_OK) return st;
   }
   // sub-block width: 16, or the largest power of two dividing a smaller group
   int SB = 16;
@@ -318,7 +376,7 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     }
     const float* lam = want_loss ? sc.lambda : nullptr;
 #define GPTQ_SWEEP_BLOCK(SBV)                                                                     \
-  launch_block<SBV, T>(grid, s, sc.Wt, sc.Err, U, perm, dead, W, ldw, r, k, s0, bw, B, G, ngroups, \
+  launch_block<SBV, T>(grid, s, sc.Wt, sc.Err, tc ? sc.Err_lo : nullptr, U, perm, dead, W, ldw, r, k, s0, bw, B, G, ngroups, \
                        maxq, lam, scales, zeros, codes, lossp, d_status)
     switch (SB) {
       case 16: GPTQ_SWEEP_BLOCK(16); break;
@@ -331,10 +389,16 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     GPTQ_CHECK_LAUNCH();
     int e0 = s0 + bw;
     if (e0 < k) {
-      sgemm<false, false, false, false, false>(r, k - e0, bw, -1.0f, sc.Err, B,
-                                               U + (int64_t)s0 * k + e0, k, 1.0f, sc.Wt + e0, k,
-                                               nullptr, s);
-      GPTQ_CHECK_LAUNCH();
+      if (tc) {
+        gptq_status st = tc_sweep_trailing(sc.Err, sc.Err_lo, B, sc.U_hi, sc.U_lo, sc.Wt, r, k,
+                                           s0, e0, d_status, s);
+        if (st != GPTQ_OK) return st;
+      } else {
+        sgemm<false, false, false, false, false>(r, k - e0, bw, -1.0f, sc.Err, B,
+                                                 U + (int64_t)s0 * k + e0, k, 1.0f, sc.Wt + e0, k,
+                                                 nullptr, s);
+        GPTQ_CHECK_LAUNCH();
+      }
     }
   }
   if (want_loss) {

@@ -1,0 +1,432 @@
+// fp32-accurate short-K updates on the 5th-generation tensor cores:
+//   D[m][n] += sign(n) * sum_k A[m][k] B[k][n]        (K <= 128)
+// with every fp32 operand split as x = hi + lo, hi = x rounded to tf32 and
+// lo = x - hi (exact), and three kind::tf32 MMAs per K step,
+//   A B ~= A_hi B_hi + A_hi B_lo + A_lo B_hi,
+// which keeps fp32-level accuracy (the dropped A_lo B_lo term and the tf32
+// rounding of lo are ~2^-21 relative).  The splits are written to global
+// memory, K-major (K contiguous) for both operands -- a transposing split
+// where the source is stored the other way -- so TMA brings hi and lo boxes
+// straight into shared memory in the 128-byte-swizzled K-major layout.
+//
+// Two uses:
+//   mode 0, lazy-batch trailing update of the GPTQ sweep ([GPTQ-tool]
+//     "GPTQ" How it works Step 7): W[:, e:] -= Err * U[s:s+B, e:], with Err
+//     (rows x B) and U^T (the transposed split of the k x k factor).
+//   mode 1, rank-b update of the inverse factor: rows [0, j0) of the work
+//     matrix += sign * R^T R', with R = A[j0:j0+b, :] split transposed into
+//     R^T (k x 64); columns c < j0 are the Schur complement (sign -1, lower
+//     triangle only), columns c >= j0 the Y update (sign +1).
+//
+// Tiles of 128 x 256 (M x N) on a persistent grid; warp 0 issues TMA, warp 1
+// the MMAs (one thread), warps 2..5 read TMEM and update D in place.  TMEM
+// holds two accumulators, so a tile's epilogue overlaps the next tile's
+// MMAs.  Every mbarrier wait is bounded; on a timeout the CTA drains its
+// own copies and MMAs, frees TMEM and raises *status.
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace gptq {
+
+namespace {
+
+constexpr int TX_M = 128, TX_N = 256, TX_KC = 32;   // tile rows, cols, K per stage
+constexpr int TX_STAGES = 2;
+constexpr int TX_A_BYTES = TX_M * TX_KC * 4;         // 16 KB
+constexpr int TX_B_BYTES = TX_N * TX_KC * 4;         // 32 KB
+constexpr int TX_STAGE_BYTES = 2 * TX_A_BYTES + 2 * TX_B_BYTES;  // hi + lo of both: 96 KB
+constexpr int TX_THREADS = 192;                      // TMA, MMA, 4 epilogue warps
+constexpr int TX_TMEM_COLS = 512;
+constexpr int TX_EPI_BYTES = 4 * 32 * 33 * 4;             // per-warp 32 x 32 transpose tiles
+constexpr size_t TX_SMEM = (size_t)TX_STAGES * TX_STAGE_BYTES + TX_EPI_BYTES + 1024 + 256;
+
+struct TxArgs {
+  float* D;
+  int64_t ldd;
+  int M, N;        // output extent from (row0, col0)
+  int row0, col0;  // output offsets in D
+  int K;           // inner extent
+  int a_k0, a_r0;  // A map coordinates of (k = 0, output row 0)
+  int b_k0, b_r0;  // B map coordinates of (k = 0, output column 0)
+  int ntm, ntiles;
+  int mode, split;
+  int32_t* status;
+  int32_t status_code;
+};
+
+__device__ __forceinline__ bool tile_skipped(const TxArgs& a, int m0, int n0) {
+  // mode 1: a tile whose columns all lie in [0, split) and strictly above the
+  // diagonal of its rows has nothing to update
+  return a.mode == 1 && n0 + TX_N <= a.split && n0 >= m0 + TX_M;
+}
+
+__global__ void __launch_bounds__(TX_THREADS, 1)
+tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
+                     const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
+                     TxArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  float* epi = (float*)(smem + TX_STAGES * TX_STAGE_BYTES);
+  uint64_t* bars = (uint64_t*)(smem + TX_STAGES * TX_STAGE_BYTES + TX_EPI_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + TX_STAGES;
+  uint64_t* tfull = bars + 2 * TX_STAGES;
+  uint64_t* tempty = bars + 2 * TX_STAGES + 2;
+  uint64_t* done = bars + 2 * TX_STAGES + 4;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * TX_STAGES + 5);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < TX_STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&tfull[b], 1);
+      tc::mbar_init(&tempty[b], 4);
+    }
+    tc::mbar_init(done, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+    tc::prefetch_tensormap(&a_hi);
+    tc::prefetch_tensormap(&a_lo);
+    tc::prefetch_tensormap(&b_hi);
+    tc::prefetch_tensormap(&b_lo);
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_slot, TX_TMEM_COLS);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nkc = (a.K + TX_KC - 1) / TX_KC;
+  const uint32_t idesc = tc::instr_desc(2, TX_M, TX_N, 0, 0);  // both operands K-major
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued[TX_STAGES];
+      uint32_t issued_parity[TX_STAGES];
+      for (int s = 0; s < TX_STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < a.ntiles && ok; t += gridDim.x) {
+        const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
+        if (tile_skipped(a, m0, n0)) continue;
+        for (int kc = 0; kc < nkc; ++kc) {
+          if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* sb = smem + (size_t)stage * TX_STAGE_BYTES;
+          tc::mbar_arrive_expect_tx(&full[stage], TX_STAGE_BYTES);
+          const int k0 = kc * TX_KC;
+          tc::tma_load_2d(sb, &a_hi, &full[stage], a.a_k0 + k0, a.a_r0 + m0);
+          tc::tma_load_2d(sb + TX_A_BYTES, &a_lo, &full[stage], a.a_k0 + k0, a.a_r0 + m0);
+          uint8_t* bb = sb + 2 * TX_A_BYTES;
+          tc::tma_load_2d(bb, &b_hi, &full[stage], a.b_k0 + k0, a.b_r0 + n0);
+          tc::tma_load_2d(bb + TX_B_BYTES, &b_lo, &full[stage], a.b_k0 + k0, a.b_r0 + n0);
+          issued[stage] = true;
+          issued_parity[stage] = phase;
+          if (++stage == TX_STAGES) stage = 0, phase ^= 1u;
+        }
+      }
+      if (!ok || *abort_flag) {
+        for (int s = 0; s < TX_STAGES; ++s)
+          if (issued[s])
+            for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
+              if (tc::mbar_try_wait(&full[s], issued_parity[s])) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int tb = 0;
+      uint32_t tphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < a.ntiles && ok; t += gridDim.x) {
+        const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
+        if (tile_skipped(a, m0, n0)) continue;
+        if (!tc::mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint32_t dcol = tmem + (uint32_t)(tb * TX_N);
+        for (int kc = 0; kc < nkc; ++kc) {
+          if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t sb = tc::smem_u32(smem + (size_t)stage * TX_STAGE_BYTES);
+          const uint32_t ah = sb, al = sb + TX_A_BYTES;
+          const uint32_t bh = sb + 2 * TX_A_BYTES, bl = bh + TX_B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TX_KC / 8; ++kk) {
+            // K-major, 128-byte swizzle: 8-row groups 1024 B apart, K step 32 B
+            const uint64_t dah = tc::smem_desc_sw128(ah + kk * 32, 16, 1024);
+            const uint64_t dal = tc::smem_desc_sw128(al + kk * 32, 16, 1024);
+            const uint64_t dbh = tc::smem_desc_sw128(bh + kk * 32, 16, 1024);
+            const uint64_t dbl = tc::smem_desc_sw128(bl + kk * 32, 16, 1024);
+            const uint32_t acc0 = (kc > 0 || kk > 0) ? 1u : 0u;
+            tc::mma_tf32_ss(dcol, dal, dbh, idesc, acc0);  // small terms first
+            tc::mma_tf32_ss(dcol, dah, dbl, idesc, 1u);
+            tc::mma_tf32_ss(dcol, dah, dbh, idesc, 1u);
+          }
+          tc::mma_commit(&empty[stage]);
+          if (++stage == TX_STAGES) stage = 0, phase ^= 1u;
+        }
+        if (!ok) break;
+        tc::mma_commit(&tfull[tb]);
+        if (++tb == 2) tb = 0, tphase ^= 1u;
+      }
+      tc::mma_commit(done);
+      for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
+        if (tc::mbar_try_wait(done, 0)) break;
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31 = tile rows; each
+    // 32 x 32 chunk goes through shared memory so that every update of D
+    // touches 32 consecutive columns of one row (one 128-byte line)
+    const int quarter = warp & 3;
+    float* tbuf = epi + (warp - 2) * 32 * 33;
+    int tb = 0;
+    uint32_t tphase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < a.ntiles && ok; t += gridDim.x) {
+      const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
+      if (tile_skipped(a, m0, n0)) continue;
+      if (!tc::mbar_wait(&tfull[tb], tphase, abort_flag)) { ok = false; break; }
+      tc::tc_fence_after();
+      for (int cc = 0; cc < TX_N / 32; ++cc) {
+        float v[32];
+        tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(tb * TX_N + cc * 32), v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) tbuf[lane * 33 + q] = v[q];
+        __syncwarp();
+        const int col = n0 + cc * 32 + lane;  // relative output column of this lane
+        const int c = a.col0 + col;           // absolute column
+        const int gm0 = m0 + quarter * 32;    // first relative row of this warp
+        // all 32 loads first (independent), then the updates and stores
+        float dv[32];
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+          const bool okr = (gm0 + rr < a.M) && (col < a.N);
+          dv[rr] = okr ? a.D[(int64_t)(a.row0 + gm0 + rr) * a.ldd + c] : 0.f;
+        }
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+          const int gm = gm0 + rr;
+          if (gm < a.M && col < a.N) {
+            const float val = tbuf[rr * 33 + lane];
+            float out;
+            bool wr = true;
+            if (a.mode == 0) out = dv[rr] - val;
+            else if (c >= a.split) out = dv[rr] + val;
+            else if (c <= a.row0 + gm) out = dv[rr] - val;
+            else { out = dv[rr]; wr = false; }
+            if (wr) a.D[(int64_t)(a.row0 + gm) * a.ldd + c] = out;
+          }
+        }
+        __syncwarp();
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty[tb]);
+      if (++tb == 2) tb = 0, tphase ^= 1u;
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0 && a.status != nullptr) atomicCAS(a.status, 0, a.status_code);
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tmem, TX_TMEM_COLS);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// fp32 2-D map (cols inner, rows outer), row stride ld floats, box {32, box_rows}.
+bool make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int64_t ld,
+              uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld * 4};
+  cuuint32_t box[2] = {32, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), gdim, gstride, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+gptq_status launch(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMap& bh,
+                   const CUtensorMap& bl, TxArgs& a, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(tf32x3_update_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TX_SMEM) != cudaSuccess)
+      return GPTQ_ERR_CUDA;
+    attr = true;
+  }
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::min(a.ntiles, nsm);
+  if (grid <= 0) return GPTQ_OK;
+  tf32x3_update_kernel<<<grid, TX_THREADS, TX_SMEM, s>>>(ah, al, bh, bl, a);
+  GPTQ_CHECK_LAUNCH();
+  return GPTQ_OK;
+}
+
+
+// hi = x rounded to tf32 (nearest, ties away), lo = x - hi
+__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
+  uint32_t h;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+  hi = __uint_as_float(h);
+  lo = x - hi;
+}
+
+// dst[c][r] = split(src[r][c]) for r < rows, c < cols (32 x 32 tiles
+// through shared memory, so both the reads and the writes are coalesced).
+__global__ void split_transpose_kernel(const float* __restrict__ src, int64_t lds, int rows,
+                                       int cols, float* __restrict__ hi, float* __restrict__ lo,
+                                       int64_t ldo) {
+  __shared__ float tile[32][33];
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  for (int y = ty; y < 32; y += 8) {
+    const int r = r0 + y, c = c0 + tx;
+    tile[y][tx] = (r < rows && c < cols) ? src[(int64_t)r * lds + c] : 0.f;
+  }
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int c = c0 + y, r = r0 + tx;
+    if (c < cols && r < rows) {
+      float h, l;
+      split_tf32(tile[tx][y], h, l);
+      hi[(int64_t)c * ldo + r] = h;
+      lo[(int64_t)c * ldo + r] = l;
+    }
+  }
+}
+
+// Rt[c][m] = split(R[m][c]), R = A[j0:j0+b, :] with the diagonal block read as
+// upper triangular (its lower part holds stale values); m in [b, 64) is 0.
+__global__ void split_rowblock_t_kernel(const float* __restrict__ A, int k, int j0, int b,
+                                        float* __restrict__ hi, float* __restrict__ lo,
+                                        const int32_t* __restrict__ d_info) {
+  if (*d_info != 0) return;
+  __shared__ float tile[64][33];
+  const int c0 = blockIdx.x * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  for (int m = ty; m < 64; m += 8) {
+    const int c = c0 + tx;
+    float x = 0.f;
+    if (m < b && c < k) {
+      x = A[(int64_t)(j0 + m) * k + c];
+      if (c >= j0 && c < j0 + b && c - j0 < m) x = 0.f;
+    }
+    tile[m][tx] = x;
+  }
+  __syncthreads();
+  for (int cc = ty; cc < 32; cc += 8) {
+    const int c = c0 + cc;
+    if (c >= k) continue;
+    for (int m = tx; m < 64; m += 32) {
+      float h, l;
+      split_tf32(tile[m][cc], h, l);
+      hi[(int64_t)c * 64 + m] = h;
+      lo[(int64_t)c * 64 + m] = l;
+    }
+  }
+}
+
+}  // namespace
+
+bool tc_update_supported(int64_t k) { return k % 4 == 0 && encode_fn() != nullptr; }
+
+gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float* hi,
+                               float* lo, int64_t ldo, cudaStream_t s) {
+  if (rows <= 0 || cols <= 0) return GPTQ_OK;
+  dim3 grid((unsigned)cdiv(cols, 32), (unsigned)cdiv(rows, 32));
+  split_transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(src, lds, rows, cols, hi, lo, ldo);
+  GPTQ_CHECK_LAUNCH();
+  return GPTQ_OK;
+}
+
+// Wt[0:r, e:k] -= Err[0:r, 0:B] * U[s:s+B, e:k]   (Err_hi/lo: r x B, ld B;
+// Ut_hi/lo: the transposed split of U, k x k).  A timeout sets
+// *d_status = GPTQ_ERR_TIMEOUT.
+gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* ut_hi,
+                              const float* ut_lo, float* Wt, int r, int k, int s0, int e,
+                              int32_t* d_status, cudaStream_t s) {
+  CUtensorMap ah, al, bh, bl;
+  if (!make_map(&ah, err_hi, B, r, B, TX_M) || !make_map(&al, err_lo, B, r, B, TX_M) ||
+      !make_map(&bh, ut_hi, k, k, k, TX_N) || !make_map(&bl, ut_lo, k, k, k, TX_N))
+    return GPTQ_ERR_INVALID_ARG;
+  TxArgs a;
+  a.D = Wt;
+  a.ldd = k;
+  a.M = r;
+  a.N = k - e;
+  a.row0 = 0;
+  a.col0 = e;
+  a.K = B;
+  a.a_k0 = 0;
+  a.a_r0 = 0;
+  a.b_k0 = s0;
+  a.b_r0 = e;
+  a.ntm = (int)cdiv(r, TX_M);
+  a.ntiles = a.ntm * (int)cdiv(k - e, TX_N);
+  a.mode = 0;
+  a.split = 0;
+  a.status = d_status;
+  a.status_code = GPTQ_ERR_TIMEOUT;
+  return launch(ah, al, bh, bl, a, s);
+}
+
+// Rows [0, j0) of the k x k work matrix A += sign * R^T R (see the file
+// comment), R = A[j0:j0+b, :] split transposed into rt_hi / rt_lo (k x 64
+// scratch).  A timeout sets *d_info = k + 1.
+gptq_status tc_rank_update(float* A, int k, int j0, int b, float* rt_hi, float* rt_lo,
+                           int32_t* d_info, cudaStream_t s) {
+  split_rowblock_t_kernel<<<(unsigned)cdiv(k, 32), dim3(32, 8), 0, s>>>(A, k, j0, b, rt_hi, rt_lo,
+                                                                        d_info);
+  GPTQ_CHECK_LAUNCH();
+  CUtensorMap ah, al, bh, bl;
+  if (!make_map(&ah, rt_hi, 64, k, 64, TX_M) || !make_map(&al, rt_lo, 64, k, 64, TX_M) ||
+      !make_map(&bh, rt_hi, 64, k, 64, TX_N) || !make_map(&bl, rt_lo, 64, k, 64, TX_N))
+    return GPTQ_ERR_INVALID_ARG;
+  TxArgs a;
+  a.D = A;
+  a.ldd = k;
+  a.M = j0;
+  a.N = k;
+  a.row0 = 0;
+  a.col0 = 0;
+  a.K = b;
+  a.a_k0 = 0;
+  a.a_r0 = 0;
+  a.b_k0 = 0;
+  a.b_r0 = 0;
+  a.ntm = (int)cdiv(j0, TX_M);
+  a.ntiles = a.ntm * (int)cdiv(k, TX_N);
+  a.mode = 1;
+  a.split = j0;
+  a.status = d_info;
+  a.status_code = k + 1;
+  return launch(ah, al, bh, bl, a, s);
+}
+
+}  // namespace gptq
