@@ -20,8 +20,11 @@
 //   (w0 - q) H0 (w0 - q)^T = sum_i err_i^2 - lambda * sum_i (w0_i - q_i)^2
 // (H0 = Hd - lambda I, dead columns count with w0 = 0); no k x k product.
 // The fp32 working copy Wt (processing order) lives in the workspace.
+#include <algorithm>
+
 #include "common.cuh"
 #include "sgemm.cuh"
+#include "tc_ptx.cuh"
 
 namespace gptq {
 
@@ -33,6 +36,29 @@ constexpr int SW_LDU = SW_MAX_B + 4;  // UtS column stride
 constexpr size_t SW_SMEM = sizeof(float) * ((size_t)SW_MAX_B * SW_LDU + (size_t)SW_MAX_B * SW_LDW +
                                             SW_MAX_B) +
                            sizeof(int32_t) * SW_MAX_B;
+
+// Layout of the lane kernel for L lanes per row (L = 4 or 8): S = 128 / L
+// slots per lane, record segments of S + 4 floats (the pad spreads the lanes'
+// float4 reads over distinct banks).
+template <int L> struct SqLayout {
+  static constexpr int S = SW_MAX_B / L;             // slots (columns) per lane
+  static constexpr int SEG = S + 4;                  // floats per (column, lane) segment
+  static constexpr int LDI = L * SEG;                // floats per column of Uq
+  static constexpr int UQ = SW_MAX_B * LDI;
+  static constexpr int UD = (SW_MAX_B / L) * L * L;  // diagonal L x L tiles
+  static constexpr size_t REC_BYTES =
+      sizeof(float) * ((size_t)UQ + UD + SW_MAX_B) + sizeof(int32_t) * SW_MAX_B;
+  static constexpr size_t SMEM = REC_BYTES + 64;
+  static constexpr int ROWS_PER_WARP = 32 / L;
+};
+constexpr int SQ_MAX_WARPS = 12;
+constexpr uint32_t SQ_COPY_CHUNK = 16384;
+constexpr size_t SQ_REC_MAX = SqLayout<8>::REC_BYTES > SqLayout<4>::REC_BYTES
+                                  ? SqLayout<8>::REC_BYTES
+                                  : SqLayout<4>::REC_BYTES;
+
+// per-block records of the lane kernel (one per lazy block)
+static size_t sweep_records_bytes(int64_t k, int B) { return (size_t)cdiv(k, B) * SQ_REC_MAX; }
 
 bool tc_update_supported(int64_t k);
 gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float* hi,
@@ -48,11 +74,12 @@ struct SweepScratch {
   float* U_hi;    // [k * k] tf32 split of U^T (tensor-core path)
   float* U_lo;    // [k * k]
   float* lambda;  // [1] damping added to the Hessian diagonal (for the loss)
+  uint8_t* rec;   // per-block records of the 4-lanes-per-row kernel
 };
 
 size_t sweep_workspace_bytes(int64_t r, int64_t k, int B) {
   size_t b = align256(sizeof(float) * (size_t)r * k) + 2 * align256(sizeof(float) * (size_t)r * B) +
-             align256(sizeof(float));
+             align256(sizeof(float)) + align256(sweep_records_bytes(k, B));
   if (tc_update_supported(k)) b += 2 * align256(sizeof(float) * (size_t)k * k);
   return b;
 }
@@ -64,6 +91,7 @@ static SweepScratch carve_sweep(void* ws, int64_t r, int64_t k, int B, bool tc) 
   s.Err = (float*)p; p += align256(sizeof(float) * (size_t)r * B);
   s.Err_lo = (float*)p; p += align256(sizeof(float) * (size_t)r * B);
   s.lambda = (float*)p; p += align256(sizeof(float));
+  s.rec = (uint8_t*)p; p += align256(sweep_records_bytes(k, B));
   s.U_hi = tc ? (float*)p : nullptr;
   if (tc) p += align256(sizeof(float) * (size_t)k * k);
   s.U_lo = tc ? (float*)p : nullptr;
@@ -151,14 +179,12 @@ __global__ void group_grid_kernel(const float* __restrict__ Wt, int r, int k, in
 // SIMT issues it once); the rank-SB updates of the rest of the block and the
 // outputs are split by q.  SB divides the group size when groups are smaller
 // than the block, so a group always starts at a sub-block boundary.
-template <int SB, typename T>
+template <int SB>
 __global__ void __launch_bounds__(SW_THREADS)
 sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
                    float* __restrict__ Err_lo, const float* __restrict__ U,
-                   const int32_t* __restrict__ perm,
-                   const uint8_t* __restrict__ dead, const T* __restrict__ W0, int64_t ldw, int r,
-                   int k, int s, int bw, int B, int G, int ngroups, float maxq,
-                   const float* __restrict__ lambda, float* __restrict__ scales,
+                   const int32_t* __restrict__ perm, int r, int k, int s, int bw, int B, int G,
+                   int ngroups, float maxq, float* __restrict__ scales,
                    int32_t* __restrict__ zeros, uint8_t* __restrict__ codes,
                    double* __restrict__ loss, int32_t* __restrict__ d_status) {
   extern __shared__ float sm_sweep[];
@@ -193,8 +219,7 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
     scale = scales[(int64_t)row * ngroups + g];
     zero = (float)zeros[(int64_t)row * ngroups + g];
   }
-  const float lam = (lambda != nullptr) ? *lambda : 0.f;
-  double e2 = 0.0, d2 = 0.0;
+  double e2 = 0.0;
   bool nonfinite = false;
 
   for (int c0 = 0; c0 < bw; c0 += SB) {
@@ -222,19 +247,6 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
         zeros[(int64_t)row * ngroups + (s + c0) / G] = (int32_t)zero;
       }
     }
-    // original weights of the columns this thread reports (ii % 4 == q),
-    // fetched before the column chain so their latency overlaps it
-    constexpr int NQ = (SB + 3) / 4;
-    float w0r[NQ];
-#pragma unroll
-    for (int u = 0; u < NQ; ++u) {
-      const int ii = 4 * u + q;
-      w0r[u] = 0.f;
-      if (loss != nullptr && valid && ii < SB && c0 + ii < bw) {
-        const int oc = pcol[c0 + ii];
-        w0r[u] = dead[oc] ? 0.f : to_f32(W0[(int64_t)row * ldw + oc]);
-      }
-    }
     float errs[SB];
 #pragma unroll
     for (int ii = 0; ii < SB; ++ii) {
@@ -254,11 +266,7 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
         if (valid && (ii & 3) == q) {
           const int oc = pcol[col];
           codes[(int64_t)row * k + oc] = (uint8_t)c;
-          if (loss != nullptr) {
-            const double dd = (double)w0r[ii >> 2] - (double)qv;
-            d2 += dd * dd;
-            e2 += (double)err * (double)err;
-          }
+          if (loss != nullptr) e2 += (double)err * (double)err;
         }
       }
       errs[ii] = err;
@@ -292,12 +300,309 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
   }
   if (loss != nullptr) {
     e2 += __shfl_xor_sync(0xffffffffu, e2, 1);
-    d2 += __shfl_xor_sync(0xffffffffu, d2, 1);
     e2 += __shfl_xor_sync(0xffffffffu, e2, 2);
-    d2 += __shfl_xor_sync(0xffffffffu, d2, 2);
-    if (valid && q == 0) atomicAdd(&loss[row], e2 - (double)lam * d2);
+    if (valid && q == 0) loss[row] += e2;
   }
   if (nonfinite && valid && d_status != nullptr) atomicCAS(d_status, 0, (int32_t)GPTQ_ERR_NONFINITE);
+}
+
+// rint(w / scale) with the IEEE quotient.
+__device__ __noinline__ float rint_exact_div(float w, float scale) {
+  return rintf(__fdiv_rn(w, scale));
+}
+
+// ---- the lane block kernel ----------------------------------------------------
+//
+// L lanes per row (L = 8 or 4).  Lane l owns the block columns l + L j
+// (j = 0 .. S-1, S = 128 / L), held in registers w[]; after each sub-block of L
+// columns the registers shift down by one, so w[0] is always the current
+// sub-block and the loop body is the same for every sub-block.  The
+// sub-block's L columns are gathered into x[0..L-1] of the row's lanes by
+// shuffles and quantized there (every lane of the row runs the same column
+// chain); then each lane applies the L errors to its later columns (a rank-L
+// update with packed fp32x2 FMAs, in column order).  The block runs in four
+// phases whose register windows (S, 3S/4, S/2, S/4 slots) cover the columns
+// still ahead, so little update work is spent on dead slots.
+//
+// The quantization decision takes rint(w * (1/scale)).  Where that product
+// lies within 1e-6 (relative) of a half-integer -- the only place where it
+// can round differently from the correctly rounded quotient -- the warp redoes
+// the sub-block with rint(w / scale) throughout, so every code equals
+// clamp(rint(w / scale) + zero, 0, maxq) with the IEEE quotient.
+//
+// Per lazy block, a record built once per layer from U and perm holds, in
+// the order the kernel reads them:
+//   Uq[i][l][j] = U[s+i][s + l + L (i/L + j)]  (j = 1..S-1; 0 for j = 0, past
+//                  the block, and in the pad)
+//   Ud[m][o][o2] = U[s+Lm+o][s+Lm+o2]           (o2 > o; the L x L diagonal tiles)
+//   rdg[i] = 1 / U[s+i][s+i],  pcol[i] = perm[s+i]
+// and one bulk copy brings it into shared memory.
+template <int L>
+__global__ void sweep_records_kernel(const float* __restrict__ U, const int32_t* __restrict__ perm,
+                                     int k, int B, uint8_t* __restrict__ rec_all) {
+  using Ly = SqLayout<L>;
+  const int b = blockIdx.x;
+  const int s = b * B, bw = min(B, k - s);
+  float* Uq = (float*)(rec_all + (size_t)b * SQ_REC_MAX);
+  float* Ud = Uq + Ly::UQ;
+  float* rdg = Ud + Ly::UD;
+  int32_t* pcol = (int32_t*)(rdg + SW_MAX_B);
+  for (int e = threadIdx.x; e < Ly::UQ; e += blockDim.x) {
+    const int i = e / Ly::LDI, rem = e % Ly::LDI, l = rem / Ly::SEG, j = rem % Ly::SEG;
+    const int col = l + L * (i / L + j);
+    Uq[e] = (j >= 1 && j < Ly::S && i < bw && col < bw) ? U[(int64_t)(s + i) * k + s + col] : 0.f;
+  }
+  for (int e = threadIdx.x; e < Ly::UD; e += blockDim.x) {
+    const int m = e / (L * L), o = (e / L) % L, o2 = e % L;
+    Ud[e] = (o2 > o && L * m + o2 < bw) ? U[(int64_t)(s + L * m + o) * k + s + L * m + o2] : 0.f;
+  }
+  for (int i = threadIdx.x; i < SW_MAX_B; i += blockDim.x) {
+    rdg[i] = (i < bw) ? 1.0f / U[(int64_t)(s + i) * k + s + i] : 0.f;
+    pcol[i] = (i < bw) ? perm[s + i] : 0;
+  }
+}
+
+struct SqArgs {
+  const float* Wt;
+  float* Err;
+  float* Err_lo;
+  const uint8_t* rec;  // this block's record
+  int r, k, s, bw, B, G, ngroups;
+  float maxq;
+  float* scales;
+  int32_t* zeros;
+  uint8_t* codes;
+  double* loss;
+  int32_t* d_status;
+};
+
+template <int L>
+struct SqState {
+  float w[SqLayout<L>::S];
+  float scale, zero, inv_s, lo_d, hi_d;
+  double e2;
+  bool nonfinite;
+};
+
+// One sub-block (columns L m .. L m + L - 1) with a register window of W + 1 slots.
+template <int L, int W, int MODE>
+__device__ __forceinline__ void sq_sub_block(SqState<L>& st, int m, const SqArgs& a,
+                                             const float* Uq, const float* Ud, const float* rdg,
+                                             const int32_t* pcol, int l, int row, bool valid) {
+  using Ly = SqLayout<L>;
+  float x[L];
+#pragma unroll
+  for (int o = 0; o < L; ++o) x[o] = __shfl_sync(0xffffffffu, st.w[0], o, L);
+  if (MODE == 1 && (L * m) % a.G == 0) {
+    // a group starts here: its grid from the current weights of its columns
+    // [Lm, Lm + G) (slots past the block hold 0, which min(., 0) / max(., 0) absorb)
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int o = 1; o < L; ++o) mn = fminf(mn, x[o]), mx = fmaxf(mx, x[o]);
+    const int gq = a.G / L;
+    float pn = INFINITY, px = -INFINITY;
+#pragma unroll
+    for (int j = 1; j <= W; ++j)
+      if (j < gq) pn = fminf(pn, st.w[j]), px = fmaxf(px, st.w[j]);
+#pragma unroll
+    for (int o = 1; o < L; o <<= 1) {
+      pn = fminf(pn, __shfl_xor_sync(0xffffffffu, pn, o, L));
+      px = fmaxf(px, __shfl_xor_sync(0xffffffffu, px, o, L));
+    }
+    grid_from_range(fminf(mn, pn), fmaxf(mx, px), a.maxq, st.scale, st.zero);
+    st.inv_s = 1.0f / st.scale;
+    st.lo_d = -st.zero;
+    st.hi_d = a.maxq - st.zero;
+    if (valid && l == 0) {
+      const int g = (a.s + L * m) / a.G;
+      a.scales[(int64_t)row * a.ngroups + g] = st.scale;
+      a.zeros[(int64_t)row * a.ngroups + g] = (int32_t)st.zero;
+    }
+  }
+  float rd[L];
+#pragma unroll
+  for (int v = 0; v < L / 4; ++v) {
+    const float4 r4 = *(const float4*)(rdg + L * m + 4 * v);
+    rd[4 * v] = r4.x, rd[4 * v + 1] = r4.y, rd[4 * v + 2] = r4.z, rd[4 * v + 3] = r4.w;
+  }
+  float x0[L];
+#pragma unroll
+  for (int o = 0; o < L; ++o) x0[o] = x[o];
+  float err[L], dq[L];
+  bool tie = false;
+#pragma unroll
+  for (int o = 0; o < L; ++o) {
+    const float t = x[o] * st.inv_s;
+    const float rq = rintf(t);
+    tie |= fabsf(fabsf(t - rq) - 0.5f) <= 1e-6f * fabsf(t);
+    const float d = fminf(fmaxf(rq, st.lo_d), st.hi_d);  // code - zero
+    const float e = (x[o] - st.scale * d) * rd[o];
+    err[o] = e;
+    dq[o] = d;
+    if (o + 1 < L) {
+      const float* ur = Ud + (m * L + o) * L;
+#pragma unroll
+      for (int o2 = o + 1; o2 < L; ++o2) x[o2] = fmaf(-e, ur[o2], x[o2]);
+    }
+  }
+  if (__any_sync(0xffffffffu, tie)) {
+#pragma unroll
+    for (int o = 0; o < L; ++o) x[o] = x0[o];
+#pragma unroll
+    for (int o = 0; o < L; ++o) {
+      const float d = fminf(fmaxf(rint_exact_div(x[o], st.scale), st.lo_d), st.hi_d);
+      const float e = (x[o] - st.scale * d) * rd[o];
+      err[o] = e;
+      dq[o] = d;
+      if (o + 1 < L) {
+        const float* ur = Ud + (m * L + o) * L;
+#pragma unroll
+        for (int o2 = o + 1; o2 < L; ++o2) x[o2] = fmaf(-e, ur[o2], x[o2]);
+      }
+    }
+  }
+  // rank-L update of the later columns, one column's error at a time
+#pragma unroll
+  for (int o = 0; o < L; ++o) {
+    const float4* up = (const float4*)(Uq + (L * m + o) * Ly::LDI + l * Ly::SEG);
+    const float2 ne = make_float2(-err[o], -err[o]);
+#pragma unroll
+    for (int v = 0; v < (W + 1) / 4; ++v) {
+      const float4 u4 = up[v];
+      float2 p0 = make_float2(st.w[4 * v], st.w[4 * v + 1]);
+      float2 p1 = make_float2(st.w[4 * v + 2], st.w[4 * v + 3]);
+      p0 = __ffma2_rn(ne, make_float2(u4.x, u4.y), p0);
+      p1 = __ffma2_rn(ne, make_float2(u4.z, u4.w), p1);
+      st.w[4 * v] = p0.x, st.w[4 * v + 1] = p0.y;
+      st.w[4 * v + 2] = p1.x, st.w[4 * v + 3] = p1.y;
+    }
+  }
+  // this lane's column of the sub-block
+  float e_own = err[0], d_own = dq[0];
+#pragma unroll
+  for (int o = 1; o < L; ++o)
+    if (l == o) e_own = err[o], d_own = dq[o];
+  const int c = L * m + l;
+  if (valid && c < a.bw) {
+    a.codes[(int64_t)row * a.k + pcol[c]] = (uint8_t)(d_own + st.zero);
+    if (a.Err_lo != nullptr) {
+      float h, lo;
+      split_tf32(e_own, h, lo);
+      a.Err[(int64_t)row * a.B + c] = h;
+      a.Err_lo[(int64_t)row * a.B + c] = lo;
+    } else {
+      a.Err[(int64_t)row * a.B + c] = e_own;
+    }
+    st.nonfinite |= !isfinite(e_own);
+    st.e2 += (double)e_own * (double)e_own;
+  }
+#pragma unroll
+  for (int j = 0; j < W; ++j) st.w[j] = st.w[j + 1];
+  st.w[W] = 0.f;
+}
+
+// One lazy block [s, s + bw) for 32 / L rows per warp.  MODE 1: groups start
+// inside the block (G <= B, G % L == 0); MODE 0: the block lies inside one
+// group whose grid is already in scales / zeros.  Adds sum_i err_i^2 of the
+// block to loss[row] (the Optimal Brain Surgeon part of the layer loss).
+template <int L, int MODE>
+__global__ void __launch_bounds__(SQ_MAX_WARPS * 32, 1) sweep_block_lane_kernel(SqArgs a) {
+  using Ly = SqLayout<L>;
+  extern __shared__ __align__(128) uint8_t smq[];
+  float* Uq = (float*)smq;
+  float* Ud = Uq + Ly::UQ;
+  float* rdg = Ud + Ly::UD;
+  const int32_t* pcol = (const int32_t*)(rdg + SW_MAX_B);
+  uint64_t* bar = (uint64_t*)(smq + Ly::REC_BYTES);
+  volatile int* abort_flag = (volatile int*)(bar + 1);
+  const int tid = threadIdx.x, lane = tid & 31, l = lane % L;
+  const int row = (blockIdx.x * (blockDim.x / 32) + (tid >> 5)) * Ly::ROWS_PER_WARP + lane / L;
+  const bool valid = row < a.r;
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(bar, (uint32_t)Ly::REC_BYTES);
+    for (uint32_t off = 0; off < Ly::REC_BYTES; off += SQ_COPY_CHUNK) {
+      const uint32_t n = min(SQ_COPY_CHUNK, (uint32_t)Ly::REC_BYTES - off);
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              tc::smem_u32(smq + off)),
+          "l"(a.rec + off), "r"(n), "r"(tc::smem_u32(bar))
+          : "memory");
+    }
+  }
+  SqState<L> st;
+#pragma unroll
+  for (int j = 0; j < Ly::S; ++j) {
+    const int c = l + L * j;
+    st.w[j] = (valid && c < a.bw) ? a.Wt[(int64_t)row * a.k + a.s + c] : 0.f;
+  }
+  st.scale = 1.f, st.zero = 0.f;
+  if (MODE == 0 && valid) {
+    const int g = a.s / a.G;
+    st.scale = a.scales[(int64_t)row * a.ngroups + g];
+    st.zero = (float)a.zeros[(int64_t)row * a.ngroups + g];
+  }
+  st.inv_s = 1.0f / st.scale;
+  st.lo_d = -st.zero;
+  st.hi_d = a.maxq - st.zero;
+  st.e2 = 0.0;
+  st.nonfinite = false;
+  if (!tc::mbar_wait(bar, 0, abort_flag)) {
+    // the record never arrived: let the copy land (bounded) and report
+    for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
+      if (tc::mbar_try_wait(bar, 0)) break;
+    if (tid == 0 && a.d_status != nullptr) atomicCAS(a.d_status, 0, (int32_t)GPTQ_ERR_TIMEOUT);
+    return;
+  }
+  constexpr int S = Ly::S;
+  const int nsb = (a.bw + L - 1) / L;
+  int m = 0;
+  for (; m < min(nsb, S / 4); ++m)
+    sq_sub_block<L, S - 1, MODE>(st, m, a, Uq, Ud, rdg, pcol, l, row, valid);
+  for (; m < min(nsb, S / 2); ++m)
+    sq_sub_block<L, 3 * S / 4 - 1, MODE>(st, m, a, Uq, Ud, rdg, pcol, l, row, valid);
+  for (; m < min(nsb, 3 * S / 4); ++m)
+    sq_sub_block<L, S / 2 - 1, MODE>(st, m, a, Uq, Ud, rdg, pcol, l, row, valid);
+  for (; m < nsb; ++m)
+    sq_sub_block<L, S / 4 - 1, MODE>(st, m, a, Uq, Ud, rdg, pcol, l, row, valid);
+  double e2 = st.e2;
+#pragma unroll
+  for (int o = 1; o < L; o <<= 1) e2 += __shfl_xor_sync(0xffffffffu, e2, o, L);
+  if (a.loss != nullptr && valid && l == 0) a.loss[row] += e2;
+  if (st.nonfinite && a.d_status != nullptr) atomicCAS(a.d_status, 0, (int32_t)GPTQ_ERR_NONFINITE);
+}
+
+// Layer loss, second part: loss[row] -= lambda * sum_c (w0_c - q_c)^2 over the
+// original columns, q = scale * (code - zero) of the column's group (dead
+// columns count with w0 = 0).  One warp per row.
+template <typename T>
+__global__ void loss_finish_kernel(const T* __restrict__ W0, int64_t ldw, int r, int k,
+                                   const uint8_t* __restrict__ dead,
+                                   const uint8_t* __restrict__ codes,
+                                   const float* __restrict__ scales,
+                                   const int32_t* __restrict__ zeros,
+                                   const int32_t* __restrict__ g_idx, int ngroups,
+                                   const float* __restrict__ lambda, double* __restrict__ loss) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) / kWarp;
+  const int lane = threadIdx.x % kWarp;
+  if (row >= r) return;
+  double acc = 0.0;
+  for (int c = lane; c < k; c += kWarp) {
+    const int g = g_idx[c];
+    const float sc = scales[(int64_t)row * ngroups + g];
+    const float z = (float)zeros[(int64_t)row * ngroups + g];
+    const float q = sc * ((float)codes[(int64_t)row * k + c] - z);
+    const float w0 = dead[c] ? 0.f : to_f32(W0[(int64_t)row * ldw + c]);
+    const double dd = (double)w0 - (double)q;
+    acc += dd * dd;
+  }
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) loss[row] -= (double)(*lambda) * acc;
 }
 
 __global__ void loss_total_kernel(double* __restrict__ loss, int r) {
@@ -314,21 +619,31 @@ __global__ void loss_total_kernel(double* __restrict__ loss, int r) {
   }
 }
 
-template <int SB, typename T>
+template <int SB>
 static void launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* Err,
-                         float* Err_lo, const float* U, const int32_t* perm, const uint8_t* dead, const T* W0,
-                         int64_t ldw, int r, int k, int s0, int bw, int B, int G, int ngroups,
-                         float maxq, const float* lambda, float* scales, int32_t* zeros,
-                         uint8_t* codes, double* loss, int32_t* d_status) {
+                         float* Err_lo, const float* U, const int32_t* perm, int r, int k, int s0,
+                         int bw, int B, int G, int ngroups, float maxq, float* scales,
+                         int32_t* zeros, uint8_t* codes, double* loss, int32_t* d_status) {
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(sweep_block_kernel<SB, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(sweep_block_kernel<SB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)SW_SMEM);
     attr = true;
   }
-  sweep_block_kernel<SB, T><<<grid, SW_THREADS, SW_SMEM, s>>>(
-      Wt, Err, Err_lo, U, perm, dead, W0, ldw, r, k, s0, bw, B, G, ngroups, maxq, lambda, scales, zeros,
-      codes, loss, d_status);
+  sweep_block_kernel<SB><<<grid, SW_THREADS, SW_SMEM, s>>>(Wt, Err, Err_lo, U, perm, r, k, s0, bw,
+                                                           B, G, ngroups, maxq, scales, zeros,
+                                                           codes, loss, d_status);
+}
+
+template <int L, int MODE>
+static void launch_lane(unsigned grid, int threads, cudaStream_t s, const SqArgs& a) {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(sweep_block_lane_kernel<L, MODE>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SqLayout<L>::SMEM);
+    attr = true;
+  }
+  sweep_block_lane_kernel<L, MODE><<<grid, threads, SqLayout<L>::SMEM, s>>>(a);
 }
 
 template <typename T>
@@ -359,14 +674,36 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     gptq_status st = tc_split_transpose(U, k, k, k, sc.U_hi, sc.U_lo, k, s);
     if (st != GPTQ_OK) return st;
   }
-  // sub-block width: 16, or the largest power of two dividing a smaller group
+  // block kernel: the lane kernel when the groups inside a block have a
+  // multiple of 4 columns (or the block lies inside one group) -- 8 lanes per
+  // row unless the rows alone fill the SMs with 2 warps per scheduler, or the
+  // groups need 4 -- else the 4-threads-per-row kernel
+  int lane_mode = -1, lanes = 8;
+  if (G > B) lane_mode = 0;
+  else if (G % 4 == 0) lane_mode = 1;
+  const int nblocks = (int)cdiv(k, B);
+  int q_warps = 1;
+  unsigned q_grid = 0;
+  if (lane_mode >= 0) {
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if ((lane_mode == 1 && G % 8 != 0) || cdiv(r, 8) >= (int64_t)nsm * 8) lanes = 4;
+    const int64_t warps = cdiv(r, 32 / lanes);
+    q_warps = (int)std::min<int64_t>(SQ_MAX_WARPS, std::max<int64_t>(1, cdiv(warps, nsm)));
+    q_grid = (unsigned)cdiv(warps, q_warps);
+    if (lanes == 8) sweep_records_kernel<8><<<(unsigned)nblocks, 256, 0, s>>>(U, perm, k, B, sc.rec);
+    else sweep_records_kernel<4><<<(unsigned)nblocks, 256, 0, s>>>(U, perm, k, B, sc.rec);
+    GPTQ_CHECK_LAUNCH();
+  }
   int SB = 16;
   if (G < B) {
     SB = 1;
     while (SB < 16 && G % (SB * 2) == 0) SB *= 2;
   }
   const unsigned grid = (unsigned)cdiv(r, SW_ROWS);
-  for (int s0 = 0; s0 < k; s0 += B) {
+  float* err_lo = tc ? sc.Err_lo : nullptr;
+  for (int s0 = 0, b = 0; s0 < k; s0 += B, ++b) {
     int bw = min(B, k - s0);
     if (G > B && s0 % G == 0) {
       int gw = min(G, k - s0);
@@ -374,18 +711,39 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
           sc.Wt, r, k, s0, gw, s0 / G, ngroups, maxq, scales, zeros);
       GPTQ_CHECK_LAUNCH();
     }
-    const float* lam = want_loss ? sc.lambda : nullptr;
-#define GPTQ_SWEEP_BLOCK(SBV)                                                                     \
-  launch_block<SBV, T>(grid, s, sc.Wt, sc.Err, tc ? sc.Err_lo : nullptr, U, perm, dead, W, ldw, r, k, s0, bw, B, G, ngroups, \
-                       maxq, lam, scales, zeros, codes, lossp, d_status)
-    switch (SB) {
-      case 16: GPTQ_SWEEP_BLOCK(16); break;
-      case 8: GPTQ_SWEEP_BLOCK(8); break;
-      case 4: GPTQ_SWEEP_BLOCK(4); break;
-      case 2: GPTQ_SWEEP_BLOCK(2); break;
-      default: GPTQ_SWEEP_BLOCK(1); break;
-    }
+    if (lane_mode >= 0) {
+      SqArgs a;
+      a.Wt = sc.Wt;
+      a.Err = sc.Err;
+      a.Err_lo = err_lo;
+      a.rec = sc.rec + (size_t)b * SQ_REC_MAX;
+      a.r = r, a.k = k, a.s = s0, a.bw = bw, a.B = B, a.G = G, a.ngroups = ngroups;
+      a.maxq = maxq;
+      a.scales = scales;
+      a.zeros = zeros;
+      a.codes = codes;
+      a.loss = lossp;
+      a.d_status = d_status;
+      if (lanes == 8) {
+        if (lane_mode == 0) launch_lane<8, 0>(q_grid, 32 * q_warps, s, a);
+        else launch_lane<8, 1>(q_grid, 32 * q_warps, s, a);
+      } else {
+        if (lane_mode == 0) launch_lane<4, 0>(q_grid, 32 * q_warps, s, a);
+        else launch_lane<4, 1>(q_grid, 32 * q_warps, s, a);
+      }
+    } else {
+#define GPTQ_SWEEP_BLOCK(SBV)                                                                  \
+  launch_block<SBV>(grid, s, sc.Wt, sc.Err, err_lo, U, perm, r, k, s0, bw, B, G, ngroups, maxq, \
+                    scales, zeros, codes, lossp, d_status)
+      switch (SB) {
+        case 16: GPTQ_SWEEP_BLOCK(16); break;
+        case 8: GPTQ_SWEEP_BLOCK(8); break;
+        case 4: GPTQ_SWEEP_BLOCK(4); break;
+        case 2: GPTQ_SWEEP_BLOCK(2); break;
+        default: GPTQ_SWEEP_BLOCK(1); break;
+      }
 #undef GPTQ_SWEEP_BLOCK
+    }
     GPTQ_CHECK_LAUNCH();
     int e0 = s0 + bw;
     if (e0 < k) {
@@ -402,6 +760,9 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     }
   }
   if (want_loss) {
+    loss_finish_kernel<T><<<(unsigned)cdiv((int64_t)r * kWarp, 256), 256, 0, s>>>(
+        W, ldw, r, k, dead, codes, scales, zeros, g_idx, ngroups, sc.lambda, loss);
+    GPTQ_CHECK_LAUNCH();
     loss_total_kernel<<<1, 1024, 0, s>>>(loss, r);
     GPTQ_CHECK_LAUNCH();
   }

@@ -18,11 +18,16 @@
 //     R^T (k x 64); columns c < j0 are the Schur complement (sign -1, lower
 //     triangle only), columns c >= j0 the Y update (sign +1).
 //
-// Tiles of 128 x 256 (M x N) on a persistent grid; warp 0 issues TMA, warp 1
-// the MMAs (one thread), warps 2..5 read TMEM and update D in place.  TMEM
+// Tiles of 128 x 256 (M x N) on a persistent grid; warp 0 issues the operand
+// TMA loads, warp 1 the MMAs (one thread), warps 2..5 are the epilogue.  TMEM
 // holds two accumulators, so a tile's epilogue overlaps the next tile's
-// MMAs.  Every mbarrier wait is bounded; on a timeout the CTA drains its
-// own copies and MMAs, frees TMEM and raises *status.
+// MMAs.  The epilogue moves D through a two-slot shared-memory ring of
+// 128 x 32 chunks, by TMA in both directions: one epilogue thread loads
+// chunk g + 2 as soon as chunk g has been stored, the 128 threads add their
+// TMEM row to the chunk in place (128-byte swizzle, conflict-free), and the
+// chunk goes back with a TMA store that clips at the tensor's extent.  Every
+// mbarrier wait is bounded; on a timeout the CTA drains its own copies and
+// MMAs, frees TMEM and raises *status.
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -37,8 +42,11 @@ constexpr int TX_B_BYTES = TX_N * TX_KC * 4;         // 32 KB
 constexpr int TX_STAGE_BYTES = 2 * TX_A_BYTES + 2 * TX_B_BYTES;  // hi + lo of both: 96 KB
 constexpr int TX_THREADS = 192;                      // TMA, MMA, 4 epilogue warps
 constexpr int TX_TMEM_COLS = 512;
-constexpr int TX_EPI_BYTES = 4 * 32 * 33 * 4;             // per-warp 32 x 32 transpose tiles
-constexpr size_t TX_SMEM = (size_t)TX_STAGES * TX_STAGE_BYTES + TX_EPI_BYTES + 1024 + 256;
+constexpr int TX_DC = 32;                             // D chunk columns (one 128-byte row)
+constexpr int TX_D_BYTES = TX_M * TX_DC * 4;          // 16 KB per D chunk
+constexpr int TX_D_SLOTS = 2;
+constexpr size_t TX_SMEM =
+    (size_t)TX_STAGES * TX_STAGE_BYTES + (size_t)TX_D_SLOTS * TX_D_BYTES + 1024 + 256;
 
 struct TxArgs {
   float* D;
@@ -60,20 +68,31 @@ __device__ __forceinline__ bool tile_skipped(const TxArgs& a, int m0, int n0) {
   return a.mode == 1 && n0 + TX_N <= a.split && n0 >= m0 + TX_M;
 }
 
+// Next tile of this CTA after t (t = -1: the first) that has work, or ntiles.
+__device__ __forceinline__ int next_tile(const TxArgs& a, int t) {
+  for (t = (t < 0) ? (int)blockIdx.x : t + (int)gridDim.x; t < a.ntiles; t += gridDim.x) {
+    const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
+    if (!tile_skipped(a, m0, n0)) return t;
+  }
+  return a.ntiles;
+}
+
 __global__ void __launch_bounds__(TX_THREADS, 1)
 tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
                      const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
-                     TxArgs a) {
+                     const __grid_constant__ CUtensorMap d_map, TxArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  float* epi = (float*)(smem + TX_STAGES * TX_STAGE_BYTES);
-  uint64_t* bars = (uint64_t*)(smem + TX_STAGES * TX_STAGE_BYTES + TX_EPI_BYTES);
+  uint8_t* ring = smem + TX_STAGES * TX_STAGE_BYTES;  // D chunks, 1024-byte aligned
+  uint64_t* bars = (uint64_t*)(ring + TX_D_SLOTS * TX_D_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + TX_STAGES;
   uint64_t* tfull = bars + 2 * TX_STAGES;
   uint64_t* tempty = bars + 2 * TX_STAGES + 2;
   uint64_t* done = bars + 2 * TX_STAGES + 4;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * TX_STAGES + 5);
+  uint64_t* dfull = bars + 2 * TX_STAGES + 5;               // D chunk landed
+  uint64_t* dwritten = dfull + TX_D_SLOTS;                   // 128 threads updated it
+  uint32_t* tmem_slot = (uint32_t*)(dwritten + TX_D_SLOTS);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -87,12 +106,17 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
       tc::mbar_init(&tempty[b], 4);
     }
     tc::mbar_init(done, 1);
+    for (int d = 0; d < TX_D_SLOTS; ++d) {
+      tc::mbar_init(&dfull[d], 1);
+      tc::mbar_init(&dwritten[d], 128);
+    }
     *abort_flag = 0;
     tc::fence_barrier_init();
     tc::prefetch_tensormap(&a_hi);
     tc::prefetch_tensormap(&a_lo);
     tc::prefetch_tensormap(&b_hi);
     tc::prefetch_tensormap(&b_lo);
+    tc::prefetch_tensormap(&d_map);
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, TX_TMEM_COLS);
   tc::tc_fence_before();
@@ -178,56 +202,87 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
         if (tc::mbar_try_wait(done, 0)) break;
     }
   } else {
-    // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31 = tile rows; each
-    // 32 x 32 chunk goes through shared memory so that every update of D
-    // touches 32 consecutive columns of one row (one 128-byte line)
+    // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31, i.e. tile rows
     const int quarter = warp & 3;
-    float* tbuf = epi + (warp - 2) * 32 * 33;
+    const int trow = quarter * 32 + lane;
+    const bool dprod = (threadIdx.x == 64);  // issues the D chunk loads and stores
+    // D chunk producer: next chunk to load is (pt, pcc); gload chunks issued so far
+    int pt = next_tile(a, -1), pcc = 0, gload = 0, gproc = 0;
+    auto issue_next = [&]() {
+      if (pt >= a.ntiles) return;
+      const int slot = gload % TX_D_SLOTS;
+      const int m0 = (pt % a.ntm) * TX_M, n0 = (pt / a.ntm) * TX_N;
+      tc::mbar_arrive_expect_tx(&dfull[slot], TX_D_BYTES);
+      tc::tma_load_2d(ring + slot * TX_D_BYTES, &d_map, &dfull[slot], a.col0 + n0 + pcc * TX_DC,
+                      a.row0 + m0);
+      ++gload;
+      if (++pcc == TX_N / TX_DC) pcc = 0, pt = next_tile(a, pt);
+    };
+    if (dprod)
+      for (int d = 0; d < TX_D_SLOTS; ++d) issue_next();
     int tb = 0;
     uint32_t tphase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < a.ntiles && ok; t += gridDim.x) {
+    for (int t = next_tile(a, -1); t < a.ntiles && ok; t = next_tile(a, t)) {
       const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
-      if (tile_skipped(a, m0, n0)) continue;
       if (!tc::mbar_wait(&tfull[tb], tphase, abort_flag)) { ok = false; break; }
       tc::tc_fence_after();
-      for (int cc = 0; cc < TX_N / 32; ++cc) {
+      const int grow = a.row0 + m0 + trow;  // absolute row of this thread
+      for (int cc = 0; cc < TX_N / TX_DC; ++cc) {
         float v[32];
-        tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(tb * TX_N + cc * 32), v);
+        tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) +
+                                   (uint32_t)(tb * TX_N + cc * TX_DC),
+                               v);
         tc::tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) tbuf[lane * 33 + q] = v[q];
-        __syncwarp();
-        const int col = n0 + cc * 32 + lane;  // relative output column of this lane
-        const int c = a.col0 + col;           // absolute column
-        const int gm0 = m0 + quarter * 32;    // first relative row of this warp
-        // all 32 loads first (independent), then the updates and stores
-        float dv[32];
-#pragma unroll
-        for (int rr = 0; rr < 32; ++rr) {
-          const bool okr = (gm0 + rr < a.M) && (col < a.N);
-          dv[rr] = okr ? a.D[(int64_t)(a.row0 + gm0 + rr) * a.ldd + c] : 0.f;
+        if (cc == TX_N / TX_DC - 1) {  // accumulator fully read: hand it back to the MMA warp
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&tempty[tb]);
         }
+        const int slot = gproc % TX_D_SLOTS;
+        if (!tc::mbar_wait(&dfull[slot], (uint32_t)(gproc / TX_D_SLOTS) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* rowp = ring + slot * TX_D_BYTES + trow * 128;
+        const int cbase = a.col0 + n0 + cc * TX_DC;  // absolute column of v[0]
 #pragma unroll
-        for (int rr = 0; rr < 32; ++rr) {
-          const int gm = gm0 + rr;
-          if (gm < a.M && col < a.N) {
-            const float val = tbuf[rr * 33 + lane];
-            float out;
-            bool wr = true;
-            if (a.mode == 0) out = dv[rr] - val;
-            else if (c >= a.split) out = dv[rr] + val;
-            else if (c <= a.row0 + gm) out = dv[rr] - val;
-            else { out = dv[rr]; wr = false; }
-            if (wr) a.D[(int64_t)(a.row0 + gm) * a.ldd + c] = out;
+        for (int u = 0; u < 8; ++u) {
+          float4* p4 = (float4*)(rowp + ((u ^ (trow & 7)) << 4));
+          const float4 d4 = *p4;
+          float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float val = v[4 * u + j];
+            const int c = cbase + 4 * u + j;
+            if (a.mode == 0) dd[j] -= val;
+            else if (c >= a.split) dd[j] += val;
+            else if (c <= grow) dd[j] -= val;
           }
+          *p4 = make_float4(dd[0], dd[1], dd[2], dd[3]);
         }
-        __syncwarp();
+        tc::fence_proxy_async_smem();  // the TMA store reads what this thread wrote
+        tc::mbar_arrive(&dwritten[slot]);
+        if (dprod) {
+          if (!tc::mbar_wait(&dwritten[slot], (uint32_t)(gproc / TX_D_SLOTS) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::tma_store_2d(&d_map, ring + slot * TX_D_BYTES, cbase, a.row0 + m0);
+          tc::bulk_commit_group();
+          tc::bulk_wait_read_all();  // the slot may be refilled once the store has read it
+          issue_next();
+        }
+        ++gproc;
       }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&tempty[tb]);
       if (++tb == 2) tb = 0, tphase ^= 1u;
+    }
+    if (dprod) {
+      tc::bulk_wait_all();
+      // on an abort, let the loads still in flight land before the CTA exits
+      for (int g = gproc; g < gload; ++g)
+        for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
+          if (tc::mbar_try_wait(&dfull[g % TX_D_SLOTS], (uint32_t)(g / TX_D_SLOTS) & 1u)) break;
     }
   }
 
@@ -270,7 +325,7 @@ bool make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int
 }
 
 gptq_status launch(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMap& bh,
-                   const CUtensorMap& bl, TxArgs& a, cudaStream_t s) {
+                   const CUtensorMap& bl, const CUtensorMap& dm, TxArgs& a, cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(tf32x3_update_kernel,
@@ -283,7 +338,7 @@ gptq_status launch(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorM
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(a.ntiles, nsm);
   if (grid <= 0) return GPTQ_OK;
-  tf32x3_update_kernel<<<grid, TX_THREADS, TX_SMEM, s>>>(ah, al, bh, bl, a);
+  tf32x3_update_kernel<<<grid, TX_THREADS, TX_SMEM, s>>>(ah, al, bh, bl, dm, a);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
 }
@@ -371,9 +426,10 @@ gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols
 gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* ut_hi,
                               const float* ut_lo, float* Wt, int r, int k, int s0, int e,
                               int32_t* d_status, cudaStream_t s) {
-  CUtensorMap ah, al, bh, bl;
+  CUtensorMap ah, al, bh, bl, dm;
   if (!make_map(&ah, err_hi, B, r, B, TX_M) || !make_map(&al, err_lo, B, r, B, TX_M) ||
-      !make_map(&bh, ut_hi, k, k, k, TX_N) || !make_map(&bl, ut_lo, k, k, k, TX_N))
+      !make_map(&bh, ut_hi, k, k, k, TX_N) || !make_map(&bl, ut_lo, k, k, k, TX_N) ||
+      !make_map(&dm, Wt, k, r, k, TX_M))
     return GPTQ_ERR_INVALID_ARG;
   TxArgs a;
   a.D = Wt;
@@ -393,7 +449,7 @@ gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, c
   a.split = 0;
   a.status = d_status;
   a.status_code = GPTQ_ERR_TIMEOUT;
-  return launch(ah, al, bh, bl, a, s);
+  return launch(ah, al, bh, bl, dm, a, s);
 }
 
 // Rows [0, j0) of the k x k work matrix A += sign * R^T R (see the file
@@ -401,12 +457,15 @@ gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, c
 // scratch).  A timeout sets *d_info = k + 1.
 gptq_status tc_rank_update(float* A, int k, int j0, int b, float* rt_hi, float* rt_lo,
                            int32_t* d_info, cudaStream_t s) {
+  if (j0 <= 0) return GPTQ_OK;
   split_rowblock_t_kernel<<<(unsigned)cdiv(k, 32), dim3(32, 8), 0, s>>>(A, k, j0, b, rt_hi, rt_lo,
                                                                         d_info);
   GPTQ_CHECK_LAUNCH();
-  CUtensorMap ah, al, bh, bl;
+  CUtensorMap ah, al, bh, bl, dm;
+  // D's map ends at row j0: rows at and below the current row block are never touched
   if (!make_map(&ah, rt_hi, 64, k, 64, TX_M) || !make_map(&al, rt_lo, 64, k, 64, TX_M) ||
-      !make_map(&bh, rt_hi, 64, k, 64, TX_N) || !make_map(&bl, rt_lo, 64, k, 64, TX_N))
+      !make_map(&bh, rt_hi, 64, k, 64, TX_N) || !make_map(&bl, rt_lo, 64, k, 64, TX_N) ||
+      !make_map(&dm, A, k, j0, k, TX_M))
     return GPTQ_ERR_INVALID_ARG;
   TxArgs a;
   a.D = A;
@@ -426,7 +485,7 @@ gptq_status tc_rank_update(float* A, int k, int j0, int b, float* rt_hi, float* 
   a.split = j0;
   a.status = d_info;
   a.status_code = k + 1;
-  return launch(ah, al, bh, bl, a, s);
+  return launch(ah, al, bh, bl, dm, a, s);
 }
 
 }  // namespace gptq

@@ -43,6 +43,17 @@ CASES = {
                                                block_size=64, bits=2),
     "int8_g64": synth.CONFIGS["q_proj"].scaled(r=128, k=512, n=8192, group_size=64,
                                                block_size=64, bits=8),
+    # group sizes the lane kernel does not take (4-threads-per-row kernel)
+    "g48_b96": synth.CONFIGS["q_proj"].scaled(r=96, k=480, n=4096, group_size=48,
+                                              block_size=96),
+    # groups of 16 with act-order and a ragged last block of 16 columns
+    "g16_act_ragged": synth.CONFIGS["down_proj"].scaled(r=64, k=400, n=4096, group_size=16),
+    # group = block = 48, rows not a multiple of 4, last block 8 columns wide
+    "gB48_ragged": synth.CONFIGS["tiny"].scaled(r=70, k=200, n=3000, group_size=48,
+                                                block_size=48),
+    # k not a multiple of 4: CUDA-core trailing and rank updates
+    "k150_cuda_core": synth.CONFIGS["tiny"].scaled(r=40, k=150, n=2000, group_size=-1,
+                                                   block_size=32),
 }
 
 
