@@ -18,11 +18,16 @@
 //   K2 panel   P = L[J, 0:j0] = U_JJ * Hp[J, 0:j0]   (in place, lower part),
 //      and     U[J, e:] = -U_JJ * Y[J, e:]          (in place, upper part):
 //              V = [[V_JJ, V_J*], [0, V_**]] gives U_J* = -V_JJ^-1 V_J* U_**.
+//              K1 and K2 also write row block J transposed and split into
+//              tf32 hi / lo, the operand of the tensor-core update.
 //   K3 one rank-64 update of rows [0, j0) (K = the 64 rows of block J), on
 //      the tensor cores in fp32-accurate 3xTF32 when the workspace holds the
 //      operand splits (tf32x3.cu), else on the CUDA cores:
 //              A[0:j0, 0:j0] (lower) -= P^T P        (Schur complement)
 //              Y[0:j0, j0:]          += P^T U[J, j0:] (V[0:j0, J] = P^T)
+//      The tensor-core form updates the whole square [0, j0)^2 (tiles that
+//      lie entirely above its diagonal excepted), so the strip
+//      A[0:j0, j0:j1] is cleared by K2 before Y's block-J columns start.
 // so every step's large work is a short-K product with a big output.
 // A final pass zeroes the strict lower triangle.
 #include "common.cuh"
@@ -32,16 +37,18 @@ namespace gptq {
 constexpr int HV_B = 64;  // block width
 
 bool tc_update_supported(int64_t k);
-gptq_status tc_rank_update(float* A, int k, int j0, int b, float* r_hi, float* r_lo,
-                           int32_t* d_info, cudaStream_t s);
+gptq_status tc_rank_update(float* A, int k, int j0, int b, const float* s_hi, const float* s_lo,
+                           const float* r_hi, const float* r_lo, int32_t* d_info, cudaStream_t s);
 
 struct HinvScratch {
   double* sum_diag;  // [1]
   float* lambda;     // [1]
   float* diag;       // [k] diag(H) after the dead-column fix
   float* ujj;        // [HV_B * HV_B] U_JJ of the current step
-  float* r_hi;       // [HV_B * k] tf32 split of the current row block (tensor-core path)
-  float* r_lo;       // [HV_B * k]
+  float* s_hi;       // [k * HV_B] signed split of the current row block, transposed (tensor-core path)
+  float* s_lo;
+  float* r_hi;       // [k * HV_B] unsigned split (columns < j0 only)
+  float* r_lo;
 };
 
 // Scratch of the CUDA-core path.
@@ -57,7 +64,7 @@ size_t hinv_workspace_min_bytes(int64_t k) {
 // Scratch of the tensor-core path (the size gptq_workspace_size reports).
 size_t hinv_workspace_bytes(int64_t k) {
   size_t b = hinv_workspace_min_bytes(k);
-  if (tc_update_supported(k)) b += 2 * align256(sizeof(float) * HV_B * (size_t)k);
+  if (tc_update_supported(k)) b += 4 * align256(sizeof(float) * HV_B * (size_t)k);
   return b;
 }
 
@@ -68,9 +75,12 @@ static HinvScratch carve(void* ws, int64_t k, bool tc) {
   s.lambda = (float*)p; p += align256(sizeof(float));
   s.diag = (float*)p; p += align256(sizeof(float) * (size_t)k);
   s.ujj = (float*)p; p += align256(sizeof(float) * HV_B * HV_B);
-  s.r_hi = tc ? (float*)p : nullptr;
-  if (tc) p += align256(sizeof(float) * HV_B * (size_t)k);
-  s.r_lo = tc ? (float*)p : nullptr;
+  float* t[4] = {nullptr, nullptr, nullptr, nullptr};
+  for (int i = 0; i < 4 && tc; ++i) {
+    t[i] = (float*)p;
+    p += align256(sizeof(float) * HV_B * (size_t)k);
+  }
+  s.s_hi = t[0], s.s_lo = t[1], s.r_hi = t[2], s.r_lo = t[3];
   return s;
 }
 
@@ -148,6 +158,14 @@ __global__ void hinv_gather_lower_kernel(const float* __restrict__ H, int k,
   }
 }
 
+// hi = x rounded to tf32 (nearest, ties away), lo = x - hi
+__device__ __forceinline__ void hv_split_tf32(float x, float& hi, float& lo) {
+  uint32_t h;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+  hi = __uint_as_float(h);
+  lo = x - hi;
+}
+
 __device__ __forceinline__ void set_info(int32_t* d_info, int idx) { atomicCAS(d_info, 0, idx + 1); }
 
 // K1: factor the diagonal block (lower storage, A_JJ = L^T L with L lower)
@@ -163,7 +181,8 @@ __device__ __forceinline__ void set_info(int32_t* d_info, int idx) { atomicCAS(d
 // combine their partial sums with shuffles, so the inverse needs no barrier.
 __global__ void __launch_bounds__(256)
 chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
-                     float* __restrict__ ujj, int32_t* __restrict__ d_info) {
+                     float* __restrict__ ujj, float* __restrict__ st_hi,
+                     float* __restrict__ st_lo, int32_t* __restrict__ d_info) {
   if (*d_info != 0) return;
   __shared__ float S[HV_B][HV_B + 1];
   __shared__ float rdg[HV_B];
@@ -251,6 +270,13 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
     const int i = part + 4 * u;
     ujj[i * HV_B + c] = y[u];
     if (i < b && c < b && c >= i) A[(int64_t)(j0 + i) * k + j0 + c] = y[u];
+    if (st_hi != nullptr && c < b) {
+      // rank-update operand s[j0 + c][i] = U_JJ[i][c] (upper triangle, 0 below it)
+      float h, l;
+      hv_split_tf32((i < b && c >= i) ? y[u] : 0.f, h, l);
+      st_hi[(int64_t)(j0 + c) * HV_B + i] = h;
+      st_lo[(int64_t)(j0 + c) * HV_B + i] = l;
+    }
   }
 }
 
@@ -259,39 +285,106 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
 //     (lower part of row block J, in place).
 //   CTAs [n_pan, ...): 64-column tiles c0 of [e, k): U[J, c] = -U_JJ * Y[J, c]
 //     (upper part of row block J, in place).
+//   CTAs [n_pan + n_row, ...): zero 64-row pieces of the strip
+//     A[0:j0, j0:j1], where Y's columns of block J start accumulating in this
+//     step's update (the tensor-core Schur update writes the whole square
+//     [0, j0)^2 and leaves values above its diagonal).
 // Each CTA reads its whole 64 x 64 tile before writing it.  Thread
-// (r = t / 4, cq = t % 4) computes row r, columns cq + 4q.
+// (r = t / 4, cq = t % 4) computes row r, columns cq + 4q.  When st_hi is
+// given, the new row-block tile also goes out transposed and split into tf32
+// hi / lo in the rank update's operand layout: st[c][m] = -R[m][c] for c < j0
+// and +R[m][c] above, rt[c][m] = R[m][c] for c < j0.
 __global__ void __launch_bounds__(256)
 panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* __restrict__ ujj,
-                      int n_pan, const int32_t* __restrict__ d_info) {
+                      int n_pan, int n_row, float* __restrict__ st_hi, float* __restrict__ st_lo,
+                      float* __restrict__ rt_hi, float* __restrict__ rt_lo,
+                      const int32_t* __restrict__ d_info) {
   if (*d_info != 0) return;
-  __shared__ float Us[HV_B][HV_B + 1];
-  __shared__ float Hs[HV_B][HV_B + 1];
+  if ((int)blockIdx.x >= n_pan + n_row) {
+    const int z0 = ((int)blockIdx.x - n_pan - n_row) * HV_B;
+    for (int e = threadIdx.x; e < HV_B * HV_B; e += 256) {
+      const int i = z0 + e / HV_B, c = j0 + e % HV_B;
+      if (i < j0 && c < j0 + b) A[(int64_t)i * k + c] = 0.f;
+    }
+    return;
+  }
+  __shared__ __align__(16) float Us[HV_B][HV_B + 4];  // row stride 68: conflict-free row reads
+  __shared__ float Hs[HV_B][HV_B + 1];                // row stride 65: conflict-free columns
   const int t = threadIdx.x;
   const bool pan = (int)blockIdx.x < n_pan;
   const int c0 = pan ? blockIdx.x * HV_B : j0 + b + (blockIdx.x - n_pan) * HV_B;
   const int cend = pan ? j0 : k;
   const float sign = pan ? 1.0f : -1.0f;
-  for (int e = t; e < HV_B * HV_B; e += 256) {
-    int i = e / HV_B, j = e % HV_B;
-    Us[i][j] = ujj[e];
-    Hs[i][j] = (i < b && c0 + j < cend) ? A[(int64_t)(j0 + i) * k + c0 + j] : 0.f;
+  const bool vec = (k % 4 == 0);
+  {
+    float4 uv[4], hv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e4 = t + 256 * q, i = e4 >> 4, j = (e4 & 15) * 4;
+      uv[q] = reinterpret_cast<const float4*>(ujj)[e4];
+      const float* src = A + (int64_t)(j0 + i) * k + c0 + j;
+      if (i < b && vec && c0 + j + 3 < cend) {
+        hv[q] = *reinterpret_cast<const float4*>(src);
+      } else {
+        hv[q].x = (i < b && c0 + j < cend) ? src[0] : 0.f;
+        hv[q].y = (i < b && c0 + j + 1 < cend) ? src[1] : 0.f;
+        hv[q].z = (i < b && c0 + j + 2 < cend) ? src[2] : 0.f;
+        hv[q].w = (i < b && c0 + j + 3 < cend) ? src[3] : 0.f;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e4 = t + 256 * q, i = e4 >> 4, j = (e4 & 15) * 4;
+      *reinterpret_cast<float4*>(&Us[i][j]) = uv[q];
+      Hs[i][j] = hv[q].x, Hs[i][j + 1] = hv[q].y, Hs[i][j + 2] = hv[q].z, Hs[i][j + 3] = hv[q].w;
+    }
   }
   __syncthreads();
   const int r = t >> 2, cq = t & 3;
-  if (r >= b) return;
   float acc[HV_B / 4];
 #pragma unroll
   for (int q = 0; q < HV_B / 4; ++q) acc[q] = 0.f;
-  for (int m = r; m < b; ++m) {
-    const float u = Us[r][m];
+  if (r < b) {
+    for (int m = r; m < b; ++m) {
+      const float u = Us[r][m];
 #pragma unroll
-    for (int q = 0; q < HV_B / 4; ++q) acc[q] = fmaf(u, Hs[m][cq + 4 * q], acc[q]);
+      for (int q = 0; q < HV_B / 4; ++q) acc[q] = fmaf(u, Hs[m][cq + 4 * q], acc[q]);
+    }
   }
+  __syncthreads();
 #pragma unroll
-  for (int q = 0; q < HV_B / 4; ++q) {
-    const int cc = c0 + cq + 4 * q;
-    if (cc < cend) A[(int64_t)(j0 + r) * k + cc] = sign * acc[q];
+  for (int q = 0; q < HV_B / 4; ++q) Hs[r][cq + 4 * q] = sign * acc[q];
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e4 = t + 256 * q, i = e4 >> 4, j = (e4 & 15) * 4;
+    if (i >= b) continue;
+    float* dst = A + (int64_t)(j0 + i) * k + c0 + j;
+    if (vec && c0 + j + 3 < cend) {
+      *reinterpret_cast<float4*>(dst) = make_float4(Hs[i][j], Hs[i][j + 1], Hs[i][j + 2], Hs[i][j + 3]);
+    } else {
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        if (c0 + j + jj < cend) dst[jj] = Hs[i][j + jj];
+    }
+  }
+  if (st_hi != nullptr) {
+#pragma unroll 4
+    for (int e = t; e < HV_B * HV_B; e += 256) {
+      const int cc = e >> 6, m = e & 63;
+      if (c0 + cc < cend) {
+        // Hs holds the new row block R (what went to A)
+        const float x = m < b ? Hs[m][cc] : 0.f;
+        float h, l;
+        hv_split_tf32(pan ? -x : x, h, l);  // st = -R for c < j0, +R for c >= j1
+        st_hi[(int64_t)(c0 + cc) * HV_B + m] = h;
+        st_lo[(int64_t)(c0 + cc) * HV_B + m] = l;
+        if (pan) {
+          rt_hi[(int64_t)(c0 + cc) * HV_B + m] = -h;
+          rt_lo[(int64_t)(c0 + cc) * HV_B + m] = -l;
+        }
+      }
+    }
   }
 }
 
@@ -440,18 +533,26 @@ gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cf
   for (int j1 = k; j1 > 0; j1 -= HV_B) {
     const int j0 = j1 > HV_B ? j1 - HV_B : 0;
     const int b = j1 - j0;
-    chol_inv_diag_kernel<<<1, 256, 0, s>>>(U, k, j0, b, sc.ujj, d_info);
+    // the tensor-core update takes row block J transposed and split into
+    // tf32 hi / lo, written by K1 (diagonal columns) and K2 (the rest); its
+    // Schur part leaves values above the diagonal of [0, j0)^2, so K2 also
+    // clears the strip where block J's Y columns start accumulating
+    const bool tcs = tc && j0 > 0;
+    chol_inv_diag_kernel<<<1, 256, 0, s>>>(U, k, j0, b, sc.ujj, tcs ? sc.s_hi : nullptr,
+                                           tcs ? sc.s_lo : nullptr, d_info);
     GPTQ_CHECK_LAUNCH();
     const int n_pan = (int)cdiv(j0, HV_B);
     const int n_row = (int)cdiv(k - j1, HV_B);
-    if (n_pan + n_row > 0) {
-      panel_rowblock_kernel<<<(unsigned)(n_pan + n_row), 256, 0, s>>>(U, k, j0, b, sc.ujj, n_pan,
-                                                                       d_info);
+    const int n_zero = tcs ? n_pan : 0;
+    if (n_pan + n_row + n_zero > 0) {
+      panel_rowblock_kernel<<<(unsigned)(n_pan + n_row + n_zero), 256, 0, s>>>(
+          U, k, j0, b, sc.ujj, n_pan, n_row, tcs ? sc.s_hi : nullptr, tcs ? sc.s_lo : nullptr,
+          tcs ? sc.r_hi : nullptr, tcs ? sc.r_lo : nullptr, d_info);
       GPTQ_CHECK_LAUNCH();
     }
     if (j0 > 0) {
       if (tc) {
-        gptq_status st = tc_rank_update(U, k, j0, b, sc.r_hi, sc.r_lo, d_info, s);
+        gptq_status st = tc_rank_update(U, k, j0, b, sc.s_hi, sc.s_lo, sc.r_hi, sc.r_lo, d_info, s);
         if (st != GPTQ_OK) return st;
       } else {
         const int nt = (int)cdiv(j0, 128);

@@ -61,17 +61,17 @@ constexpr size_t SQ_REC_MAX = SqLayout<8>::REC_BYTES > SqLayout<4>::REC_BYTES
 static size_t sweep_records_bytes(int64_t k, int B) { return (size_t)cdiv(k, B) * SQ_REC_MAX; }
 
 bool tc_update_supported(int64_t k);
-gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float* hi,
-                               float* lo, int64_t ldo, cudaStream_t s);
-gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* u_hi,
-                              const float* u_lo, float* Wt, int r, int k, int s0, int e,
+gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float sign,
+                               float* hi, float* lo, int64_t ldo, cudaStream_t s);
+gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* nut_hi,
+                              const float* nut_lo, float* Wt, int r, int k, int s0, int e,
                               int32_t* d_status, cudaStream_t s);
 
 struct SweepScratch {
   float* Wt;      // [r * k] working weights, processing order
   float* Err;     // [r * B] errors of the current block (tf32 high part on the tensor-core path)
   float* Err_lo;  // [r * B] tf32 low part (tensor-core path)
-  float* U_hi;    // [k * k] tf32 split of U^T (tensor-core path)
+  float* U_hi;    // [k * k] tf32 split of -U^T (tensor-core path)
   float* U_lo;    // [k * k]
   float* lambda;  // [1] damping added to the Hessian diagonal (for the loss)
   uint8_t* rec;   // per-block records of the 4-lanes-per-row kernel
@@ -671,7 +671,7 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     GPTQ_CHECK_LAUNCH();
   }
   if (tc) {
-    gptq_status st = tc_split_transpose(U, k, k, k, sc.U_hi, sc.U_lo, k, s);
+    gptq_status st = tc_split_transpose(U, k, k, k, -1.0f, sc.U_hi, sc.U_lo, k, s);
     if (st != GPTQ_OK) return st;
   }
   // block kernel: the lane kernel when the groups inside a block have a

@@ -1,31 +1,34 @@
 // fp32-accurate short-K updates on the 5th-generation tensor cores:
-//   D[m][n] += sign(n) * sum_k A[m][k] B[k][n]        (K <= 128)
+//   D[row][c] += sum_k R[row][k] C[c][k]                          (K <= 128)
 // with every fp32 operand split as x = hi + lo, hi = x rounded to tf32 and
 // lo = x - hi (exact), and three kind::tf32 MMAs per K step,
 //   A B ~= A_hi B_hi + A_hi B_lo + A_lo B_hi,
 // which keeps fp32-level accuracy (the dropped A_lo B_lo term and the tf32
 // rounding of lo are ~2^-21 relative).  The splits are written to global
-// memory, K-major (K contiguous) for both operands -- a transposing split
+// memory K-major (K contiguous) for both operands -- a transposing split
 // where the source is stored the other way -- so TMA brings hi and lo boxes
-// straight into shared memory in the 128-byte-swizzled K-major layout.
+// straight into shared memory in the 128-byte-swizzled K-major layout.  Any
+// sign of the update is folded into the C operand by whoever writes it, so
+// the whole tile is a plain D += R C^T.
 //
 // Two uses:
 //   mode 0, lazy-batch trailing update of the GPTQ sweep ([GPTQ-tool]
-//     "GPTQ" How it works Step 7): W[:, e:] -= Err * U[s:s+B, e:], with Err
-//     (rows x B) and U^T (the transposed split of the k x k factor).
+//     "GPTQ" How it works Step 7): W[:, e:] -= Err * U[s:s+B, e:], with
+//     R = Err (rows x B) and C = -U^T (the negated transposed split).
 //   mode 1, rank-b update of the inverse factor: rows [0, j0) of the work
-//     matrix += sign * R^T R', with R = A[j0:j0+b, :] split transposed into
-//     R^T (k x 64); columns c < j0 are the Schur complement (sign -1, lower
-//     triangle only), columns c >= j0 the Y update (sign +1).
+//     matrix += R^T S, R = A[j0:j0+b, 0:j0] and S = the row block with its
+//     columns c < j0 negated (Schur complement) and c >= j0 kept (Y update);
+//     tiles that lie entirely right of the diagonal inside [0, j0)^2 are
+//     skipped, the others are updated whole.
 //
-// Tiles of 128 x 256 (M x N) on a persistent grid; warp 0 issues the operand
-// TMA loads, warp 1 the MMAs (one thread), warps 2..5 are the epilogue.  TMEM
-// holds two accumulators, so a tile's epilogue overlaps the next tile's
-// MMAs.  The epilogue moves D through a two-slot shared-memory ring of
-// 128 x 32 chunks, by TMA in both directions: one epilogue thread loads
-// chunk g + 2 as soon as chunk g has been stored, the 128 threads add their
-// TMEM row to the chunk in place (128-byte swizzle, conflict-free), and the
-// chunk goes back with a TMA store that clips at the tensor's extent.  Every
+// Tiles of 128 x 256 (rows x columns) on a persistent grid; warp 0 issues the
+// operand TMA loads, warp 1 the MMAs (one thread), warps 2..5 are the
+// epilogue.  TMEM holds two accumulators, so a tile's epilogue overlaps the
+// next tile's MMAs.  D is never read by the kernel: the epilogue writes the
+// accumulator of a 128 x 32 chunk into a two-slot shared-memory ring
+// (128-byte swizzle, conflict-free) and one thread sends it to D with a TMA
+// tensor reduce-add, which L2 applies as D = fl(D + v) and which clips at the
+// tensor's extent.  A slot is rewritten once its reduce has read it.  Every
 // mbarrier wait is bounded; on a timeout the CTA drains its own copies and
 // MMAs, frees TMEM and raises *status.
 #include "common.cuh"
@@ -63,8 +66,8 @@ struct TxArgs {
 };
 
 __device__ __forceinline__ bool tile_skipped(const TxArgs& a, int m0, int n0) {
-  // mode 1: a tile whose columns all lie in [0, split) and strictly above the
-  // diagonal of its rows has nothing to update
+  // mode 1: a tile whose columns all lie in [0, split) and strictly right of
+  // the diagonal of its rows has nothing the factorisation reads
   return a.mode == 1 && n0 + TX_N <= a.split && n0 >= m0 + TX_M;
 }
 
@@ -90,8 +93,8 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
   uint64_t* tfull = bars + 2 * TX_STAGES;
   uint64_t* tempty = bars + 2 * TX_STAGES + 2;
   uint64_t* done = bars + 2 * TX_STAGES + 4;
-  uint64_t* dfull = bars + 2 * TX_STAGES + 5;               // D chunk landed
-  uint64_t* dwritten = dfull + TX_D_SLOTS;                   // 128 threads updated it
+  uint64_t* dfree = bars + 2 * TX_STAGES + 5;     // slot read by its reduce
+  uint64_t* dwritten = dfree + TX_D_SLOTS;        // the 4 epilogue warps wrote it
   uint32_t* tmem_slot = (uint32_t*)(dwritten + TX_D_SLOTS);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -107,8 +110,8 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
     }
     tc::mbar_init(done, 1);
     for (int d = 0; d < TX_D_SLOTS; ++d) {
-      tc::mbar_init(&dfull[d], 1);
-      tc::mbar_init(&dwritten[d], 128);
+      tc::mbar_init(&dfree[d], 1);
+      tc::mbar_init(&dwritten[d], 4);  // one arrival per epilogue warp
     }
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -205,85 +208,58 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
     // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. +31, i.e. tile rows
     const int quarter = warp & 3;
     const int trow = quarter * 32 + lane;
-    const bool dprod = (threadIdx.x == 64);  // issues the D chunk loads and stores
-    // D chunk producer: next chunk to load is (pt, pcc); gload chunks issued so far
-    int pt = next_tile(a, -1), pcc = 0, gload = 0, gproc = 0;
-    auto issue_next = [&]() {
-      if (pt >= a.ntiles) return;
-      const int slot = gload % TX_D_SLOTS;
-      const int m0 = (pt % a.ntm) * TX_M, n0 = (pt / a.ntm) * TX_N;
-      tc::mbar_arrive_expect_tx(&dfull[slot], TX_D_BYTES);
-      tc::tma_load_2d(ring + slot * TX_D_BYTES, &d_map, &dfull[slot], a.col0 + n0 + pcc * TX_DC,
-                      a.row0 + m0);
-      ++gload;
-      if (++pcc == TX_N / TX_DC) pcc = 0, pt = next_tile(a, pt);
-    };
-    if (dprod)
-      for (int d = 0; d < TX_D_SLOTS; ++d) issue_next();
-    int tb = 0;
+    const bool dprod = (threadIdx.x == 64);  // issues the reduce-adds
+    int tb = 0, g = 0;
     uint32_t tphase = 0;
     bool ok = true;
     for (int t = next_tile(a, -1); t < a.ntiles && ok; t = next_tile(a, t)) {
       const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
       if (!tc::mbar_wait(&tfull[tb], tphase, abort_flag)) { ok = false; break; }
       tc::tc_fence_after();
-      const int grow = a.row0 + m0 + trow;  // absolute row of this thread
-      for (int cc = 0; cc < TX_N / TX_DC; ++cc) {
-        float v[32];
-        tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) +
-                                   (uint32_t)(tb * TX_N + cc * TX_DC),
-                               v);
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(tb * TX_N);
+      float v[32];
+      tc::tmem_ld_32x32b_x32(tbase, v);
+      for (int cc = 0; cc < TX_N / TX_DC; ++cc, ++g) {
         tc::tmem_ld_wait();
-        if (cc == TX_N / TX_DC - 1) {  // accumulator fully read: hand it back to the MMA warp
+        const int slot = g % TX_D_SLOTS;
+        if (g >= TX_D_SLOTS) {
+          // the slot's previous reduce must have read it
+          if (!tc::mbar_wait(&dfree[slot], (uint32_t)((g / TX_D_SLOTS) - 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+        }
+        uint8_t* rowp = ring + slot * TX_D_BYTES + trow * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *(float4*)(rowp + ((u ^ (trow & 7)) << 4)) =
+              make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        if (cc + 1 < TX_N / TX_DC) {
+          tc::tmem_ld_32x32b_x32(tbase + (uint32_t)((cc + 1) * TX_DC), v);
+        } else {  // accumulator fully read: hand it back to the MMA warp
           tc::tc_fence_before();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&tempty[tb]);
         }
-        const int slot = gproc % TX_D_SLOTS;
-        if (!tc::mbar_wait(&dfull[slot], (uint32_t)(gproc / TX_D_SLOTS) & 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        uint8_t* rowp = ring + slot * TX_D_BYTES + trow * 128;
-        const int cbase = a.col0 + n0 + cc * TX_DC;  // absolute column of v[0]
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          float4* p4 = (float4*)(rowp + ((u ^ (trow & 7)) << 4));
-          const float4 d4 = *p4;
-          float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float val = v[4 * u + j];
-            const int c = cbase + 4 * u + j;
-            if (a.mode == 0) dd[j] -= val;
-            else if (c >= a.split) dd[j] += val;
-            else if (c <= grow) dd[j] -= val;
-          }
-          *p4 = make_float4(dd[0], dd[1], dd[2], dd[3]);
-        }
-        tc::fence_proxy_async_smem();  // the TMA store reads what this thread wrote
-        tc::mbar_arrive(&dwritten[slot]);
+        tc::fence_proxy_async_smem();  // the reduce reads what this thread wrote
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&dwritten[slot]);
         if (dprod) {
-          if (!tc::mbar_wait(&dwritten[slot], (uint32_t)(gproc / TX_D_SLOTS) & 1u, abort_flag)) {
+          if (!tc::mbar_wait(&dwritten[slot], (uint32_t)(g / TX_D_SLOTS) & 1u, abort_flag)) {
             ok = false;
             break;
           }
-          tc::tma_store_2d(&d_map, ring + slot * TX_D_BYTES, cbase, a.row0 + m0);
+          tc::tma_reduce_add_2d(&d_map, ring + slot * TX_D_BYTES, a.col0 + n0 + cc * TX_DC,
+                                a.row0 + m0);
           tc::bulk_commit_group();
-          tc::bulk_wait_read_all();  // the slot may be refilled once the store has read it
-          issue_next();
+          // free the other slot for the chunk after next once its reduce has read it
+          tc::bulk_wait_read_1();
+          if (g >= 1) tc::mbar_arrive(&dfree[(g - 1) % TX_D_SLOTS]);
         }
-        ++gproc;
       }
       if (++tb == 2) tb = 0, tphase ^= 1u;
     }
-    if (dprod) {
-      tc::bulk_wait_all();
-      // on an abort, let the loads still in flight land before the CTA exits
-      for (int g = gproc; g < gload; ++g)
-        for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
-          if (tc::mbar_try_wait(&dfull[g % TX_D_SLOTS], (uint32_t)(g / TX_D_SLOTS) & 1u)) break;
-    }
+    if (dprod) tc::bulk_wait_all();
   }
 
   __syncthreads();
@@ -352,11 +328,11 @@ __device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
   lo = x - hi;
 }
 
-// dst[c][r] = split(src[r][c]) for r < rows, c < cols (32 x 32 tiles
+// dst[c][r] = split(sign * src[r][c]) for r < rows, c < cols (32 x 32 tiles
 // through shared memory, so both the reads and the writes are coalesced).
 __global__ void split_transpose_kernel(const float* __restrict__ src, int64_t lds, int rows,
-                                       int cols, float* __restrict__ hi, float* __restrict__ lo,
-                                       int64_t ldo) {
+                                       int cols, float sign, float* __restrict__ hi,
+                                       float* __restrict__ lo, int64_t ldo) {
   __shared__ float tile[32][33];
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
   const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
@@ -369,40 +345,9 @@ __global__ void split_transpose_kernel(const float* __restrict__ src, int64_t ld
     const int c = c0 + y, r = r0 + tx;
     if (c < cols && r < rows) {
       float h, l;
-      split_tf32(tile[tx][y], h, l);
+      split_tf32(sign * tile[tx][y], h, l);
       hi[(int64_t)c * ldo + r] = h;
       lo[(int64_t)c * ldo + r] = l;
-    }
-  }
-}
-
-// Rt[c][m] = split(R[m][c]), R = A[j0:j0+b, :] with the diagonal block read as
-// upper triangular (its lower part holds stale values); m in [b, 64) is 0.
-__global__ void split_rowblock_t_kernel(const float* __restrict__ A, int k, int j0, int b,
-                                        float* __restrict__ hi, float* __restrict__ lo,
-                                        const int32_t* __restrict__ d_info) {
-  if (*d_info != 0) return;
-  __shared__ float tile[64][33];
-  const int c0 = blockIdx.x * 32;
-  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
-  for (int m = ty; m < 64; m += 8) {
-    const int c = c0 + tx;
-    float x = 0.f;
-    if (m < b && c < k) {
-      x = A[(int64_t)(j0 + m) * k + c];
-      if (c >= j0 && c < j0 + b && c - j0 < m) x = 0.f;
-    }
-    tile[m][tx] = x;
-  }
-  __syncthreads();
-  for (int cc = ty; cc < 32; cc += 8) {
-    const int c = c0 + cc;
-    if (c >= k) continue;
-    for (int m = tx; m < 64; m += 32) {
-      float h, l;
-      split_tf32(tile[m][cc], h, l);
-      hi[(int64_t)c * 64 + m] = h;
-      lo[(int64_t)c * 64 + m] = l;
     }
   }
 }
@@ -411,24 +356,24 @@ __global__ void split_rowblock_t_kernel(const float* __restrict__ A, int k, int 
 
 bool tc_update_supported(int64_t k) { return k % 4 == 0 && encode_fn() != nullptr; }
 
-gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float* hi,
-                               float* lo, int64_t ldo, cudaStream_t s) {
+gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float sign,
+                               float* hi, float* lo, int64_t ldo, cudaStream_t s) {
   if (rows <= 0 || cols <= 0) return GPTQ_OK;
   dim3 grid((unsigned)cdiv(cols, 32), (unsigned)cdiv(rows, 32));
-  split_transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(src, lds, rows, cols, hi, lo, ldo);
+  split_transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(src, lds, rows, cols, sign, hi, lo, ldo);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
 }
 
 // Wt[0:r, e:k] -= Err[0:r, 0:B] * U[s:s+B, e:k]   (Err_hi/lo: r x B, ld B;
-// Ut_hi/lo: the transposed split of U, k x k).  A timeout sets
+// nut_hi/lo: the split of -U^T, k x k).  A timeout sets
 // *d_status = GPTQ_ERR_TIMEOUT.
-gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* ut_hi,
-                              const float* ut_lo, float* Wt, int r, int k, int s0, int e,
+gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* nut_hi,
+                              const float* nut_lo, float* Wt, int r, int k, int s0, int e,
                               int32_t* d_status, cudaStream_t s) {
   CUtensorMap ah, al, bh, bl, dm;
   if (!make_map(&ah, err_hi, B, r, B, TX_M) || !make_map(&al, err_lo, B, r, B, TX_M) ||
-      !make_map(&bh, ut_hi, k, k, k, TX_N) || !make_map(&bl, ut_lo, k, k, k, TX_N) ||
+      !make_map(&bh, nut_hi, k, k, k, TX_N) || !make_map(&bl, nut_lo, k, k, k, TX_N) ||
       !make_map(&dm, Wt, k, r, k, TX_M))
     return GPTQ_ERR_INVALID_ARG;
   TxArgs a;
@@ -452,19 +397,18 @@ gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, c
   return launch(ah, al, bh, bl, dm, a, s);
 }
 
-// Rows [0, j0) of the k x k work matrix A += sign * R^T R (see the file
-// comment), R = A[j0:j0+b, :] split transposed into rt_hi / rt_lo (k x 64
-// scratch).  A timeout sets *d_info = k + 1.
-gptq_status tc_rank_update(float* A, int k, int j0, int b, float* rt_hi, float* rt_lo,
-                           int32_t* d_info, cudaStream_t s) {
+// Rows [0, j0) of the k x k work matrix A += R^T S (see the file comment):
+// r_hi / r_lo = row block J transposed and split (k x 64, r[c][m] =
+// A[j0 + m][c]), read for c < j0 (the rows of the update); s_hi / s_lo = the
+// same with columns c < j0 negated (the columns of the update).  Both written
+// by the caller.  A timeout sets *d_info = k + 1.
+gptq_status tc_rank_update(float* A, int k, int j0, int b, const float* s_hi, const float* s_lo,
+                           const float* r_hi, const float* r_lo, int32_t* d_info, cudaStream_t s) {
   if (j0 <= 0) return GPTQ_OK;
-  split_rowblock_t_kernel<<<(unsigned)cdiv(k, 32), dim3(32, 8), 0, s>>>(A, k, j0, b, rt_hi, rt_lo,
-                                                                        d_info);
-  GPTQ_CHECK_LAUNCH();
   CUtensorMap ah, al, bh, bl, dm;
   // D's map ends at row j0: rows at and below the current row block are never touched
-  if (!make_map(&ah, rt_hi, 64, k, 64, TX_M) || !make_map(&al, rt_lo, 64, k, 64, TX_M) ||
-      !make_map(&bh, rt_hi, 64, k, 64, TX_N) || !make_map(&bl, rt_lo, 64, k, 64, TX_N) ||
+  if (!make_map(&ah, r_hi, 64, j0, 64, TX_M) || !make_map(&al, r_lo, 64, j0, 64, TX_M) ||
+      !make_map(&bh, s_hi, 64, k, 64, TX_N) || !make_map(&bl, s_lo, 64, k, 64, TX_N) ||
       !make_map(&dm, A, k, j0, k, TX_M))
     return GPTQ_ERR_INVALID_ARG;
   TxArgs a;
