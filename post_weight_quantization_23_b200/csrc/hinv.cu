@@ -14,7 +14,8 @@
 // (rows above the processed part) and turns into U row block by row block.
 // Blocks of HV_B = 64 indices, from the last one up; step J = [j0, j1), e = j1:
 //   K1 diag    L_JJ from the Schur-updated diagonal block (lower part) and
-//              U_JJ = (L_JJ^T)^-1, written to A[J, J] (upper) and the scratch.
+//              U_JJ = (L_JJ^T)^-1, written to A[J, J] (upper) and the scratch
+//              (blocked in 16 x 16 pieces inside one CTA).
 //   K2 panel   P = L[J, 0:j0] = U_JJ * Hp[J, 0:j0]   (in place, lower part),
 //      and     U[J, e:] = -U_JJ * Y[J, e:]          (in place, upper part):
 //              V = [[V_JJ, V_J*], [0, V_**]] gives U_J* = -V_JJ^-1 V_J* U_**.
@@ -168,114 +169,202 @@ __device__ __forceinline__ void hv_split_tf32(float x, float& hi, float& lo) {
 
 __device__ __forceinline__ void set_info(int32_t* d_info, int idx) { atomicCAS(d_info, 0, idx + 1); }
 
-// K1: factor the diagonal block (lower storage, A_JJ = L^T L with L lower)
-// and invert V = L^T: U_JJ = V^-1 (upper), written to the scratch and to the
-// upper part of A[J, J].  One CTA of 256 threads.
-//   factor, c = b-1 .. 0:  a_ij -= a_ci a_cj / a_cc  (j <= i < c), then
-//   L_cj = a_cj / sqrt(a_cc) (j < c), L_cc = sqrt(a_cc);
-//   inverse, i = b-1 .. 0: U_ii = 1 / L_ii, U_ic = -(sum_{m=i+1..c} L_mi U_mc) / L_ii.
-// Factor: thread (ri = t / 4, jq = t % 4) keeps a[ri][jq + 4q] (q < 16) in
-// registers and writes them through to shared memory, where step c reads the
-// pivot row c; one barrier per step.  Inverse: thread (c = t / 4, part = t % 4)
-// keeps U[part + 4u][c] (u < 16) in registers; the four threads of a column
-// combine their partial sums with shuffles, so the inverse needs no barrier.
+// K1: the diagonal block: U_JJ with U_JJ^T U_JJ = A_JJ^-1, from the lower
+// part of the Schur-updated A_JJ.  One CTA of 256 threads.
+// With B = P A_JJ P (P reverses the indices), A_JJ = L^T L (L lower, the
+// factorisation that starts from the last index) becomes the ordinary lower
+// Cholesky B = M M^T with M = P L^T P, and U_JJ = (L^T)^-1 = P M^-1 P.  The
+// kernel factors B and inverts M in 16 x 16 blocks (rows and columns past b
+// padded with the identity):
+//   factor, block column kb = 0..3:
+//     M_kk = chol(B_kk)                 one warp, column by column
+//     M_ik = B_ik M_kk^-T   (i > kb)    one thread per row, forward substitution
+//     B_ij -= M_ik M_jk^T   (kb < j <= i) the whole CTA
+//   inverse N = M^-1:
+//     N_kk = M_kk^-1                    four warps, one block each, one lane per column
+//     N_ik = -N_ii sum_{m=k}^{i-1} M_im N_mk, by block distance i - k = 1, 2, 3
+// U_JJ goes to the scratch, to the upper part of A[J, J] and, transposed and
+// split into tf32 hi / lo, to the rank update's operand.
+// Lower Cholesky of a 16 x 16 block held by rows: lane i (of 16; the upper
+// half of the warp mirrors it) keeps row i in x[0..15]; column C of the
+// factor is broadcast by shuffles.  first_bad = the first pivot that is not
+// positive and finite (every lane sees the same pivots), else unchanged.
+// The column steps are unrolled by template recursion, which keeps x in
+// registers inside the caller's block loop.
+template <int C>
+struct Chol16 {
+  // rdiag[C] receives 1 / M_CC (from lane C)
+  __device__ __forceinline__ static void run(float (&x)[16], int i, int& first_bad,
+                                             float* rdiag) {
+    const float p = __shfl_sync(0xffffffffu, x[C], C);
+    if ((!(p > 0.f) || !isfinite(p)) && first_bad < 0) first_bad = C;
+    const float rd = rsqrtf(p);  // 1 / sqrt(p), within 2 ulp
+    const float d = p * rd;
+    if (i == C) rdiag[C] = rd;
+    x[C] = (i > C) ? x[C] * rd : (i == C ? d : x[C]);
+#pragma unroll
+    for (int j = C + 1; j < 16; ++j) {
+      const float ljc = __shfl_sync(0xffffffffu, x[C], j);
+      x[j] = (j <= i) ? fmaf(-x[C], ljc, x[j]) : x[j];
+    }
+    Chol16<C + 1>::run(x, i, first_bad, rdiag);
+  }
+};
+template <>
+struct Chol16<16> {
+  __device__ __forceinline__ static void run(float (&)[16], int, int&, float*) {}
+};
+
+constexpr int K1_BS = 16;                 // block size
+constexpr int K1_NB = HV_B / K1_BS;       // blocks per side
+constexpr int K1_LD = HV_B + 1;
+
 __global__ void __launch_bounds__(256)
 chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
                      float* __restrict__ ujj, float* __restrict__ st_hi,
                      float* __restrict__ st_lo, int32_t* __restrict__ d_info) {
   if (*d_info != 0) return;
-  __shared__ float S[HV_B][HV_B + 1];
-  __shared__ float rdg[HV_B];
-  const int t = threadIdx.x;
-  const int ri = t >> 2, jq = t & 3;
-  float r[HV_B / 4];
+  __shared__ float S[HV_B][K1_LD];                 // B, then M (lower part)
+  __shared__ float T[HV_B][K1_LD];                 // N = M^-1 (lower part)
+  __shared__ float X[K1_NB - 1][K1_BS][K1_BS + 1];  // sums of one inverse round
+  __shared__ float rdg[HV_B];                        // 1 / M_ii
+  __shared__ int fail;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  for (int e = t; e < HV_B * HV_B; e += 256) {
+    const int i = e / HV_B, j = e % HV_B;
+    S[i][j] = (i == j && i >= b) ? 1.f : 0.f;
+  }
+  if (t == 0) fail = -1;
+  __syncthreads();
+  // B[b-1-ca][b-1-ra] = A[ra][ca] for ca <= ra < b (coalesced along ca; all
+  // loads issued before the stores)
+  {
+    float v[HV_B * HV_B / 256];
 #pragma unroll
-  for (int q = 0; q < HV_B / 4; ++q) {
-    const int j = jq + 4 * q;
-    r[q] = (ri < b && j <= ri) ? A[(int64_t)(j0 + ri) * k + j0 + j] : 0.f;
-    S[ri][j] = r[q];
+    for (int q = 0; q < HV_B * HV_B / 256; ++q) {
+      const int e = t + 256 * q, ra = e / HV_B, ca = e % HV_B;
+      v[q] = (ra < b && ca <= ra) ? A[(int64_t)(j0 + ra) * k + j0 + ca] : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < HV_B * HV_B / 256; ++q) {
+      const int e = t + 256 * q, ra = e / HV_B, ca = e % HV_B;
+      if (ra < b && ca <= ra) S[b - 1 - ca][b - 1 - ra] = v[q];
+    }
   }
   __syncthreads();
-  int fail = -1;
-  for (int c = b - 1; c >= 0; --c) {
-    const float p = S[c][c];
-    if (!(p > 0.f) || !isfinite(p)) {
-      fail = c;  // every thread reads the same pivot: the exit is uniform
-      break;
+
+  for (int kb = 0; kb < K1_NB; ++kb) {
+    const int c0 = kb * K1_BS;
+    if (warp == 0) {
+      // lane i < 16 keeps row i of the block in registers; column c of the
+      // factor is broadcast by shuffles (the block is fully unrolled)
+      const int i = lane & (K1_BS - 1);
+      float x[K1_BS];
+#pragma unroll
+      for (int j = 0; j < K1_BS; ++j) x[j] = S[c0 + i][c0 + j];
+      int first_bad = -1;
+      Chol16<0>::run(x, i, first_bad, rdg + c0);
+      if (first_bad >= 0 && lane == 0) fail = c0 + first_bad;
+      if (lane < K1_BS) {
+#pragma unroll
+        for (int j = 0; j < K1_BS; ++j)
+          if (j <= i) S[c0 + i][c0 + j] = x[j];
+      }
     }
-    if (ri < c) {
-      const float f = S[c][ri] * __frcp_rn(p);
-      float cv[HV_B / 4];
+    __syncthreads();
+    if (fail >= 0) break;
+    const int r0 = c0 + K1_BS, nr = HV_B - r0;
+    if (t < nr) {
+      // x M_kk^T = b_i by columns: fix x_m, then take it out of the later ones
+      const int i = r0 + t;
+      float x[K1_BS];
 #pragma unroll
-      for (int q = 0; q < HV_B / 4; ++q) cv[q] = S[c][jq + 4 * q];
+      for (int m = 0; m < K1_BS; ++m) x[m] = S[i][c0 + m];
 #pragma unroll
-      for (int q = 0; q < HV_B / 4; ++q) {
-        const int j = jq + 4 * q;
-        if (j <= ri) {
-          r[q] = fmaf(-f, cv[q], r[q]);
-          S[ri][j] = r[q];
-        }
+      for (int m = 0; m < K1_BS; ++m) {
+        x[m] *= rdg[c0 + m];
+#pragma unroll
+        for (int q = m + 1; q < K1_BS; ++q) x[q] = fmaf(-x[m], S[c0 + q][c0 + m], x[q]);
+      }
+#pragma unroll
+      for (int m = 0; m < K1_BS; ++m) S[i][c0 + m] = x[m];
+    }
+    __syncthreads();
+    for (int e = t; e < nr * nr; e += 256) {
+      const int ii = e / nr, jj = e % nr;
+      if (jj <= ii) {
+        float acc = S[r0 + ii][r0 + jj];
+#pragma unroll
+        for (int m = 0; m < K1_BS; ++m) acc = fmaf(-S[r0 + ii][c0 + m], S[r0 + jj][c0 + m], acc);
+        S[r0 + ii][r0 + jj] = acc;
       }
     }
     __syncthreads();
   }
   if (fail >= 0) {
-    if (t == 0) set_info(d_info, j0 + fail);
+    if (t == 0) set_info(d_info, j0 + (b - 1 - fail));
     return;
   }
-  // L: scale each row by 1 / sqrt(a_ii); S then holds L
-  if (ri < b) {
-    const float d = sqrtf(S[ri][ri]);
-    const float rd = __frcp_rn(d);
+
+  // inverse of M: diagonal blocks
+  if (warp < K1_NB && lane < K1_BS) {
+    const int c0 = warp * K1_BS, j = lane;
+    // column j of M_kk^-1: fix x_i, then take it out of the later rows
+    float x[K1_BS];
 #pragma unroll
-    for (int q = 0; q < HV_B / 4; ++q) {
-      const int j = jq + 4 * q;
-      if (j < ri) r[q] *= rd;
-      else if (j == ri) r[q] = d;
+    for (int i = 0; i < K1_BS; ++i) x[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int i = 0; i < K1_BS; ++i) {
+      x[i] = (i < j) ? 0.f : x[i] * rdg[c0 + i];
+#pragma unroll
+      for (int q = i + 1; q < K1_BS; ++q) x[q] = fmaf(-S[c0 + q][c0 + i], x[i], x[q]);
     }
-    if (jq == 0) rdg[ri] = rd;
+#pragma unroll
+    for (int i = 0; i < K1_BS; ++i) T[c0 + i][c0 + j] = x[i];
   }
   __syncthreads();
+  // off-diagonal blocks by distance d
+  for (int d = 1; d < K1_NB; ++d) {
+    const int nblk = K1_NB - d;
+    for (int e = t; e < nblk * K1_BS * K1_BS; e += 256) {
+      const int q = e / (K1_BS * K1_BS), r = (e / K1_BS) % K1_BS, c = e % K1_BS;
+      const int ib = q + d;
+      float acc = 0.f;
+      for (int mb = q; mb < ib; ++mb)
 #pragma unroll
-  for (int q = 0; q < HV_B / 4; ++q) {
-    const int j = jq + 4 * q;
-    if (j <= ri) S[ri][j] = r[q];
-  }
-  __syncthreads();
-  // inverse of V = L^T by rows from the bottom; y[u] = U[part + 4u][c]
-  const int c = t >> 2, part = t & 3;
-  float y[HV_B / 4];
-#pragma unroll
-  for (int u = 0; u < HV_B / 4; ++u) y[u] = 0.f;
-#pragma unroll
-  for (int i = HV_B - 1; i >= 0; --i) {
-    if (i < b) {  // uniform
-      float sum = 0.f;
-#pragma unroll
-      for (int u = 0; u < HV_B / 4; ++u) {
-        const int m = part + 4 * u;
-        if (m > i && m <= c && m < b) sum = fmaf(S[m][i], y[u], sum);
-      }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-      if ((i & 3) == part && c < b) {
-        const float rv = rdg[i];
-        if (c == i) y[i >> 2] = rv;
-        else if (c > i) y[i >> 2] = -sum * rv;
-      }
+        for (int m = 0; m < K1_BS; ++m)
+          acc = fmaf(S[ib * K1_BS + r][mb * K1_BS + m], T[mb * K1_BS + m][q * K1_BS + c], acc);
+      X[q][r][c] = acc;
     }
-  }
+    __syncthreads();
+    for (int e = t; e < nblk * K1_BS * K1_BS; e += 256) {
+      const int q = e / (K1_BS * K1_BS), r = (e / K1_BS) % K1_BS, c = e % K1_BS;
+      const int ib = q + d;
+      float acc = 0.f;
 #pragma unroll
-  for (int u = 0; u < HV_B / 4; ++u) {
-    const int i = part + 4 * u;
-    ujj[i * HV_B + c] = y[u];
-    if (i < b && c < b && c >= i) A[(int64_t)(j0 + i) * k + j0 + c] = y[u];
-    if (st_hi != nullptr && c < b) {
-      // rank-update operand s[j0 + c][i] = U_JJ[i][c] (upper triangle, 0 below it)
+      for (int m = 0; m < K1_BS; ++m)
+        if (m <= r) acc = fmaf(T[ib * K1_BS + r][ib * K1_BS + m], X[q][m][c], acc);
+      T[ib * K1_BS + r][q * K1_BS + c] = -acc;
+    }
+    __syncthreads();
+  }
+  // U_JJ[iu][cu] = N[b-1-iu][b-1-cu] (iu <= cu < b)
+  for (int e = t; e < HV_B * HV_B; e += 256) {
+    const int iu = e / HV_B, cu = e % HV_B;
+    const bool in = (iu <= cu && cu < b);
+    const float u = in ? T[b - 1 - iu][b - 1 - cu] : 0.f;
+    ujj[e] = u;
+    if (in) A[(int64_t)(j0 + iu) * k + j0 + cu] = u;
+  }
+  if (st_hi != nullptr) {
+    // rank-update operand s[j0 + cu][iu] = U_JJ[iu][cu]  (columns of block J, sign +)
+    for (int e = t; e < b * HV_B; e += 256) {
+      const int cu = e / HV_B, iu = e % HV_B;
+      const float u = (iu <= cu) ? T[b - 1 - iu][b - 1 - cu] : 0.f;
       float h, l;
-      hv_split_tf32((i < b && c >= i) ? y[u] : 0.f, h, l);
-      st_hi[(int64_t)(j0 + c) * HV_B + i] = h;
-      st_lo[(int64_t)(j0 + c) * HV_B + i] = l;
+      hv_split_tf32(u, h, l);
+      st_hi[(int64_t)(j0 + cu) * HV_B + iu] = h;
+      st_lo[(int64_t)(j0 + cu) * HV_B + iu] = l;
     }
   }
 }
@@ -285,10 +374,10 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
 //     (lower part of row block J, in place).
 //   CTAs [n_pan, ...): 64-column tiles c0 of [e, k): U[J, c] = -U_JJ * Y[J, c]
 //     (upper part of row block J, in place).
-//   CTAs [n_pan + n_row, ...): zero 64-row pieces of the strip
-//     A[0:j0, j0:j1], where Y's columns of block J start accumulating in this
-//     step's update (the tensor-core Schur update writes the whole square
-//     [0, j0)^2 and leaves values above its diagonal).
+//   With the tensor-core update (st_hi given) each panel CTA also zeroes rows
+//     [c0, c0 + 64) of the strip A[0:j0, j0:j1], where Y's columns of block J
+//     start accumulating in this step's update (the tensor-core Schur update
+//     writes the whole square [0, j0)^2 and leaves values above its diagonal).
 // Each CTA reads its whole 64 x 64 tile before writing it.  Thread
 // (r = t / 4, cq = t % 4) computes row r, columns cq + 4q.  When st_hi is
 // given, the new row-block tile also goes out transposed and split into tf32
@@ -300,14 +389,7 @@ panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* 
                       float* __restrict__ rt_hi, float* __restrict__ rt_lo,
                       const int32_t* __restrict__ d_info) {
   if (*d_info != 0) return;
-  if ((int)blockIdx.x >= n_pan + n_row) {
-    const int z0 = ((int)blockIdx.x - n_pan - n_row) * HV_B;
-    for (int e = threadIdx.x; e < HV_B * HV_B; e += 256) {
-      const int i = z0 + e / HV_B, c = j0 + e % HV_B;
-      if (i < j0 && c < j0 + b) A[(int64_t)i * k + c] = 0.f;
-    }
-    return;
-  }
+  (void)n_row;
   __shared__ __align__(16) float Us[HV_B][HV_B + 4];  // row stride 68: conflict-free row reads
   __shared__ float Hs[HV_B][HV_B + 1];                // row stride 65: conflict-free columns
   const int t = threadIdx.x;
@@ -366,6 +448,13 @@ panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* 
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj)
         if (c0 + j + jj < cend) dst[jj] = Hs[i][j + jj];
+    }
+  }
+  if (st_hi != nullptr && pan) {
+#pragma unroll 4
+    for (int e = t; e < HV_B * HV_B; e += 256) {
+      const int i = c0 + e / HV_B, c = j0 + e % HV_B;
+      if (i < j0 && c < j0 + b) A[(int64_t)i * k + c] = 0.f;
     }
   }
   if (st_hi != nullptr) {
@@ -543,9 +632,8 @@ gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cf
     GPTQ_CHECK_LAUNCH();
     const int n_pan = (int)cdiv(j0, HV_B);
     const int n_row = (int)cdiv(k - j1, HV_B);
-    const int n_zero = tcs ? n_pan : 0;
-    if (n_pan + n_row + n_zero > 0) {
-      panel_rowblock_kernel<<<(unsigned)(n_pan + n_row + n_zero), 256, 0, s>>>(
+    if (n_pan + n_row > 0) {
+      panel_rowblock_kernel<<<(unsigned)(n_pan + n_row), 256, 0, s>>>(
           U, k, j0, b, sc.ujj, n_pan, n_row, tcs ? sc.s_hi : nullptr, tcs ? sc.s_lo : nullptr,
           tcs ? sc.r_hi : nullptr, tcs ? sc.r_lo : nullptr, d_info);
       GPTQ_CHECK_LAUNCH();
