@@ -42,6 +42,13 @@ METRIC = "GPTQ layer quantize Mweights/s end-to-end"
 UNIT = "Mweights/s"
 
 
+# DRAM traffic of hessian_tc_kernel from one ncu capture (32768 tokens, k = 4096):
+# 649.7 MB read + 67.7 MB written; both grow with the token count (X re-reads and
+# the per-unit flushes of H), so a launch over n tokens moves about n times this.
+HESS_TRAFFIC_K = 4096
+HESS_TRAFFIC_BYTES_PER_TOKEN = (649.7e6 + 67.7e6) / 32768
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -140,7 +147,8 @@ def barrier(world):
 def max_over_ranks(x, world):
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -344,9 +352,17 @@ def native_arm(args, spec, world, rank, local):
     flops = float(spec.n) * spec.k * (spec.k + 1)  # symmetric triangle, algorithmic
     t_h = phase[0] / 1e3
     achieved = flops / t_h / 1e12
+    traffic = args.traffic
+    if traffic is None and spec.k == HESS_TRAFFIC_K:
+        # DRAM bytes of one capture of this kernel at k = 4096, scaled to n tokens
+        traffic = HESS_TRAFFIC_BYTES_PER_TOKEN * spec.n
     roofline = {"bound": "tensor", "kernel": "gptq_hessian_accumulate (X^T X)",
                 "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_sustained"], "traffic": args.traffic,
+                "frac": achieved / peaks["bf16_sustained"], "traffic": traffic,
+                "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of "
+                                   "hessian_tc_kernel, 32768 x 4096 capture, scaled by tokens "
+                                   "(profiles/hessian_tc_kernel_q_proj_32k_tokens.md)")
+                if traffic is not None and args.traffic is None else None,
                 "peak_kind": f"bf16 dense sustained ({peaks['source']}); f16 has the same nominal rate",
                 "algorithmic": f"n*k*(k+1) = {flops:.4g} flop per launch"}
     sweep_bytes = sweep_model_bytes(spec)
