@@ -60,7 +60,7 @@ def _peaks():
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi every 100 ms while
+    """Samples SM clocks and throttle reasons with nvidia-smi every 25 ms while
     the timed region runs (all GPUs are queried; the one on this process's
     PCI bus is kept, or the only one)."""
     FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -81,7 +81,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "25"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.first = self.proc.stdout.readline()
         except Exception:
             self.proc = None
