@@ -177,7 +177,7 @@ __device__ __forceinline__ void set_info(int32_t* d_info, int idx) { atomicCAS(d
 // kernel factors B and inverts M in 16 x 16 blocks (rows and columns past b
 // padded with the identity):
 //   factor, block column kb = 0..3:
-//     M_kk = chol(B_kk)                 one warp, column by column
+//     M_kk = chol(B_kk)                 one warp, the block in registers
 //     M_ik = B_ik M_kk^-T   (i > kb)    one thread per row, forward substitution
 //     B_ij -= M_ik M_jk^T   (kb < j <= i) the whole CTA
 //   inverse N = M^-1:
@@ -185,34 +185,35 @@ __device__ __forceinline__ void set_info(int32_t* d_info, int idx) { atomicCAS(d
 //     N_ik = -N_ii sum_{m=k}^{i-1} M_im N_mk, by block distance i - k = 1, 2, 3
 // U_JJ goes to the scratch, to the upper part of A[J, J] and, transposed and
 // split into tf32 hi / lo, to the rank update's operand.
-// Lower Cholesky of a 16 x 16 block held by rows: lane i (of 16; the upper
-// half of the warp mirrors it) keeps row i in x[0..15]; column C of the
-// factor is broadcast by shuffles.  first_bad = the first pivot that is not
-// positive and finite (every lane sees the same pivots), else unchanged.
-// The column steps are unrolled by template recursion, which keeps x in
-// registers inside the caller's block loop.
+// Lower Cholesky of a 16 x 16 block whose lower triangle is held whole in
+// registers, a[i (i + 1) / 2 + j] = B_ij (j <= i); every lane of the warp
+// runs it (no communication).  Column C: pivot, scale, then the rank-1
+// update of the trailing triangle -- all independent instructions.  rd[C]
+// receives 1 / M_CC; first_bad = the first pivot that is not positive and
+// finite, else unchanged.  Unrolled by template recursion so that a stays
+// in registers inside the caller's block loop.
+__device__ __forceinline__ constexpr int tri(int i, int j) { return i * (i + 1) / 2 + j; }
+
 template <int C>
 struct Chol16 {
-  // rdiag[C] receives 1 / M_CC (from lane C)
-  __device__ __forceinline__ static void run(float (&x)[16], int i, int& first_bad,
-                                             float* rdiag) {
-    const float p = __shfl_sync(0xffffffffu, x[C], C);
+  __device__ __forceinline__ static void run(float (&a)[136], float (&rd)[16], int& first_bad) {
+    const float p = a[tri(C, C)];
     if ((!(p > 0.f) || !isfinite(p)) && first_bad < 0) first_bad = C;
-    const float rd = rsqrtf(p);  // 1 / sqrt(p), within 2 ulp
-    const float d = p * rd;
-    if (i == C) rdiag[C] = rd;
-    x[C] = (i > C) ? x[C] * rd : (i == C ? d : x[C]);
+    const float r = rsqrtf(p);  // 1 / sqrt(p), within 2 ulp
+    rd[C] = r;
+    a[tri(C, C)] = p * r;
 #pragma unroll
-    for (int j = C + 1; j < 16; ++j) {
-      const float ljc = __shfl_sync(0xffffffffu, x[C], j);
-      x[j] = (j <= i) ? fmaf(-x[C], ljc, x[j]) : x[j];
-    }
-    Chol16<C + 1>::run(x, i, first_bad, rdiag);
+    for (int i = C + 1; i < 16; ++i) a[tri(i, C)] *= r;
+#pragma unroll
+    for (int i = C + 1; i < 16; ++i)
+#pragma unroll
+      for (int j = C + 1; j <= i; ++j) a[tri(i, j)] = fmaf(-a[tri(i, C)], a[tri(j, C)], a[tri(i, j)]);
+    Chol16<C + 1>::run(a, rd, first_bad);
   }
 };
 template <>
 struct Chol16<16> {
-  __device__ __forceinline__ static void run(float (&)[16], int, int&, float*) {}
+  __device__ __forceinline__ static void run(float (&)[136], float (&)[16], int&) {}
 };
 
 constexpr int K1_BS = 16;                 // block size
@@ -256,19 +257,22 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
   for (int kb = 0; kb < K1_NB; ++kb) {
     const int c0 = kb * K1_BS;
     if (warp == 0) {
-      // lane i < 16 keeps row i of the block in registers; column c of the
-      // factor is broadcast by shuffles (the block is fully unrolled)
-      const int i = lane & (K1_BS - 1);
-      float x[K1_BS];
+      // every lane factors the whole block in registers; lane 0 writes it back
+      float a[136], rd[16];
 #pragma unroll
-      for (int j = 0; j < K1_BS; ++j) x[j] = S[c0 + i][c0 + j];
+      for (int i = 0; i < 16; ++i)
+#pragma unroll
+        for (int j = 0; j <= i; ++j) a[tri(i, j)] = S[c0 + i][c0 + j];
       int first_bad = -1;
-      Chol16<0>::run(x, i, first_bad, rdg + c0);
-      if (first_bad >= 0 && lane == 0) fail = c0 + first_bad;
-      if (lane < K1_BS) {
+      Chol16<0>::run(a, rd, first_bad);
+      if (lane == 0) {
 #pragma unroll
-        for (int j = 0; j < K1_BS; ++j)
-          if (j <= i) S[c0 + i][c0 + j] = x[j];
+        for (int i = 0; i < 16; ++i) {
+#pragma unroll
+          for (int j = 0; j <= i; ++j) S[c0 + i][c0 + j] = a[tri(i, j)];
+          rdg[c0 + i] = rd[i];
+        }
+        if (first_bad >= 0) fail = c0 + first_bad;
       }
     }
     __syncthreads();
@@ -369,109 +373,105 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
   }
 }
 
-// K2, one launch, two independent roles:
-//   CTAs [0, n_pan): 64-column tiles c0 of [0, j0): P[:, c] = U_JJ * A[J, c]
+// K2, one launch, two independent roles (16-column tiles, so that the launch
+// fills the GPU; each CTA reads its whole 64 x 16 tile before writing it):
+//   CTAs [0, n_pan): columns c0 .. c0+15 of [0, j0): P[:, c] = U_JJ * A[J, c]
 //     (lower part of row block J, in place).
-//   CTAs [n_pan, ...): 64-column tiles c0 of [e, k): U[J, c] = -U_JJ * Y[J, c]
+//   CTAs [n_pan, ...): columns c0 .. c0+15 of [e, k): U[J, c] = -U_JJ * Y[J, c]
 //     (upper part of row block J, in place).
 //   With the tensor-core update (st_hi given) each panel CTA also zeroes rows
-//     [c0, c0 + 64) of the strip A[0:j0, j0:j1], where Y's columns of block J
+//     [c0, c0 + 16) of the strip A[0:j0, j0:j1], where Y's columns of block J
 //     start accumulating in this step's update (the tensor-core Schur update
 //     writes the whole square [0, j0)^2 and leaves values above its diagonal).
-// Each CTA reads its whole 64 x 64 tile before writing it.  Thread
-// (r = t / 4, cq = t % 4) computes row r, columns cq + 4q.  When st_hi is
-// given, the new row-block tile also goes out transposed and split into tf32
-// hi / lo in the rank update's operand layout: st[c][m] = -R[m][c] for c < j0
-// and +R[m][c] above, rt[c][m] = R[m][c] for c < j0.
+// Thread (r = t / 4, cq = t % 4) computes row r, columns 4 cq .. 4 cq + 3.  When
+// st_hi is given, the new row-block tile also goes out transposed and split
+// into tf32 hi / lo in the rank update's operand layout: st[c][m] = -R[m][c]
+// for c < j0 and +R[m][c] above, rt[c][m] = R[m][c] for c < j0.
+constexpr int K2_W = 16;  // columns per CTA
+
 __global__ void __launch_bounds__(256)
 panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* __restrict__ ujj,
-                      int n_pan, int n_row, float* __restrict__ st_hi, float* __restrict__ st_lo,
+                      int n_pan, float* __restrict__ st_hi, float* __restrict__ st_lo,
                       float* __restrict__ rt_hi, float* __restrict__ rt_lo,
                       const int32_t* __restrict__ d_info) {
   if (*d_info != 0) return;
-  (void)n_row;
   __shared__ __align__(16) float Us[HV_B][HV_B + 4];  // row stride 68: conflict-free row reads
-  __shared__ float Hs[HV_B][HV_B + 1];                // row stride 65: conflict-free columns
+  __shared__ __align__(16) float Hs[HV_B][K2_W + 4];  // row stride 20: aligned float4 rows
+  __shared__ float Os[HV_B][K2_W + 1];                // results; stride 17: conflict-free columns
   const int t = threadIdx.x;
   const bool pan = (int)blockIdx.x < n_pan;
-  const int c0 = pan ? blockIdx.x * HV_B : j0 + b + (blockIdx.x - n_pan) * HV_B;
+  const int c0 = pan ? blockIdx.x * K2_W : j0 + b + (blockIdx.x - n_pan) * K2_W;
   const int cend = pan ? j0 : k;
   const float sign = pan ? 1.0f : -1.0f;
   const bool vec = (k % 4 == 0);
+  const int r = t >> 2, j = (t & 3) * 4;  // this thread's row and first column in the tile
   {
-    float4 uv[4], hv[4];
+    float4 uv[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int e4 = t + 256 * q, i = e4 >> 4, j = (e4 & 15) * 4;
-      uv[q] = reinterpret_cast<const float4*>(ujj)[e4];
-      const float* src = A + (int64_t)(j0 + i) * k + c0 + j;
-      if (i < b && vec && c0 + j + 3 < cend) {
-        hv[q] = *reinterpret_cast<const float4*>(src);
-      } else {
-        hv[q].x = (i < b && c0 + j < cend) ? src[0] : 0.f;
-        hv[q].y = (i < b && c0 + j + 1 < cend) ? src[1] : 0.f;
-        hv[q].z = (i < b && c0 + j + 2 < cend) ? src[2] : 0.f;
-        hv[q].w = (i < b && c0 + j + 3 < cend) ? src[3] : 0.f;
-      }
+    for (int q = 0; q < 4; ++q) uv[q] = reinterpret_cast<const float4*>(ujj)[t + 256 * q];
+    float4 hv;
+    const float* src = A + (int64_t)(j0 + r) * k + c0 + j;
+    if (r < b && vec && c0 + j + 3 < cend) {
+      hv = *reinterpret_cast<const float4*>(src);
+    } else {
+      hv.x = (r < b && c0 + j < cend) ? src[0] : 0.f;
+      hv.y = (r < b && c0 + j + 1 < cend) ? src[1] : 0.f;
+      hv.z = (r < b && c0 + j + 2 < cend) ? src[2] : 0.f;
+      hv.w = (r < b && c0 + j + 3 < cend) ? src[3] : 0.f;
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int e4 = t + 256 * q, i = e4 >> 4, j = (e4 & 15) * 4;
-      *reinterpret_cast<float4*>(&Us[i][j]) = uv[q];
-      Hs[i][j] = hv[q].x, Hs[i][j + 1] = hv[q].y, Hs[i][j + 2] = hv[q].z, Hs[i][j + 3] = hv[q].w;
+      const int e4 = t + 256 * q;
+      *reinterpret_cast<float4*>(&Us[e4 >> 4][(e4 & 15) * 4]) = uv[q];
     }
+    *reinterpret_cast<float4*>(&Hs[r][j]) = hv;
   }
   __syncthreads();
-  const int r = t >> 2, cq = t & 3;
-  float acc[HV_B / 4];
-#pragma unroll
-  for (int q = 0; q < HV_B / 4; ++q) acc[q] = 0.f;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   if (r < b) {
     for (int m = r; m < b; ++m) {
       const float u = Us[r][m];
-#pragma unroll
-      for (int q = 0; q < HV_B / 4; ++q) acc[q] = fmaf(u, Hs[m][cq + 4 * q], acc[q]);
+      const float4 h = *reinterpret_cast<const float4*>(&Hs[m][j]);
+      a0 = fmaf(u, h.x, a0);
+      a1 = fmaf(u, h.y, a1);
+      a2 = fmaf(u, h.z, a2);
+      a3 = fmaf(u, h.w, a3);
     }
   }
-  __syncthreads();
-#pragma unroll
-  for (int q = 0; q < HV_B / 4; ++q) Hs[r][cq + 4 * q] = sign * acc[q];
-  __syncthreads();
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int e4 = t + 256 * q, i = e4 >> 4, j = (e4 & 15) * 4;
-    if (i >= b) continue;
-    float* dst = A + (int64_t)(j0 + i) * k + c0 + j;
+  Os[r][j] = sign * a0, Os[r][j + 1] = sign * a1, Os[r][j + 2] = sign * a2, Os[r][j + 3] = sign * a3;
+  if (r < b) {
+    float* dst = A + (int64_t)(j0 + r) * k + c0 + j;
+    const float o[4] = {sign * a0, sign * a1, sign * a2, sign * a3};
     if (vec && c0 + j + 3 < cend) {
-      *reinterpret_cast<float4*>(dst) = make_float4(Hs[i][j], Hs[i][j + 1], Hs[i][j + 2], Hs[i][j + 3]);
+      *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
     } else {
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj)
-        if (c0 + j + jj < cend) dst[jj] = Hs[i][j + jj];
+        if (c0 + j + jj < cend) dst[jj] = o[jj];
     }
   }
-  if (st_hi != nullptr && pan) {
-#pragma unroll 4
-    for (int e = t; e < HV_B * HV_B; e += 256) {
-      const int i = c0 + e / HV_B, c = j0 + e % HV_B;
+  if (st_hi == nullptr) return;
+  if (pan) {
+    // rows c0 .. c0+15 of the strip A[0:j0, j0:j0+b)
+#pragma unroll
+    for (int q = 0; q < K2_W * HV_B / 256; ++q) {
+      const int e = t + 256 * q, i = c0 + e / HV_B, c = j0 + e % HV_B;
       if (i < j0 && c < j0 + b) A[(int64_t)i * k + c] = 0.f;
     }
   }
-  if (st_hi != nullptr) {
-#pragma unroll 4
-    for (int e = t; e < HV_B * HV_B; e += 256) {
-      const int cc = e >> 6, m = e & 63;
-      if (c0 + cc < cend) {
-        // Hs holds the new row block R (what went to A)
-        const float x = m < b ? Hs[m][cc] : 0.f;
-        float h, l;
-        hv_split_tf32(pan ? -x : x, h, l);  // st = -R for c < j0, +R for c >= j1
-        st_hi[(int64_t)(c0 + cc) * HV_B + m] = h;
-        st_lo[(int64_t)(c0 + cc) * HV_B + m] = l;
-        if (pan) {
-          rt_hi[(int64_t)(c0 + cc) * HV_B + m] = -h;
-          rt_lo[(int64_t)(c0 + cc) * HV_B + m] = -l;
-        }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < K2_W * HV_B / 256; ++q) {
+    const int e = t + 256 * q, cc = e / HV_B, m = e % HV_B;
+    if (c0 + cc < cend) {
+      const float x = m < b ? Os[m][cc] : 0.f;  // the new row block R
+      float h, l;
+      hv_split_tf32(pan ? -x : x, h, l);  // st = -R for c < j0, +R for c >= j1
+      st_hi[(int64_t)(c0 + cc) * HV_B + m] = h;
+      st_lo[(int64_t)(c0 + cc) * HV_B + m] = l;
+      if (pan) {
+        rt_hi[(int64_t)(c0 + cc) * HV_B + m] = -h;
+        rt_lo[(int64_t)(c0 + cc) * HV_B + m] = -l;
       }
     }
   }
@@ -630,11 +630,11 @@ gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cf
     chol_inv_diag_kernel<<<1, 256, 0, s>>>(U, k, j0, b, sc.ujj, tcs ? sc.s_hi : nullptr,
                                            tcs ? sc.s_lo : nullptr, d_info);
     GPTQ_CHECK_LAUNCH();
-    const int n_pan = (int)cdiv(j0, HV_B);
-    const int n_row = (int)cdiv(k - j1, HV_B);
+    const int n_pan = (int)cdiv(j0, K2_W);
+    const int n_row = (int)cdiv(k - j1, K2_W);
     if (n_pan + n_row > 0) {
       panel_rowblock_kernel<<<(unsigned)(n_pan + n_row), 256, 0, s>>>(
-          U, k, j0, b, sc.ujj, n_pan, n_row, tcs ? sc.s_hi : nullptr, tcs ? sc.s_lo : nullptr,
+          U, k, j0, b, sc.ujj, n_pan, tcs ? sc.s_hi : nullptr, tcs ? sc.s_lo : nullptr,
           tcs ? sc.r_hi : nullptr, tcs ? sc.r_lo : nullptr, d_info);
       GPTQ_CHECK_LAUNCH();
     }

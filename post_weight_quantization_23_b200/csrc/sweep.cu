@@ -62,7 +62,7 @@ static size_t sweep_records_bytes(int64_t k, int B) { return (size_t)cdiv(k, B) 
 
 bool tc_update_supported(int64_t k);
 gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float sign,
-                               float* hi, float* lo, int64_t ldo, cudaStream_t s);
+                               int upper_only, float* hi, float* lo, int64_t ldo, cudaStream_t s);
 gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* nut_hi,
                               const float* nut_lo, float* Wt, int r, int k, int s0, int e,
                               int32_t* d_status, cudaStream_t s);
@@ -347,16 +347,18 @@ __global__ void sweep_records_kernel(const float* __restrict__ U, const int32_t*
   float* Ud = Uq + Ly::UQ;
   float* rdg = Ud + Ly::UD;
   int32_t* pcol = (int32_t*)(rdg + SW_MAX_B);
-  for (int e = threadIdx.x; e < Ly::UQ; e += blockDim.x) {
+  // blockIdx.y splits the record's elements between CTAs
+  const int tid = blockIdx.y * blockDim.x + threadIdx.x, nth = gridDim.y * blockDim.x;
+  for (int e = tid; e < Ly::UQ; e += nth) {
     const int i = e / Ly::LDI, rem = e % Ly::LDI, l = rem / Ly::SEG, j = rem % Ly::SEG;
     const int col = l + L * (i / L + j);
     Uq[e] = (j >= 1 && j < Ly::S && i < bw && col < bw) ? U[(int64_t)(s + i) * k + s + col] : 0.f;
   }
-  for (int e = threadIdx.x; e < Ly::UD; e += blockDim.x) {
+  for (int e = tid; e < Ly::UD; e += nth) {
     const int m = e / (L * L), o = (e / L) % L, o2 = e % L;
     Ud[e] = (o2 > o && L * m + o2 < bw) ? U[(int64_t)(s + L * m + o) * k + s + L * m + o2] : 0.f;
   }
-  for (int i = threadIdx.x; i < SW_MAX_B; i += blockDim.x) {
+  for (int i = tid; i < SW_MAX_B; i += nth) {
     rdg[i] = (i < bw) ? 1.0f / U[(int64_t)(s + i) * k + s + i] : 0.f;
     pcol[i] = (i < bw) ? perm[s + i] : 0;
   }
@@ -592,12 +594,15 @@ __global__ void loss_finish_kernel(const T* __restrict__ W0, int64_t ldw, int r,
   const int lane = threadIdx.x % kWarp;
   if (row >= r) return;
   double acc = 0.0;
+  const uint8_t* crow = codes + (int64_t)row * k;
+  const T* wrow = W0 + (int64_t)row * ldw;
+  const float* srow = scales + (int64_t)row * ngroups;
+  const int32_t* zrow = zeros + (int64_t)row * ngroups;
+#pragma unroll 4
   for (int c = lane; c < k; c += kWarp) {
     const int g = g_idx[c];
-    const float sc = scales[(int64_t)row * ngroups + g];
-    const float z = (float)zeros[(int64_t)row * ngroups + g];
-    const float q = sc * ((float)codes[(int64_t)row * k + c] - z);
-    const float w0 = dead[c] ? 0.f : to_f32(W0[(int64_t)row * ldw + c]);
+    const float q = srow[g] * ((float)crow[c] - (float)zrow[g]);
+    const float w0 = dead[c] ? 0.f : to_f32(wrow[c]);
     const double dd = (double)w0 - (double)q;
     acc += dd * dd;
   }
@@ -671,7 +676,8 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     GPTQ_CHECK_LAUNCH();
   }
   if (tc) {
-    gptq_status st = tc_split_transpose(U, k, k, k, -1.0f, sc.U_hi, sc.U_lo, k, s);
+    // the trailing updates read -U^T only at (c, i) with c > i
+    gptq_status st = tc_split_transpose(U, k, k, k, -1.0f, 1, sc.U_hi, sc.U_lo, k, s);
     if (st != GPTQ_OK) return st;
   }
   // block kernel: the lane kernel when the groups inside a block have a
@@ -692,8 +698,9 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     const int64_t warps = cdiv(r, 32 / lanes);
     q_warps = (int)std::min<int64_t>(SQ_MAX_WARPS, std::max<int64_t>(1, cdiv(warps, nsm)));
     q_grid = (unsigned)cdiv(warps, q_warps);
-    if (lanes == 8) sweep_records_kernel<8><<<(unsigned)nblocks, 256, 0, s>>>(U, perm, k, B, sc.rec);
-    else sweep_records_kernel<4><<<(unsigned)nblocks, 256, 0, s>>>(U, perm, k, B, sc.rec);
+    const dim3 rgrid((unsigned)nblocks, 16);
+    if (lanes == 8) sweep_records_kernel<8><<<rgrid, 256, 0, s>>>(U, perm, k, B, sc.rec);
+    else sweep_records_kernel<4><<<rgrid, 256, 0, s>>>(U, perm, k, B, sc.rec);
     GPTQ_CHECK_LAUNCH();
   }
   int SB = 16;

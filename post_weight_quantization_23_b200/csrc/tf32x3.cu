@@ -330,11 +330,15 @@ __device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
 
 // dst[c][r] = split(sign * src[r][c]) for r < rows, c < cols (32 x 32 tiles
 // through shared memory, so both the reads and the writes are coalesced).
+// upper_only: src is upper triangular and only dst[c][r] with c >= r is
+// wanted; tiles with every c < r are left unwritten.
 __global__ void split_transpose_kernel(const float* __restrict__ src, int64_t lds, int rows,
-                                       int cols, float sign, float* __restrict__ hi,
-                                       float* __restrict__ lo, int64_t ldo) {
+                                       int cols, float sign, int upper_only,
+                                       float* __restrict__ hi, float* __restrict__ lo,
+                                       int64_t ldo) {
   __shared__ float tile[32][33];
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  if (upper_only && c0 + 31 < r0) return;
   const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
   for (int y = ty; y < 32; y += 8) {
     const int r = r0 + y, c = c0 + tx;
@@ -357,10 +361,11 @@ __global__ void split_transpose_kernel(const float* __restrict__ src, int64_t ld
 bool tc_update_supported(int64_t k) { return k % 4 == 0 && encode_fn() != nullptr; }
 
 gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float sign,
-                               float* hi, float* lo, int64_t ldo, cudaStream_t s) {
+                               int upper_only, float* hi, float* lo, int64_t ldo, cudaStream_t s) {
   if (rows <= 0 || cols <= 0) return GPTQ_OK;
   dim3 grid((unsigned)cdiv(cols, 32), (unsigned)cdiv(rows, 32));
-  split_transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(src, lds, rows, cols, sign, hi, lo, ldo);
+  split_transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(src, lds, rows, cols, sign, upper_only, hi,
+                                                      lo, ldo);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
 }
