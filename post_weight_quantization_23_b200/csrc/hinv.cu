@@ -224,6 +224,8 @@ __global__ void __launch_bounds__(256)
 chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
                      float* __restrict__ ujj, float* __restrict__ st_hi,
                      float* __restrict__ st_lo, int32_t* __restrict__ d_info) {
+  pdl_wait();
+  pdl_trigger();
   if (*d_info != 0) return;
   __shared__ float S[HV_B][K1_LD];                 // B, then M (lower part)
   __shared__ float T[HV_B][K1_LD];                 // N = M^-1 (lower part)
@@ -394,6 +396,8 @@ panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* 
                       int n_pan, float* __restrict__ st_hi, float* __restrict__ st_lo,
                       float* __restrict__ rt_hi, float* __restrict__ rt_lo,
                       const int32_t* __restrict__ d_info) {
+  pdl_wait();
+  pdl_trigger();
   if (*d_info != 0) return;
   __shared__ __align__(16) float Us[HV_B][HV_B + 4];  // row stride 68: conflict-free row reads
   __shared__ __align__(16) float Hs[HV_B][K2_W + 4];  // row stride 20: aligned float4 rows
@@ -627,15 +631,16 @@ gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cf
     // Schur part leaves values above the diagonal of [0, j0)^2, so K2 also
     // clears the strip where block J's Y columns start accumulating
     const bool tcs = tc && j0 > 0;
-    chol_inv_diag_kernel<<<1, 256, 0, s>>>(U, k, j0, b, sc.ujj, tcs ? sc.s_hi : nullptr,
-                                           tcs ? sc.s_lo : nullptr, d_info);
+    launch_pdl(chol_inv_diag_kernel, dim3(1), dim3(256), 0, s, U, k, j0, b, sc.ujj,
+               tcs ? sc.s_hi : nullptr, tcs ? sc.s_lo : nullptr, d_info);
     GPTQ_CHECK_LAUNCH();
     const int n_pan = (int)cdiv(j0, K2_W);
     const int n_row = (int)cdiv(k - j1, K2_W);
     if (n_pan + n_row > 0) {
-      panel_rowblock_kernel<<<(unsigned)(n_pan + n_row), 256, 0, s>>>(
-          U, k, j0, b, sc.ujj, n_pan, tcs ? sc.s_hi : nullptr, tcs ? sc.s_lo : nullptr,
-          tcs ? sc.r_hi : nullptr, tcs ? sc.r_lo : nullptr, d_info);
+      launch_pdl(panel_rowblock_kernel, dim3((unsigned)(n_pan + n_row)), dim3(256), 0, s, U, k, j0,
+                 b, (const float*)sc.ujj, n_pan, tcs ? sc.s_hi : nullptr,
+                 tcs ? sc.s_lo : nullptr, tcs ? sc.r_hi : nullptr, tcs ? sc.r_lo : nullptr,
+                 (const int32_t*)d_info);
       GPTQ_CHECK_LAUNCH();
     }
     if (j0 > 0) {

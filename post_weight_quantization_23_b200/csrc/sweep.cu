@@ -537,6 +537,10 @@ __global__ void __launch_bounds__(SQ_MAX_WARPS * 32, 1) sweep_block_lane_kernel(
           : "memory");
     }
   }
+  // the record comes from a kernel that finished before the previous one
+  // started; the weights (and a group grid) come from the previous kernels
+  pdl_wait();
+  pdl_trigger();
   SqState<L> st;
 #pragma unroll
   for (int j = 0; j < Ly::S; ++j) {
@@ -640,15 +644,21 @@ static void launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* 
                                                            codes, loss, d_status);
 }
 
+// pdl: launch early behind the previous kernel (every block but the first,
+// whose record may still be in flight from the kernel right before it)
 template <int L, int MODE>
-static void launch_lane(unsigned grid, int threads, cudaStream_t s, const SqArgs& a) {
+static void launch_lane(unsigned grid, int threads, cudaStream_t s, const SqArgs& a, bool pdl) {
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(sweep_block_lane_kernel<L, MODE>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SqLayout<L>::SMEM);
     attr = true;
   }
-  sweep_block_lane_kernel<L, MODE><<<grid, threads, SqLayout<L>::SMEM, s>>>(a);
+  if (pdl)
+    launch_pdl(sweep_block_lane_kernel<L, MODE>, dim3(grid), dim3(threads), SqLayout<L>::SMEM, s,
+               a);
+  else
+    sweep_block_lane_kernel<L, MODE><<<grid, threads, SqLayout<L>::SMEM, s>>>(a);
 }
 
 template <typename T>
@@ -731,12 +741,13 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
       a.codes = codes;
       a.loss = lossp;
       a.d_status = d_status;
+      const bool pdl = b > 0 && !(G > B && s0 % G == 0);  // right behind a trailing update
       if (lanes == 8) {
-        if (lane_mode == 0) launch_lane<8, 0>(q_grid, 32 * q_warps, s, a);
-        else launch_lane<8, 1>(q_grid, 32 * q_warps, s, a);
+        if (lane_mode == 0) launch_lane<8, 0>(q_grid, 32 * q_warps, s, a, pdl);
+        else launch_lane<8, 1>(q_grid, 32 * q_warps, s, a, pdl);
       } else {
-        if (lane_mode == 0) launch_lane<4, 0>(q_grid, 32 * q_warps, s, a);
-        else launch_lane<4, 1>(q_grid, 32 * q_warps, s, a);
+        if (lane_mode == 0) launch_lane<4, 0>(q_grid, 32 * q_warps, s, a, pdl);
+        else launch_lane<4, 1>(q_grid, 32 * q_warps, s, a, pdl);
       }
     } else {
 #define GPTQ_SWEEP_BLOCK(SBV)                                                                  \

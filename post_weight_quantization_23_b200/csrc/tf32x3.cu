@@ -125,6 +125,9 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
+  // set-up above overlaps the previous kernel; its outputs are read below
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const int nkc = (a.K + TX_KC - 1) / TX_KC;
   const uint32_t idesc = tc::instr_desc(2, TX_M, TX_N, 0, 0);  // both operands K-major
@@ -314,7 +317,8 @@ gptq_status launch(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorM
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(a.ntiles, nsm);
   if (grid <= 0) return GPTQ_OK;
-  tf32x3_update_kernel<<<grid, TX_THREADS, TX_SMEM, s>>>(ah, al, bh, bl, dm, a);
+  launch_pdl(tf32x3_update_kernel, dim3(grid), dim3(TX_THREADS), TX_SMEM, s, ah, al, bh, bl, dm,
+             a);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
 }
