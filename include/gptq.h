@@ -74,7 +74,11 @@ typedef enum { GPTQ_F32 = 0, GPTQ_F16 = 1, GPTQ_BF16 = 2 } gptq_dtype;
  *   block_size  lazy-batch width B ([GPTQ-tool] Step 7), 16..128, multiple of 16.
  *   percdamp    damping fraction of mean(diag H) ([GPTQ-tool] Step 4), >= 0.
  *   act_order   nonzero: process columns by descending diag(H).
- *   sym         reserved, must be 0 (asymmetric grid only). */
+ *   sym         0: asymmetric grid, zero point fitted per group (rint(-min/scale));
+ *               1: symmetric grid about 0, scale = 2 max(|min|, |max|) / maxq and
+ *               zero point (maxq + 1) / 2 for every group ("GPTQ",
+ *               ozercemkelahmet.com/tools/gptq, Optional refinements).
+ *               Other values: GPTQ_ERR_INVALID_ARG. */
 typedef struct {
   int bits;
   int group_size;

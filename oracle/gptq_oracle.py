@@ -38,6 +38,11 @@ R10 Groups and lazy blocks are aligned: group_size divides block_size or
 R11 Layer loss = tr((W0 - Qhat) H0 (W0 - Qhat)^T) with the undamped H0, i.e.
     (2/n)·||(W0 - Qhat) X^T||_F^2 ([GPTQ-tool] Step 2 objective and *Reading a
     quantization log*).
+R14 Symmetric grid ([GPTQ-tool] *Optional refinements*: "simpler", no fitted
+    zero point; nothing else is said): the range is made symmetric about 0,
+    [-a, a] with a = max(|min|, |max|) (0 included), scale = max(2a, 1e-8) /
+    maxq, and every group's zero point is the grid's middle code
+    (maxq + 1) / 2, so codes cover [-(maxq+1)/2, (maxq-1)/2] steps.
 """
 
 from __future__ import annotations
@@ -166,8 +171,8 @@ def hinv_upper_factor(H):
 # Quantization grid
 # ---------------------------------------------------------------------------
 
-def grid_params(wg, maxq, include_zero=True, decide_dtype=F32):
-    """Asymmetric min/max grid for each row of ``wg`` (r, g).
+def grid_params(wg, maxq, include_zero=True, decide_dtype=F32, sym=False):
+    """Min/max grid for each row of ``wg`` (r, g).
 
     [GPTQ-tool] sketch: scale = clamp(max - min, min=1e-8) / maxq and
     zero = round(-min / scale); *Optional refinements* (asymmetric grids use a
@@ -175,14 +180,24 @@ def grid_params(wg, maxq, include_zero=True, decide_dtype=F32):
     zero).  READING R6: the range includes 0 unless ``include_zero`` is False.
     Computed in ``decide_dtype`` (fp32, as the sketch) because the zero point
     is an integer decision.  Returns (scale, zero) as arrays of decide_dtype.
+
+    ``sym`` ([GPTQ-tool] *Optional refinements*: symmetric grids, no fitted
+    zero point; READING R14): the range is made symmetric, [-a, a] with
+    a = max(|lo|, |hi|), so scale = max(2a, 1e-8) / maxq, and the zero point is
+    the grid's middle code (maxq + 1) / 2 for every group.
     """
     dt = decide_dtype
     w = np.asarray(wg, dtype=F64).astype(dt)
     lo = w.min(axis=1)
     hi = w.max(axis=1)
-    if include_zero:
+    if include_zero or sym:
         lo = np.minimum(lo, dt(0))
         hi = np.maximum(hi, dt(0))
+    if sym:
+        a = np.maximum(-lo, hi)
+        scale = np.maximum(a + a, dt(1e-8)) / dt(maxq)
+        zero = np.full(scale.shape, (maxq + 1) // 2, dtype=dt)
+        return scale.astype(dt), zero
     scale = np.maximum(hi - lo, dt(1e-8)) / dt(maxq)
     zero = np.rint(-lo / scale)
     return scale.astype(dt), zero.astype(dt)
@@ -227,7 +242,7 @@ def _check_groups(k, group_size, block_size=None):
 # ---------------------------------------------------------------------------
 
 def sweep_unblocked(W, U, bits, group_size, include_zero=True, decide_dtype=F32,
-                    fixed_grid=None):
+                    fixed_grid=None, sym=False):
     """Column-by-column GPTQ sweep (no lazy batching).
 
     [GPTQ-tool] *How it works*, Step 5 and the sketch's loop: for each column
@@ -259,7 +274,7 @@ def sweep_unblocked(W, U, bits, group_size, include_zero=True, decide_dtype=F32,
     s = z = None
     for i in range(k):
         if i % G == 0:
-            s, z = _group_grid(W[:, i:i + G], maxq, include_zero, decide_dtype, fixed_grid, r)
+            s, z = _group_grid(W[:, i:i + G], maxq, include_zero, decide_dtype, fixed_grid, r, sym)
             scales[:, i // G] = s
             zeros[:, i // G] = z
         w = W[:, i].copy()
@@ -274,16 +289,16 @@ def sweep_unblocked(W, U, bits, group_size, include_zero=True, decide_dtype=F32,
     return dict(codes=codes, scales=scales, zeros=zeros, qhat=qhat, err=errs, w_at=w_at)
 
 
-def _group_grid(wg, maxq, include_zero, dt, fixed_grid, r):
+def _group_grid(wg, maxq, include_zero, dt, fixed_grid, r, sym=False):
     if fixed_grid is None:
-        return grid_params(wg, maxq, include_zero, dt)
+        return grid_params(wg, maxq, include_zero, dt, sym)
     s, z = fixed_grid
     return np.full(r, s, dtype=dt), np.full(r, z, dtype=dt)
 
 
 def sweep_blocked(W, U, bits, group_size, block_size, include_zero=True,
                   decide_dtype=F32, force_codes=None, force_zeros=None, tau=None,
-                  fixed_grid=None):
+                  fixed_grid=None, sym=False):
     """Lazy-batch GPTQ sweep.
 
     [GPTQ-tool] Step 7 (blocks of ``block_size`` columns: updates inside the
@@ -320,8 +335,9 @@ def sweep_blocked(W, U, bits, group_size, block_size, include_zero=True,
         Err = np.zeros((r, e0 - s0))
         for i in range(s0, e0):
             if i % G == 0:
-                s, z = _group_grid(W[:, i:i + G], maxq, include_zero, decide_dtype, fixed_grid, r)
-                if force_zeros is not None:
+                s, z = _group_grid(W[:, i:i + G], maxq, include_zero, decide_dtype, fixed_grid, r,
+                                   sym)
+                if force_zeros is not None and not sym:  # a symmetric grid's zero is fixed
                     z, nf = _force_ties(-np.minimum(W[:, i:i + G].astype(decide_dtype).min(axis=1), 0)
                                         if include_zero else
                                         -W[:, i:i + G].astype(decide_dtype).min(axis=1),
@@ -370,7 +386,7 @@ def _force_ties(neg_lo, s, z, forced, tau, dt):
 
 
 def sweep_replay(W, U, bits, group_size, block_size, force_codes, force_zeros,
-                 tau=1e-3, include_zero=True, decide_dtype=F32):
+                 tau=1e-3, include_zero=True, decide_dtype=F32, sym=False):
     """Tie-aware replay: the lazy-blocked sweep in fp64, except that wherever
     a candidate result (``force_codes``, ``force_zeros``, sweep order) differs
     from the oracle's decision by exactly one step AND the oracle's value
@@ -380,11 +396,11 @@ def sweep_replay(W, U, bits, group_size, block_size, force_codes, force_zeros,
     decision must then agree exactly.  Returns the same dict as
     ``sweep_blocked`` with ``n_forced``."""
     return sweep_blocked(W, U, bits, group_size, block_size, include_zero,
-                         decide_dtype, force_codes, force_zeros, tau)
+                         decide_dtype, force_codes, force_zeros, tau, sym=sym)
 
 
 def sweep_obs(W, Hd, bits, group_size, include_zero=True, decide_dtype=F32,
-              fixed_grid=None):
+              fixed_grid=None, sym=False):
     """Column sweep with an explicit inverse Hessian and the Optimal Brain
     Surgeon downdate.
 
@@ -412,7 +428,7 @@ def sweep_obs(W, Hd, bits, group_size, include_zero=True, decide_dtype=F32,
     s = z = None
     for i in range(k):
         if i % G == 0:
-            s, z = _group_grid(W[:, i:i + G], maxq, include_zero, decide_dtype, fixed_grid, r)
+            s, z = _group_grid(W[:, i:i + G], maxq, include_zero, decide_dtype, fixed_grid, r, sym)
             scales[:, i // G] = s
             zeros[:, i // G] = z
         w = W[:, i].copy()
@@ -426,7 +442,7 @@ def sweep_obs(W, Hd, bits, group_size, include_zero=True, decide_dtype=F32,
     return dict(codes=codes, scales=scales, zeros=zeros, qhat=qhat)
 
 
-def rtn(W, bits, group_size, include_zero=True, decide_dtype=F32):
+def rtn(W, bits, group_size, include_zero=True, decide_dtype=F32, sym=False):
     """Round-to-nearest baseline ([GPTQ-breakdown] *The Problem*; [GPTQ-tool]
     *A worked example*, "plain rounding"; *Glossary*): every weight is rounded
     on its group's grid independently, with no error compensation.  Group
@@ -442,7 +458,7 @@ def rtn(W, bits, group_size, include_zero=True, decide_dtype=F32):
     zeros = np.zeros((r, ng), dtype=decide_dtype)
     for g in range(ng):
         a, b = g * G, min((g + 1) * G, k)
-        s, z = grid_params(W[:, a:b], maxq, include_zero, decide_dtype)
+        s, z = grid_params(W[:, a:b], maxq, include_zero, decide_dtype, sym)
         c = quantize_codes(W[:, a:b], s[:, None], z[:, None], maxq, decide_dtype)
         codes[:, a:b] = c
         qhat[:, a:b] = _dequant_f64(c, s[:, None], z[:, None])
@@ -466,7 +482,7 @@ def layer_loss(W0, qhat, H0):
 # ---------------------------------------------------------------------------
 
 def gptq(W, H, bits=4, group_size=128, block_size=128, percdamp=0.01,
-         act_order=False, include_zero=True, decide_dtype=F32, blocked=True,
+         act_order=False, include_zero=True, decide_dtype=F32, blocked=True, sym=False,
          force_codes=None, force_zeros=None, tau=1e-3, force_perm=None, tau_perm=1e-5):
     """GPTQ for one linear layer, given W (r, k) and the undamped Hessian H.
 
@@ -497,11 +513,12 @@ def gptq(W, H, bits=4, group_size=128, block_size=128, percdamp=0.01,
     if force_codes is not None:
         fc = np.asarray(force_codes)[:, perm]
         res = sweep_replay(Wp, U, bits, group_size, block_size, fc, force_zeros,
-                           tau, include_zero, decide_dtype)
+                           tau, include_zero, decide_dtype, sym)
     elif blocked:
-        res = sweep_blocked(Wp, U, bits, group_size, block_size, include_zero, decide_dtype)
+        res = sweep_blocked(Wp, U, bits, group_size, block_size, include_zero, decide_dtype,
+                            sym=sym)
     else:
-        res = sweep_unblocked(Wp, U, bits, group_size, include_zero, decide_dtype)
+        res = sweep_unblocked(Wp, U, bits, group_size, include_zero, decide_dtype, sym=sym)
     G = k if group_size == -1 else group_size
     codes = np.zeros((r, k))
     qhat = np.zeros((r, k))

@@ -65,9 +65,10 @@ class GptqConfig(ctypes.Structure):
     ]
 
 
-def make_config(bits=4, group_size=128, block_size=128, percdamp=0.01, act_order=False):
+def make_config(bits=4, group_size=128, block_size=128, percdamp=0.01, act_order=False,
+                sym=False):
     return GptqConfig(int(bits), int(group_size), int(block_size), float(percdamp),
-                      int(bool(act_order)), 0)
+                      int(bool(act_order)), int(bool(sym)))
 
 
 _lib = None

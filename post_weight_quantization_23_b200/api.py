@@ -27,10 +27,11 @@ class QuantConfig:
     block_size: int = 128
     percdamp: float = 0.01
     act_order: bool = False
+    sym: bool = False  # symmetric grid (zero point at the middle code)
 
     def c(self):
         return make_config(self.bits, self.group_size, self.block_size, self.percdamp,
-                           self.act_order)
+                           self.act_order, self.sym)
 
     def ngroups(self, k: int) -> int:
         G = k if self.group_size == -1 else self.group_size

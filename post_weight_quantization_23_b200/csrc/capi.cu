@@ -41,7 +41,7 @@ bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 8; }
 gptq_status check_config(const gptq_config* cfg, int64_t k) {
   if (cfg == nullptr) return GPTQ_ERR_INVALID_ARG;
   if (!valid_bits(cfg->bits)) return GPTQ_ERR_UNSUPPORTED;
-  if (cfg->sym != 0) return GPTQ_ERR_UNSUPPORTED;
+  if (cfg->sym != 0 && cfg->sym != 1) return GPTQ_ERR_INVALID_ARG;
   if (!(cfg->percdamp >= 0.0f) || !isfinite(cfg->percdamp)) return GPTQ_ERR_INVALID_ARG;
   const int B = cfg->block_size;
   if (B < 16 || B > 128 || B % 16 != 0) return GPTQ_ERR_UNSUPPORTED;

@@ -62,11 +62,20 @@ __device__ __forceinline__ float quant_code(float w, float scale, float zero, fl
   return fminf(fmaxf(c, 0.0f), maxq);
 }
 
-// Grid parameters of one group from its min and max:
-// lo = min(0, min), hi = max(0, max), scale = max(hi - lo, 1e-8) / maxq, zero = rint(-lo / scale).
+// Grid parameters of one group from its min and max, lo = min(0, min),
+// hi = max(0, max):
+//   asymmetric: scale = max(hi - lo, 1e-8) / maxq, zero = rint(-lo / scale);
+//   symmetric:  a = max(-lo, hi), scale = max(2a, 1e-8) / maxq,
+//               zero = (maxq + 1) / 2 (the grid's middle code).
 __device__ __forceinline__ void grid_from_range(float mn, float mx, float maxq, float& scale,
-                                                float& zero) {
+                                                float& zero, bool sym = false) {
   float lo = fminf(mn, 0.0f), hi = fmaxf(mx, 0.0f);
+  if (sym) {
+    const float a = fmaxf(-lo, hi);
+    scale = __fdiv_rn(fmaxf(__fadd_rn(a, a), 1e-8f), maxq);
+    zero = (maxq + 1.0f) * 0.5f;
+    return;
+  }
   scale = __fdiv_rn(fmaxf(__fsub_rn(hi, lo), 1e-8f), maxq);
   zero = rintf(__fdiv_rn(-lo, scale));
 }

@@ -150,8 +150,8 @@ __global__ void sweep_lambda_kernel(const float* __restrict__ H0, int k, float p
 
 // Per-row grid of a group [s, s+gw) wider than the lazy block: one warp per row.
 __global__ void group_grid_kernel(const float* __restrict__ Wt, int r, int k, int s, int gw,
-                                  int gidx, int ngroups, float maxq, float* __restrict__ scales,
-                                  int32_t* __restrict__ zeros) {
+                                  int gidx, int ngroups, float maxq, int sym,
+                                  float* __restrict__ scales, int32_t* __restrict__ zeros) {
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) / kWarp;
   int lane = threadIdx.x % kWarp;
   if (warp >= r) return;
@@ -168,7 +168,7 @@ __global__ void group_grid_kernel(const float* __restrict__ Wt, int r, int k, in
   }
   if (lane == 0) {
     float sc, z;
-    grid_from_range(mn, mx, maxq, sc, z);
+    grid_from_range(mn, mx, maxq, sc, z, sym != 0);
     scales[(int64_t)warp * ngroups + gidx] = sc;
     zeros[(int64_t)warp * ngroups + gidx] = (int32_t)z;
   }
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(SW_THREADS)
 sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
                    float* __restrict__ Err_lo, const float* __restrict__ U,
                    const int32_t* __restrict__ perm, int r, int k, int s, int bw, int B, int G,
-                   int ngroups, float maxq, float* __restrict__ scales,
+                   int ngroups, float maxq, int sym, float* __restrict__ scales,
                    int32_t* __restrict__ zeros, uint8_t* __restrict__ codes,
                    double* __restrict__ loss, int32_t* __restrict__ d_status) {
   extern __shared__ float sm_sweep[];
@@ -241,7 +241,7 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      grid_from_range(mn, mx, maxq, scale, zero);
+      grid_from_range(mn, mx, maxq, scale, zero, sym != 0);
       if (valid && q == 0) {
         scales[(int64_t)row * ngroups + (s + c0) / G] = scale;
         zeros[(int64_t)row * ngroups + (s + c0) / G] = (int32_t)zero;
@@ -371,6 +371,7 @@ struct SqArgs {
   const uint8_t* rec;  // this block's record
   int r, k, s, bw, B, G, ngroups;
   float maxq;
+  int sym;  // symmetric grid
   float* scales;
   int32_t* zeros;
   uint8_t* codes;
@@ -411,7 +412,7 @@ __device__ __forceinline__ void sq_sub_block(SqState<L>& st, int m, const SqArgs
       pn = fminf(pn, __shfl_xor_sync(0xffffffffu, pn, o, L));
       px = fmaxf(px, __shfl_xor_sync(0xffffffffu, px, o, L));
     }
-    grid_from_range(fminf(mn, pn), fmaxf(mx, px), a.maxq, st.scale, st.zero);
+    grid_from_range(fminf(mn, pn), fmaxf(mx, px), a.maxq, st.scale, st.zero, a.sym != 0);
     st.inv_s = 1.0f / st.scale;
     st.lo_d = -st.zero;
     st.hi_d = a.maxq - st.zero;
@@ -631,7 +632,7 @@ __global__ void loss_total_kernel(double* __restrict__ loss, int r) {
 template <int SB>
 static void launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* Err,
                          float* Err_lo, const float* U, const int32_t* perm, int r, int k, int s0,
-                         int bw, int B, int G, int ngroups, float maxq, float* scales,
+                         int bw, int B, int G, int ngroups, float maxq, int sym, float* scales,
                          int32_t* zeros, uint8_t* codes, double* loss, int32_t* d_status) {
   static bool attr = false;
   if (!attr) {
@@ -640,8 +641,8 @@ static void launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* 
     attr = true;
   }
   sweep_block_kernel<SB><<<grid, SW_THREADS, SW_SMEM, s>>>(Wt, Err, Err_lo, U, perm, r, k, s0, bw,
-                                                           B, G, ngroups, maxq, scales, zeros,
-                                                           codes, loss, d_status);
+                                                           B, G, ngroups, maxq, sym, scales,
+                                                           zeros, codes, loss, d_status);
 }
 
 // pdl: launch early behind the previous kernel (every block but the first,
@@ -725,7 +726,7 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     if (G > B && s0 % G == 0) {
       int gw = min(G, k - s0);
       group_grid_kernel<<<(unsigned)cdiv((int64_t)r * kWarp, 256), 256, 0, s>>>(
-          sc.Wt, r, k, s0, gw, s0 / G, ngroups, maxq, scales, zeros);
+          sc.Wt, r, k, s0, gw, s0 / G, ngroups, maxq, cfg->sym, scales, zeros);
       GPTQ_CHECK_LAUNCH();
     }
     if (lane_mode >= 0) {
@@ -736,6 +737,7 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
       a.rec = sc.rec + (size_t)b * SQ_REC_MAX;
       a.r = r, a.k = k, a.s = s0, a.bw = bw, a.B = B, a.G = G, a.ngroups = ngroups;
       a.maxq = maxq;
+      a.sym = cfg->sym;
       a.scales = scales;
       a.zeros = zeros;
       a.codes = codes;
@@ -752,7 +754,7 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     } else {
 #define GPTQ_SWEEP_BLOCK(SBV)                                                                  \
   launch_block<SBV>(grid, s, sc.Wt, sc.Err, err_lo, U, perm, r, k, s0, bw, B, G, ngroups, maxq, \
-                    scales, zeros, codes, lossp, d_status)
+                    cfg->sym, scales, zeros, codes, lossp, d_status)
       switch (SB) {
         case 16: GPTQ_SWEEP_BLOCK(16); break;
         case 8: GPTQ_SWEEP_BLOCK(8); break;

@@ -86,6 +86,9 @@ def test_host_argument_checks(lib):
     assert q(cfgp, ws=None) == _lib.GPTQ_ERR_WORKSPACE
     assert q(cfgp, nbytes=16) == _lib.GPTQ_ERR_WORKSPACE
     assert q(cfgp, ws=ctypes.c_void_p(257)) == _lib.GPTQ_ERR_WORKSPACE
+    bad_sym = _lib.make_config(4, 128, 128, 0.01, False)
+    bad_sym.sym = 2
+    assert q(ctypes.byref(bad_sym)) == _lib.GPTQ_ERR_INVALID_ARG
 
 
 def test_binding_refuses_cpu_tensors():

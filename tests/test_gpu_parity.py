@@ -23,9 +23,10 @@ def _np(t):
     return t.float().numpy() if t.dtype == torch.bfloat16 else t.numpy()
 
 
-def _cfg(spec):
+def _cfg(spec, sym=False):
     from post_weight_quantization_23_b200 import QuantConfig
-    return QuantConfig(spec.bits, spec.group_size, spec.block_size, spec.percdamp, spec.act_order)
+    return QuantConfig(spec.bits, spec.group_size, spec.block_size, spec.percdamp, spec.act_order,
+                       sym)
 
 
 CASES = {
@@ -51,6 +52,10 @@ CASES = {
     # group = block = 48, rows not a multiple of 4, last block 8 columns wide
     "gB48_ragged": synth.CONFIGS["tiny"].scaled(r=70, k=200, n=3000, group_size=48,
                                                 block_size=48),
+    # groups of 4 columns: the 4-lanes-per-row kernel
+    "g4_b32": synth.CONFIGS["q_proj"].scaled(r=64, k=256, n=4096, group_size=4, block_size=32),
+    # groups of 6 columns: the 4-threads-per-row kernel
+    "g6_b48": synth.CONFIGS["tiny"].scaled(r=40, k=192, n=3000, group_size=6, block_size=48),
     # k not a multiple of 4: CUDA-core trailing and rank updates
     "k150_cuda_core": synth.CONFIGS["tiny"].scaled(r=40, k=150, n=2000, group_size=-1,
                                                    block_size=32),
@@ -66,6 +71,40 @@ def test_layer_parity(name):
     a = compare(gpu, _np(W), _np(X), cfg)
     print(name, a)
     a.assert_ok()
+
+
+SYM_CASES = {
+    # symmetric grid (READING R14): groups inside the block, act-order, per row, 3 bits
+    "sym_q_proj_g64": synth.CONFIGS["q_proj"].scaled(r=128, k=512, n=8192, group_size=64),
+    "sym_down_act": synth.CONFIGS["down_proj"].scaled(r=64, k=400, n=4096, group_size=16),
+    "sym_opt_per_row_3bit": synth.CONFIGS["opt175_width"].scaled(r=64, k=384, n=4096),
+    "sym_g6_b48": synth.CONFIGS["tiny"].scaled(r=40, k=96, n=2048, group_size=6, block_size=48),
+}
+
+
+@pytest.mark.parametrize("name", list(SYM_CASES))
+def test_layer_parity_symmetric(name):
+    spec = SYM_CASES[name]
+    W, X, Wd, Xd = layer_inputs(spec, seed=4)
+    cfg = _cfg(spec, sym=True)
+    gpu = gpu_quantize(Wd, Xd, cfg)
+    z = gpu["zeros"].numpy()
+    assert np.all(z == (2 ** cfg.bits) // 2)
+    a = compare(gpu, _np(W), _np(X), cfg)
+    print(name, a)
+    # The symmetric grid's scale 2 max|w| / maxq puts every group's largest-
+    # magnitude weight exactly on a rounding tie (w / s = -(maxq + 1) / 2 + 1/2),
+    # so the two sides' fp32 values pick either code there, and each such choice
+    # re-enters its row's compensation and later group grids.  What must hold:
+    # the tie-aware replay matches exactly, including the layer loss with the
+    # GPU's tie decisions, and the plain match rate stays high.
+    from _parity import TOL_H_REL_FRO, TOL_LOSS_REL, TOL_SCALE_REL
+    assert a.h_rel_fro <= TOL_H_REL_FRO, a
+    assert a.perm_equal and a.gidx_equal, a
+    assert a.replay_mismatch == 0 and a.zero_mismatch_replay == 0, a
+    assert a.scale_rel_replay <= TOL_SCALE_REL, a
+    assert a.loss_rel_replay <= TOL_LOSS_REL, a
+    assert a.code_match >= 0.99, a
 
 
 @pytest.mark.parametrize("name", ["tiny", "q_proj_small", "opt175_small", "down_proj_small"])

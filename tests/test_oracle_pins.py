@@ -197,6 +197,53 @@ def test_grid_properties():
     assert s[0] == np.float32(1e-8) / np.float32(15) and z[0] == 0
 
 
+def test_symmetric_grid_closed_form_and_properties():
+    # READING R14 (symmetric grid: range [-a, a], zero point (maxq + 1) / 2).
+    # Exact binary values, 2 bits: a = 0.75, scale = 1.5 / 3 = 0.5, zero = 2;
+    # w / s = -1.5, 0.5, 1.0 round half to even to -2, 0, 1 -> codes 0, 2, 3.
+    w = np.array([[-0.75, 0.25, 0.5]])
+    s, z = O.grid_params(w, 3, sym=True)
+    assert s[0] == np.float32(0.5) and z[0] == 2
+    c = O.quantize_codes(w, s[:, None], z[:, None], 3)
+    assert c.tolist() == [[0.0, 2.0, 3.0]]
+    assert (s[0] * (c - z[0])).tolist() == [[-1.0, 0.0, 0.5]]
+    rng = np.random.default_rng(7)
+    x = rng.normal(0, 0.02, (40, 32)) + rng.normal(0, 0.01, (40, 1))  # skewed groups
+    for bits in (2, 3, 4, 8):
+        maxq = 2 ** bits - 1
+        s, z = O.grid_params(x, maxq, sym=True)
+        assert np.all(z == (maxq + 1) // 2)
+        a = np.maximum(np.abs(x.astype(np.float32)).max(axis=1), 0)
+        assert np.array_equal(s, ((a + a) / np.float32(maxq)).astype(np.float32))
+        c = O.quantize_codes(x, s[:, None], z[:, None], maxq)
+        assert np.all((c >= 0) & (c <= maxq))
+    # all-positive group: only the upper half of the codes is used
+    s, z = O.grid_params(np.abs(x), 15, sym=True)
+    c = O.quantize_codes(np.abs(x), s[:, None], z[:, None], 15)
+    assert np.all(c >= z[:, None])
+
+
+@pytest.mark.parametrize("gs,bs,act", [(32, 32, False), (-1, 32, False), (64, 32, True)])
+def test_symmetric_invariants(gs, bs, act):
+    # R14 with the pinned invariants: diagonal H == RTN, blocked == unblocked,
+    # Cholesky sweep == OBS downdate.
+    rng = np.random.default_rng(12)
+    W = rng.normal(0, 0.02, (16, 96))
+    H = np.diag(rng.lognormal(0, 1, 96))
+    res = O.gptq(W, H, bits=4, group_size=gs, block_size=bs, act_order=act, sym=True)
+    ref = O.rtn(W[:, res["perm"]], 4, gs, sym=True)
+    assert np.array_equal(res["codes"][:, res["perm"]], ref["codes"])
+    assert np.array_equal(res["scales"], ref["scales"])
+    W2, _, H2 = _rand_layer(8, 12, 96)
+    U = O.hinv_upper_factor(O.damp(H2, 0.01))
+    a = O.sweep_unblocked(W2, U, 3, gs, sym=True)
+    b = O.sweep_blocked(W2, U, 3, gs, bs, sym=True)
+    assert np.array_equal(a["codes"], b["codes"])
+    assert np.all(a["zeros"] == 4)
+    c = O.sweep_obs(W2, O.damp(H2, 0.01), 3, gs, sym=True)
+    assert np.array_equal(a["codes"], c["codes"])
+
+
 def test_half_to_even_rounding():
     c = O.quantize_codes(np.array([6.5, 7.5, -0.5, 2.4999]), 1.0, 0.0, None)
     assert list(c) == [6, 8, 0, 2]
