@@ -15,7 +15,7 @@
 // Accuracy: the tensor core accumulates at most 256 tokens (16 MMAs) in TMEM;
 // the epilogue then adds that partial into fp32 registers (TMEM is double
 // buffered, so the next 256 tokens accumulate meanwhile) and flushes the
-// register sum into H with fp32 atomics once per unit of up to 16384 tokens.
+// register sum into H with fp32 atomics once per unit of up to 65536 tokens.
 // A plain fp32 running sum over all n tokens would miss the 1e-5 relative
 // Frobenius target at n = 262144.
 //
@@ -45,7 +45,7 @@ constexpr int HT_A_BYTES = 2 * HT_BOX_BYTES;            // 16 KB
 constexpr int HT_STAGE_BYTES = HT_B_BYTES + HT_A_BYTES; // 48 KB
 constexpr int HT_THREADS = 320;                         // TMA warp, MMA warp, 8 epilogue warps
 constexpr int HT_TMEM_COLS = 512;                       // 2 accumulators x 256 columns
-constexpr int HT_MAX_CHUNK = 16384;
+constexpr int HT_MAX_CHUNK = 65536;
 constexpr size_t HT_SMEM = (size_t)HT_STAGES * HT_STAGE_BYTES + 1024 + 256;
 
 struct HtArgs {
@@ -325,7 +325,7 @@ gptq_status hessian_tc(const void* X, gptq_dtype dt, int64_t n, int64_t k, int64
   a.nJ = (int)cdiv(k, HT_N);
   a.ntiles = 0;
   for (int i = 0; i < a.nI; ++i) a.ntiles += max(0, a.nJ - i / 2);
-  // token chunk per unit: enough units for ~4 per SM, 256..16384 tokens
+  // token chunk per unit: enough units for ~4 per SM, 256..65536 tokens
   int64_t want = cdiv(n * a.ntiles, 4 * (int64_t)nsm);
   int64_t chunk = cdiv(want, 256) * 256;
   chunk = std::min<int64_t>(std::max<int64_t>(chunk, 256), HT_MAX_CHUNK);
