@@ -42,11 +42,12 @@ METRIC = "GPTQ layer quantize Mweights/s end-to-end"
 UNIT = "Mweights/s"
 
 
-# DRAM traffic of hessian_tc_kernel from one ncu capture (32768 tokens, k = 4096):
-# 649.7 MB read + 67.7 MB written; both grow with the token count (X re-reads and
-# the per-unit flushes of H), so a launch over n tokens moves about n times this.
+# DRAM traffic of hessian_tc_kernel from one ncu capture (32768 tokens, k = 4096,
+# units of 15104 tokens): 645.9 MB read + 65.9 MB written.  Scaled by tokens to a
+# full launch -- an estimate: a full q_proj launch runs 65536-token units, whose
+# reuse of X in L2 differs.
 HESS_TRAFFIC_K = 4096
-HESS_TRAFFIC_BYTES_PER_TOKEN = (649.7e6 + 67.7e6) / 32768
+HESS_TRAFFIC_BYTES_PER_TOKEN = (645.9e6 + 65.9e6) / 32768
 
 
 def _peaks():
@@ -359,9 +360,9 @@ def native_arm(args, spec, world, rank, local):
     roofline = {"bound": "tensor", "kernel": "gptq_hessian_accumulate (X^T X)",
                 "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_sustained"], "traffic": traffic,
-                "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of "
-                                   "hessian_tc_kernel, 32768 x 4096 capture, scaled by tokens "
-                                   "(profiles/hessian_tc_kernel_q_proj_32k_tokens.md)")
+                "traffic_source": ("estimate: ncu dram__bytes_read.sum + dram__bytes_write.sum "
+                                   "of hessian_tc_kernel on a 32768 x 4096 capture, scaled by "
+                                   "tokens (profiles/hessian_tc_kernel_q_proj_32k_tokens.md)")
                 if traffic is not None and args.traffic is None else None,
                 "peak_kind": f"bf16 dense sustained ({peaks['source']}); f16 has the same nominal rate",
                 "algorithmic": f"n*k*(k+1) = {flops:.4g} flop per launch"}
