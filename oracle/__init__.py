@@ -35,6 +35,7 @@ from .gptq_oracle import (  # noqa: F401
     damp,
     hinv_upper_factor,
     grid_params,
+    static_grids,
     quantize_codes,
     sweep_unblocked,
     sweep_blocked,

@@ -43,6 +43,15 @@ R14 Symmetric grid ([GPTQ-tool] *Optional refinements*: "simpler", no fitted
     [-a, a] with a = max(|min|, |max|) (0 included), scale = max(2a, 1e-8) /
     maxq, and every group's zero point is the grid's middle code
     (maxq + 1) / 2, so codes cover [-(maxq+1)/2, (maxq-1)/2] steps.
+R15 Static groups (the ``static_groups`` flag of the AutoGPTQ configuration
+    listed by [GPTQ-guide] *Configuration Deep Dive*; its meaning is not
+    given): every group's grid is fixed before the sweep, from the
+    dead-column-fixed ORIGINAL weights of the group's original columns
+    [g G, (g+1) G) (the grid RTN would use); the sweep never refits a grid.
+    Under act-order a column keeps its original group, so g_idx[c] = c // G,
+    and each column is quantized on that group's grid when its turn comes.
+    Because no grid depends on the sweep, groups need not align with the
+    lazy blocks (READING R10 is not needed).
 """
 
 from __future__ import annotations
@@ -237,12 +246,29 @@ def _check_groups(k, group_size, block_size=None):
     return max(G, 1)
 
 
+def static_grids(W, bits, group_size, include_zero=True, decide_dtype=F32, sym=False):
+    """READING R15: the grid of every group g, fitted once to the original
+    columns [g G, (g+1) G) of ``W`` (r, k), before any error compensation.
+    Returns (scales, zeros), each (r, ngroups) in decide_dtype."""
+    W = np.asarray(W, dtype=F64)
+    r, k = W.shape
+    maxq = 2 ** bits - 1
+    G = _check_groups(k, group_size)
+    ng = group_count(k, group_size)
+    scales = np.zeros((r, ng), dtype=decide_dtype)
+    zeros = np.zeros((r, ng), dtype=decide_dtype)
+    for g in range(ng):
+        scales[:, g], zeros[:, g] = grid_params(W[:, g * G:min((g + 1) * G, k)], maxq,
+                                                include_zero, decide_dtype, sym)
+    return scales, zeros
+
+
 # ---------------------------------------------------------------------------
 # Column sweeps
 # ---------------------------------------------------------------------------
 
 def sweep_unblocked(W, U, bits, group_size, include_zero=True, decide_dtype=F32,
-                    fixed_grid=None, sym=False):
+                    fixed_grid=None, sym=False, static=None):
     """Column-by-column GPTQ sweep (no lazy batching).
 
     [GPTQ-tool] *How it works*, Step 5 and the sketch's loop: for each column
@@ -257,7 +283,9 @@ def sweep_unblocked(W, U, bits, group_size, include_zero=True, decide_dtype=F32,
     err (r, k) scaled errors and w_at (r, k), each column's value at the
     moment it is quantized, all in sweep order.  ``fixed_grid`` = (scale,
     zero) replaces the min/max grid by a fixed one (the worked examples of the
-    pages use a fixed step).
+    pages use a fixed step).  ``static`` = (scales, zeros, gcol) gives every
+    column a grid fixed before the sweep (READING R15): column i uses group
+    gcol[i] of the (r, ngroups) tables, which are returned unchanged.
     """
     W = np.array(W, dtype=F64, copy=True)
     U = np.asarray(U, dtype=F64)
@@ -273,7 +301,9 @@ def sweep_unblocked(W, U, bits, group_size, include_zero=True, decide_dtype=F32,
     zeros = np.zeros((r, ng), dtype=decide_dtype)
     s = z = None
     for i in range(k):
-        if i % G == 0:
+        if static is not None:
+            s, z = _static_grid(static, i)
+        elif i % G == 0:
             s, z = _group_grid(W[:, i:i + G], maxq, include_zero, decide_dtype, fixed_grid, r, sym)
             scales[:, i // G] = s
             zeros[:, i // G] = z
@@ -286,7 +316,15 @@ def sweep_unblocked(W, U, bits, group_size, include_zero=True, decide_dtype=F32,
         qhat[:, i] = q
         errs[:, i] = err
         w_at[:, i] = w
+    if static is not None:
+        scales, zeros = static[0], static[1]
     return dict(codes=codes, scales=scales, zeros=zeros, qhat=qhat, err=errs, w_at=w_at)
+
+
+def _static_grid(static, i):
+    """Column i's fixed grid (READING R15)."""
+    sc, zc, gcol = static
+    return sc[:, gcol[i]], zc[:, gcol[i]]
 
 
 def _group_grid(wg, maxq, include_zero, dt, fixed_grid, r, sym=False):
@@ -298,7 +336,7 @@ def _group_grid(wg, maxq, include_zero, dt, fixed_grid, r, sym=False):
 
 def sweep_blocked(W, U, bits, group_size, block_size, include_zero=True,
                   decide_dtype=F32, force_codes=None, force_zeros=None, tau=None,
-                  fixed_grid=None, sym=False):
+                  fixed_grid=None, sym=False, static=None):
     """Lazy-batch GPTQ sweep.
 
     [GPTQ-tool] Step 7 (blocks of ``block_size`` columns: updates inside the
@@ -311,7 +349,8 @@ def sweep_blocked(W, U, bits, group_size, block_size, include_zero=True,
 
     ``force_codes`` / ``force_zeros`` (sweep order) turn this into the
     tie-aware replay of ``sweep_replay``; leave them None otherwise.
-    ``fixed_grid`` as in ``sweep_unblocked``.
+    ``fixed_grid`` and ``static`` as in ``sweep_unblocked``; with ``static``
+    the groups need not align with the blocks (READING R15).
     """
     W = np.array(W, dtype=F64, copy=True)
     U = np.asarray(U, dtype=F64)
@@ -320,7 +359,7 @@ def sweep_blocked(W, U, bits, group_size, block_size, include_zero=True,
     B = int(block_size)
     if B <= 0:
         raise ValueError("block_size must be positive")
-    G = _check_groups(k, group_size, B)
+    G = _check_groups(k, group_size, None if static is not None else B)
     ng = group_count(k, group_size)
     codes = np.zeros((r, k))
     qhat = np.zeros((r, k))
@@ -334,7 +373,9 @@ def sweep_blocked(W, U, bits, group_size, block_size, include_zero=True,
         e0 = min(s0 + B, k)
         Err = np.zeros((r, e0 - s0))
         for i in range(s0, e0):
-            if i % G == 0:
+            if static is not None:
+                s, z = _static_grid(static, i)
+            elif i % G == 0:
                 s, z = _group_grid(W[:, i:i + G], maxq, include_zero, decide_dtype, fixed_grid, r,
                                    sym)
                 if force_zeros is not None and not sym:  # a symmetric grid's zero is fixed
@@ -361,6 +402,8 @@ def sweep_blocked(W, U, bits, group_size, block_size, include_zero=True,
             w_at[:, i] = w
         if e0 < k:
             W[:, e0:] -= Err @ U[s0:e0, e0:]
+    if static is not None:
+        scales, zeros = static[0], static[1]
     return dict(codes=codes, scales=scales, zeros=zeros, qhat=qhat, err=errs, w_at=w_at,
                 n_forced=n_forced)
 
@@ -386,7 +429,7 @@ def _force_ties(neg_lo, s, z, forced, tau, dt):
 
 
 def sweep_replay(W, U, bits, group_size, block_size, force_codes, force_zeros,
-                 tau=1e-3, include_zero=True, decide_dtype=F32, sym=False):
+                 tau=1e-3, include_zero=True, decide_dtype=F32, sym=False, static=None):
     """Tie-aware replay: the lazy-blocked sweep in fp64, except that wherever
     a candidate result (``force_codes``, ``force_zeros``, sweep order) differs
     from the oracle's decision by exactly one step AND the oracle's value
@@ -394,13 +437,15 @@ def sweep_replay(W, U, bits, group_size, block_size, force_codes, force_zeros,
     a rounding tie, the candidate's decision is taken.  Both decisions are
     valid there (the fp32 and fp64 inputs straddle the tie); every other
     decision must then agree exactly.  Returns the same dict as
-    ``sweep_blocked`` with ``n_forced``."""
+    ``sweep_blocked`` with ``n_forced``.  Static grids (``static``) are
+    fixed before the sweep from the same fp32 inputs, so only codes are
+    replayed there."""
     return sweep_blocked(W, U, bits, group_size, block_size, include_zero,
-                         decide_dtype, force_codes, force_zeros, tau, sym=sym)
+                         decide_dtype, force_codes, force_zeros, tau, sym=sym, static=static)
 
 
 def sweep_obs(W, Hd, bits, group_size, include_zero=True, decide_dtype=F32,
-              fixed_grid=None, sym=False):
+              fixed_grid=None, sym=False, static=None):
     """Column sweep with an explicit inverse Hessian and the Optimal Brain
     Surgeon downdate.
 
@@ -412,8 +457,8 @@ def sweep_obs(W, Hd, bits, group_size, include_zero=True, decide_dtype=F32,
     remaining j; then Hinv -= Hinv[:, i] Hinv[i, :] / Hinv[i, i].  [GPTQ-tool]
     Step 6 says the rows of the Cholesky factor hold exactly these numbers, so
     this equals ``sweep_unblocked`` up to rounding (a pin, not a product path).
-    ``Hd`` is the damped Hessian in sweep order; ``fixed_grid`` as in
-    ``sweep_unblocked``.
+    ``Hd`` is the damped Hessian in sweep order; ``fixed_grid`` and
+    ``static`` as in ``sweep_unblocked``.
     """
     W = np.array(W, dtype=F64, copy=True)
     r, k = W.shape
@@ -427,7 +472,9 @@ def sweep_obs(W, Hd, bits, group_size, include_zero=True, decide_dtype=F32,
     zeros = np.zeros((r, ng), dtype=decide_dtype)
     s = z = None
     for i in range(k):
-        if i % G == 0:
+        if static is not None:
+            s, z = _static_grid(static, i)
+        elif i % G == 0:
             s, z = _group_grid(W[:, i:i + G], maxq, include_zero, decide_dtype, fixed_grid, r, sym)
             scales[:, i // G] = s
             zeros[:, i // G] = z
@@ -439,6 +486,8 @@ def sweep_obs(W, Hd, bits, group_size, include_zero=True, decide_dtype=F32,
         Hinv = Hinv - np.outer(Hinv[:, i], Hinv[i, :]) / Hinv[i, i]
         codes[:, i] = c
         qhat[:, i] = q
+    if static is not None:
+        scales, zeros = static[0], static[1]
     return dict(codes=codes, scales=scales, zeros=zeros, qhat=qhat)
 
 
@@ -483,7 +532,8 @@ def layer_loss(W0, qhat, H0):
 
 def gptq(W, H, bits=4, group_size=128, block_size=128, percdamp=0.01,
          act_order=False, include_zero=True, decide_dtype=F32, blocked=True, sym=False,
-         force_codes=None, force_zeros=None, tau=1e-3, force_perm=None, tau_perm=1e-5):
+         force_codes=None, force_zeros=None, tau=1e-3, force_perm=None, tau_perm=1e-5,
+         static_groups=False):
     """GPTQ for one linear layer, given W (r, k) and the undamped Hessian H.
 
     Order of steps ([GPTQ-tool] *How it works* Steps 3-8): dead columns
@@ -497,6 +547,10 @@ def gptq(W, H, bits=4, group_size=128, block_size=128, percdamp=0.01,
     tie-aware replay (``sweep_replay``); ``force_perm`` a candidate act-order
     permutation, accepted only where it is a valid order within ``tau_perm``
     (see ``act_order_perm``).
+
+    ``static_groups`` (READING R15): grids fixed before the sweep from the
+    dead-column-fixed weights in their original column order; scales / zeros
+    are then per (row, original group) and g_idx[c] = c // G.
     """
     W0 = np.asarray(W, dtype=F64)
     H0 = np.asarray(H, dtype=F64)
@@ -510,22 +564,31 @@ def gptq(W, H, bits=4, group_size=128, block_size=128, percdamp=0.01,
     Hp = Hf[np.ix_(perm, perm)]
     Hd = damp(Hp, percdamp)
     U = hinv_upper_factor(Hd)
+    G = k if group_size == -1 else group_size
+    static = None
+    if static_groups:
+        ss, zz = static_grids(Wf, bits, group_size, include_zero, decide_dtype, sym)
+        static = (ss, zz, perm // G)
     if force_codes is not None:
         fc = np.asarray(force_codes)[:, perm]
-        res = sweep_replay(Wp, U, bits, group_size, block_size, fc, force_zeros,
-                           tau, include_zero, decide_dtype, sym)
+        res = sweep_replay(Wp, U, bits, group_size, block_size, fc,
+                           None if static_groups else force_zeros,
+                           tau, include_zero, decide_dtype, sym, static)
     elif blocked:
         res = sweep_blocked(Wp, U, bits, group_size, block_size, include_zero, decide_dtype,
-                            sym=sym)
+                            sym=sym, static=static)
     else:
-        res = sweep_unblocked(Wp, U, bits, group_size, include_zero, decide_dtype, sym=sym)
-    G = k if group_size == -1 else group_size
+        res = sweep_unblocked(Wp, U, bits, group_size, include_zero, decide_dtype, sym=sym,
+                              static=static)
     codes = np.zeros((r, k))
     qhat = np.zeros((r, k))
     codes[:, perm] = res["codes"]
     qhat[:, perm] = res["qhat"]
-    g_idx = np.zeros(k, dtype=np.int64)
-    g_idx[perm] = np.arange(k) // G
+    if static_groups:
+        g_idx = np.arange(k, dtype=np.int64) // G
+    else:
+        g_idx = np.zeros(k, dtype=np.int64)
+        g_idx[perm] = np.arange(k) // G
     loss, per_row = layer_loss(W0, qhat, H0)
     return dict(codes=codes.astype(np.int64), scales=res["scales"], zeros=res["zeros"],
                 g_idx=g_idx, perm=perm, dead=dead, U=U, qhat=qhat, loss=loss,

@@ -244,6 +244,113 @@ def test_symmetric_invariants(gs, bs, act):
     assert np.array_equal(a["codes"], c["codes"])
 
 
+# ---------------------------------------------------------------- static groups (R15)
+
+def test_static_grid_closed_form():
+    # READING R15: a static grid is fitted to the ORIGINAL columns of its group.
+    # 2 bits (maxq 3), G = 2: group 1 holds 0.75 and 0.25 (exact binary values),
+    # so lo = min(0, 0.25) = 0, hi = 0.75, scale = 0.75 / 3 = 0.25, zero = 0.
+    # Column 0 (0.6 on a grid of step ~0.25, zero 1) is rounded with an error,
+    # and a strongly correlated H moves columns 2 and 3 before they are
+    # quantized, so the dynamic grid of group 1 (fitted after compensation)
+    # differs while the first group's grid is the same either way.
+    W = np.array([[0.6, -0.15, 0.75, 0.25]])
+    C = np.array([[1.0, 0.9, 0.8, 0.7], [0.9, 1.0, 0.9, 0.8], [0.8, 0.9, 1.0, 0.9],
+                  [0.7, 0.8, 0.9, 1.0]])
+    st = O.gptq(W, C, bits=2, group_size=2, block_size=2, percdamp=0.01, static_groups=True)
+    assert st["scales"][0, 1] == 0.25 and st["zeros"][0, 1] == 0
+    dy = O.gptq(W, C, bits=2, group_size=2, block_size=2, percdamp=0.01)
+    assert dy["scales"][0, 0] == st["scales"][0, 0] and dy["zeros"][0, 0] == 1
+    assert dy["scales"][0, 1] != 0.25
+    # column 0 is quantized first on either grid: rint(0.6 / 0.25) + 1 = 3
+    assert st["codes"][0, 0] == 3 and dy["codes"][0, 0] == 3
+
+
+@pytest.mark.parametrize("gs,bs", [(32, 32), (48, 32), (-1, 64), (16, 64)])
+def test_static_groups_diagonal_hessian_is_rtn_in_original_order(gs, bs):
+    # A diagonal H means no compensation, so every column is rounded on its
+    # grid alone; with static groups those grids are RTN's on the ORIGINAL
+    # columns, whatever order act-order imposes.  Processing-order groups (the
+    # dynamic rule) would fail this under act-order.  Dead column 7 counts as 0.
+    rng = np.random.default_rng(21)
+    r, k = 12, 96
+    W = rng.normal(0, 0.02, (r, k))
+    d = rng.lognormal(0, 1, k)
+    d[7] = 0.0
+    H = np.diag(d)
+    res = O.gptq(W, H, bits=3, group_size=gs, block_size=bs, act_order=True,
+                 static_groups=True)
+    assert not np.array_equal(res["perm"], np.arange(k))
+    W0 = W.copy()
+    W0[:, 7] = 0.0
+    ref = O.rtn(W0, 3, gs)
+    assert np.array_equal(res["codes"], ref["codes"])
+    assert np.array_equal(res["scales"], ref["scales"])
+    assert np.array_equal(res["zeros"], ref["zeros"])
+    G = k if gs == -1 else gs
+    assert np.array_equal(res["g_idx"], np.arange(k) // G)
+
+
+@pytest.mark.parametrize("gs,B,act", [(48, 32, True), (32, 32, False), (8, 96, True),
+                                      (100, 64, False)])
+def test_static_groups_blocked_unblocked_obs_agree(gs, B, act):
+    # With grids fixed before the sweep, the lazy blocks cannot change a grid,
+    # so the blocked sweep equals the column-by-column one for ANY group and
+    # block sizes (no alignment needed), and both equal the OBS downdate.
+    W, _, H = _rand_layer(31, 10, 192)
+    k = W.shape[1]
+    G = k if gs == -1 else gs
+    Hf, Wf, _ = O.fix_dead_columns(H, W)
+    perm = O.act_order_perm(Hf) if act else np.arange(k)
+    Wp, Hd = Wf[:, perm], O.damp(Hf[np.ix_(perm, perm)], 0.01)
+    U = O.hinv_upper_factor(Hd)
+    ss, zz = O.static_grids(Wf, 4, gs)
+    st = (ss, zz, perm // G)
+    a = O.sweep_unblocked(Wp, U, 4, gs, static=st)
+    b = O.sweep_blocked(Wp, U, 4, gs, B, static=st)
+    c = O.sweep_obs(Wp, Hd, 4, gs, static=st)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["codes"], c["codes"])
+    assert np.allclose(a["qhat"], b["qhat"], rtol=0, atol=1e-15)
+    res = O.gptq(W, H, 4, gs, B, 0.01, act, static_groups=True)
+    assert np.array_equal(res["codes"][:, perm], b["codes"])
+
+
+@pytest.mark.parametrize("act", [False, True])
+def test_static_equals_dynamic_for_one_group_per_row(act):
+    # group_size = -1: the dynamic rule already takes the row's one grid from
+    # the original row before the first column (READING R5), so static and
+    # dynamic groups are the same computation.
+    W, _, H = _rand_layer(5, 8, 64)
+    a = O.gptq(W, H, 4, -1, 32, 0.01, act)
+    b = O.gptq(W, H, 4, -1, 32, 0.01, act, static_groups=True)
+    assert np.array_equal(a["codes"], b["codes"])
+    assert np.array_equal(a["scales"], b["scales"]) and np.array_equal(a["zeros"], b["zeros"])
+    assert a["loss"] == b["loss"]
+
+
+def test_static_groups_loss_identity_and_sym():
+    # The OBS accounting (loss = sum err^2 - lambda ||W0 - Q||^2) does not depend
+    # on how the grids were chosen; checked with static groups, act-order, dead
+    # columns and both grid kinds.  Static symmetric grids keep zero = (maxq+1)/2.
+    spec = synth.CONFIGS["q_proj"].scaled(r=16, k=128, n=2000)
+    W = synth.make_w(spec, 4).numpy().astype(np.float64)
+    X = synth.make_x(spec, 4).numpy()
+    X[:, 9] = 0
+    H = O.hessian(X)
+    for sym in (False, True):
+        res = O.gptq(W, H, 4, 32, 64, 0.01, True, sym=sym, static_groups=True)
+        Hf, Wf, _ = O.fix_dead_columns(H, W)
+        perm = res["perm"]
+        lam = 0.01 * np.mean(np.diag(Hf))
+        ss, zz = O.static_grids(Wf, 4, 32, sym=sym)
+        sw = O.sweep_blocked(Wf[:, perm], res["U"], 4, 32, 64, sym=sym, static=(ss, zz, perm // 32))
+        e2 = (sw["err"] ** 2).sum(axis=1)
+        d2 = ((Wf[:, perm] - sw["qhat"]) ** 2).sum(axis=1)
+        assert np.allclose(e2 - lam * d2, res["loss_rows"], rtol=1e-10, atol=0)
+        if sym:
+            assert np.all(res["zeros"] == 8)
+
+
 def test_half_to_even_rounding():
     c = O.quantize_codes(np.array([6.5, 7.5, -0.5, 2.4999]), 1.0, 0.0, None)
     assert list(c) == [6, 8, 0, 2]
