@@ -174,16 +174,24 @@ def oracle_sample(spec, seed, n_tokens, n_rows):
     Hd = O.damp(Hf[np.ix_(perm, perm)], spec.percdamp)
     U = O.hinv_upper_factor(Hd)
     t2 = time.perf_counter()
-    res = O.sweep_blocked(Wf[:, perm], U, spec.bits, spec.group_size, spec.block_size)
+    G = spec.k if spec.group_size == -1 else spec.group_size
+    static = None
+    if spec.static_groups:
+        ss, zz = O.static_grids(Wf, spec.bits, spec.group_size, sym=spec.sym)
+        static = (ss, zz, perm // G)
+    res = O.sweep_blocked(Wf[:, perm], U, spec.bits, spec.group_size, spec.block_size,
+                          sym=spec.sym, static=static)
     codes = np.zeros_like(res["codes"], dtype=np.int64)
     codes[:, perm] = res["codes"]
     qhat = np.zeros_like(res["qhat"])
     qhat[:, perm] = res["qhat"]
     O.layer_loss(Wn, qhat, H)
     t3 = time.perf_counter()
-    G = spec.k if spec.group_size == -1 else spec.group_size
-    g_idx = np.zeros(spec.k, dtype=np.int64)
-    g_idx[perm] = np.arange(spec.k) // G
+    if spec.static_groups:
+        g_idx = np.arange(spec.k, dtype=np.int64) // G
+    else:
+        g_idx = np.zeros(spec.k, dtype=np.int64)
+        g_idx[perm] = np.arange(spec.k) // G
     qw = O.pack(codes, spec.bits)
     O.dequant(O.unpack(qw, spec.k, spec.bits), res["scales"], res["zeros"], g_idx, np.float16)
     t4 = time.perf_counter()
@@ -237,8 +245,10 @@ def workload_config(spec):
     G = "per-row" if spec.group_size == -1 else f"g{spec.group_size}"
     return {
         "workload": (f"{spec.name}: W {spec.r}x{spec.k} {spec.w_dtype}, X {spec.n}x{spec.k} "
-                     f"{spec.x_dtype} ({spec.x_kind}), int{spec.bits} asym {G} B{spec.block_size} "
-                     f"damp {spec.percdamp}{' act-order' if spec.act_order else ''}"),
+                     f"{spec.x_dtype} ({spec.x_kind}), int{spec.bits} "
+                     f"{'sym' if spec.sym else 'asym'} {G} B{spec.block_size} "
+                     f"damp {spec.percdamp}{' act-order' if spec.act_order else ''}"
+                     f"{' static-groups' if spec.static_groups else ''}"),
         "l2": f"inputs larger than L2 (X {spec.n * spec.k * 2 / 1e9:.2f} GB), no flush",
     }
 
@@ -251,7 +261,8 @@ def native_arm(args, spec, world, rank, local):
 
     dev = torch.device("cuda", local if world > 1 else 0)
     seed = args.seed + rank  # independent layer per rank (weak scaling)
-    cfg = QuantConfig(spec.bits, spec.group_size, spec.block_size, spec.percdamp, spec.act_order)
+    cfg = QuantConfig(spec.bits, spec.group_size, spec.block_size, spec.percdamp, spec.act_order,
+                      spec.sym, spec.static_groups)
     xdt = synth.dtype_of(spec.x_dtype)
     X_host = torch.empty(spec.n, spec.k, dtype=xdt, pin_memory=True)
     synth.make_x(spec, seed, out=X_host)
@@ -465,12 +476,18 @@ def main():
     ap.add_argument("--rows", type=int, default=None, help="override the row count of W")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per Hessian launch from an ncu capture of this kernel")
+    ap.add_argument("--act-order", action="store_true", help="variant: act-order")
+    ap.add_argument("--sym", action="store_true", help="variant: symmetric grid")
+    ap.add_argument("--static-groups", action="store_true", help="variant: static groups")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     spec = synth.CONFIGS[args.config]
     if args.tokens or args.rows:
         spec = spec.scaled(r=args.rows, n=args.tokens)
+    if args.act_order or args.sym or args.static_groups:
+        spec = spec.scaled(act_order=spec.act_order or args.act_order, sym=args.sym,
+                           static_groups=args.static_groups)
     if args.impl == "reference":
         # CPU only: rank 0 runs the oracle, other ranks exit without work
         return reference_arm(args, spec, int(os.environ.get("WORLD_SIZE", "1")),

@@ -70,7 +70,8 @@ typedef enum { GPTQ_F32 = 0, GPTQ_F16 = 1, GPTQ_BF16 = 2 } gptq_dtype;
  *   bits        2, 3, 4 or 8: codes are 0 .. 2^bits-1 on an asymmetric grid.
  *   group_size  columns (in processing order) sharing one scale/zero per row;
  *               -1 = one group per row.  Must divide block_size or be a
- *               multiple of it, so a group never straddles a lazy block.
+ *               multiple of it, so a group never straddles a lazy block
+ *               (any positive size when static_groups is set).
  *   block_size  lazy-batch width B ([GPTQ-tool] Step 7), 16..128, multiple of 16.
  *   percdamp    damping fraction of mean(diag H) ([GPTQ-tool] Step 4), >= 0.
  *   act_order   nonzero: process columns by descending diag(H).
@@ -78,6 +79,17 @@ typedef enum { GPTQ_F32 = 0, GPTQ_F16 = 1, GPTQ_BF16 = 2 } gptq_dtype;
  *               1: symmetric grid about 0, scale = 2 max(|min|, |max|) / maxq and
  *               zero point (maxq + 1) / 2 for every group ("GPTQ",
  *               ozercemkelahmet.com/tools/gptq, Optional refinements).
+ *               Other values: GPTQ_ERR_INVALID_ARG.
+ *   static_groups  0: each group's grid is fitted when the sweep reaches the
+ *               group, to the already-compensated weights (groups of
+ *               consecutive processing positions; g_idx[c] = position / G).
+ *               1: every grid is fitted before the sweep to the original
+ *               weights (dead columns as 0) of the original columns
+ *               [g G, (g+1) G); a column keeps its original group under
+ *               act_order, so g_idx[c] = c / G.  (The static_groups flag of
+ *               the AutoGPTQ configuration in "GPTQ Quantization: Complete
+ *               Technical Guide", Configuration Deep Dive; its meaning there
+ *               is not spelled out and this is the plain reading of the name.)
  *               Other values: GPTQ_ERR_INVALID_ARG. */
 typedef struct {
   int bits;
@@ -86,6 +98,7 @@ typedef struct {
   float percdamp;
   int act_order;
   int sym;
+  int static_groups;
 } gptq_config;
 
 typedef enum {

@@ -62,13 +62,14 @@ class GptqConfig(ctypes.Structure):
         ("percdamp", ctypes.c_float),
         ("act_order", ctypes.c_int),
         ("sym", ctypes.c_int),
+        ("static_groups", ctypes.c_int),
     ]
 
 
 def make_config(bits=4, group_size=128, block_size=128, percdamp=0.01, act_order=False,
-                sym=False):
+                sym=False, static_groups=False):
     return GptqConfig(int(bits), int(group_size), int(block_size), float(percdamp),
-                      int(bool(act_order)), int(bool(sym)))
+                      int(bool(act_order)), int(bool(sym)), int(bool(static_groups)))
 
 
 _lib = None

@@ -28,10 +28,11 @@ class QuantConfig:
     percdamp: float = 0.01
     act_order: bool = False
     sym: bool = False  # symmetric grid (zero point at the middle code)
+    static_groups: bool = False  # grids fitted before the sweep, original column groups
 
     def c(self):
         return make_config(self.bits, self.group_size, self.block_size, self.percdamp,
-                           self.act_order, self.sym)
+                           self.act_order, self.sym, self.static_groups)
 
     def ngroups(self, k: int) -> int:
         G = k if self.group_size == -1 else self.group_size

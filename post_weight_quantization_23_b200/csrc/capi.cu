@@ -42,13 +42,15 @@ gptq_status check_config(const gptq_config* cfg, int64_t k) {
   if (cfg == nullptr) return GPTQ_ERR_INVALID_ARG;
   if (!valid_bits(cfg->bits)) return GPTQ_ERR_UNSUPPORTED;
   if (cfg->sym != 0 && cfg->sym != 1) return GPTQ_ERR_INVALID_ARG;
+  if (cfg->static_groups != 0 && cfg->static_groups != 1) return GPTQ_ERR_INVALID_ARG;
   if (!(cfg->percdamp >= 0.0f) || !isfinite(cfg->percdamp)) return GPTQ_ERR_INVALID_ARG;
   const int B = cfg->block_size;
   if (B < 16 || B > 128 || B % 16 != 0) return GPTQ_ERR_UNSUPPORTED;
   const int G = cfg->group_size;
   if (G != -1) {
     if (G <= 0) return GPTQ_ERR_INVALID_ARG;
-    if (!(B % G == 0 || G % B == 0)) return GPTQ_ERR_INVALID_ARG;
+    // dynamic grids are fitted at a group's start inside one lazy block
+    if (!cfg->static_groups && !(B % G == 0 || G % B == 0)) return GPTQ_ERR_INVALID_ARG;
   }
   (void)k;
   return GPTQ_OK;

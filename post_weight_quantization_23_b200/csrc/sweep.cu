@@ -109,15 +109,17 @@ __device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
 template <typename T>
 __global__ void sweep_init_kernel(const T* __restrict__ W, int64_t ldw, int r, int k,
                                   const int32_t* __restrict__ perm,
-                                  const uint8_t* __restrict__ dead, int G, float* __restrict__ Wt,
-                                  int32_t* __restrict__ g_idx, double* __restrict__ loss,
-                                  int32_t* __restrict__ d_status) {
+                                  const uint8_t* __restrict__ dead, int G, int static_groups,
+                                  float* __restrict__ Wt, int32_t* __restrict__ g_idx,
+                                  double* __restrict__ loss, int32_t* __restrict__ d_status) {
   int row = blockIdx.y;
   for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < k; j += gridDim.x * blockDim.x) {
     int c = perm[j];
     float v = dead[c] ? 0.f : to_f32(W[(int64_t)row * ldw + c]);
     Wt[(int64_t)row * k + j] = v;
-    if (row == 0) g_idx[c] = j / G;
+    // dynamic groups are runs of processing positions; static ones keep the
+    // original columns together
+    if (row == 0) g_idx[c] = (static_groups ? c : j) / G;
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     if (loss != nullptr) {
@@ -171,6 +173,38 @@ __global__ void group_grid_kernel(const float* __restrict__ Wt, int r, int k, in
     grid_from_range(mn, mx, maxq, sc, z, sym != 0);
     scales[(int64_t)warp * ngroups + gidx] = sc;
     zeros[(int64_t)warp * ngroups + gidx] = (int32_t)z;
+  }
+}
+
+// Static groups: the grid of every (row, group), fitted before the sweep to
+// the original weights of the original columns [g G, g G + G) (dead columns
+// count as 0).  One warp per (row, group).
+template <typename T>
+__global__ void static_grid_kernel(const T* __restrict__ W, int64_t ldw, int r, int k,
+                                   const uint8_t* __restrict__ dead, int G, int ngroups,
+                                   float maxq, int sym, float* __restrict__ scales,
+                                   int32_t* __restrict__ zeros) {
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / kWarp;
+  const int lane = threadIdx.x % kWarp;
+  if (warp >= (int64_t)r * ngroups) return;
+  const int row = (int)(warp / ngroups), g = (int)(warp % ngroups);
+  const int c0 = g * G, c1 = min(k, c0 + G);
+  const T* w = W + (int64_t)row * ldw;
+  float mn = INFINITY, mx = -INFINITY;
+  for (int c = c0 + lane; c < c1; c += kWarp) {
+    const float v = dead[c] ? 0.f : to_f32(w[c]);
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    float sc, z;
+    grid_from_range(mn, mx, maxq, sc, z, sym != 0);
+    scales[warp] = sc;
+    zeros[warp] = (int32_t)z;
   }
 }
 
@@ -383,9 +417,24 @@ template <int L>
 struct SqState {
   float w[SqLayout<L>::S];
   float scale, zero, inv_s, lo_d, hi_d;
+  float next_scale, next_zero;  // MODE 2: this lane's column of the next sub-block
   double e2;
   bool nonfinite;
 };
+
+// MODE 2 (static groups): fetch the fixed grid of this lane's column in
+// sub-block m, i.e. group perm[s + c] / G of the row.
+template <int L>
+__device__ __forceinline__ void sq_fetch_static(SqState<L>& st, int m, const SqArgs& a,
+                                                const int32_t* pcol, int l, int row, bool valid) {
+  const int c = L * m + l;
+  st.next_scale = 1.f, st.next_zero = 0.f;
+  if (valid && c < a.bw) {
+    const int64_t idx = (int64_t)row * a.ngroups + pcol[c] / a.G;
+    st.next_scale = a.scales[idx];
+    st.next_zero = (float)a.zeros[idx];
+  }
+}
 
 // One sub-block (columns L m .. L m + L - 1) with a register window of W + 1 slots.
 template <int L, int W, int MODE>
@@ -422,6 +471,22 @@ __device__ __forceinline__ void sq_sub_block(SqState<L>& st, int m, const SqArgs
       a.zeros[(int64_t)row * a.ngroups + g] = (int32_t)st.zero;
     }
   }
+  // MODE 2: every column has its own fixed grid; lane o holds column o's
+  // (fetched one sub-block ahead) and the row's lanes share them by shuffles
+  float own_zero = st.zero;
+  float gs[L], gi[L], gz[L];
+  if (MODE == 2) {
+    const float own_scale = st.next_scale;
+    own_zero = st.next_zero;
+    sq_fetch_static(st, m + 1, a, pcol, l, row, valid);
+    const float own_inv = 1.0f / own_scale;
+#pragma unroll
+    for (int o = 0; o < L; ++o) {
+      gs[o] = __shfl_sync(0xffffffffu, own_scale, o, L);
+      gi[o] = __shfl_sync(0xffffffffu, own_inv, o, L);
+      gz[o] = __shfl_sync(0xffffffffu, own_zero, o, L);
+    }
+  }
   float rd[L];
 #pragma unroll
   for (int v = 0; v < L / 4; ++v) {
@@ -435,11 +500,14 @@ __device__ __forceinline__ void sq_sub_block(SqState<L>& st, int m, const SqArgs
   bool tie = false;
 #pragma unroll
   for (int o = 0; o < L; ++o) {
-    const float t = x[o] * st.inv_s;
+    const float sc = MODE == 2 ? gs[o] : st.scale;
+    const float lo_d = MODE == 2 ? -gz[o] : st.lo_d;
+    const float hi_d = MODE == 2 ? a.maxq - gz[o] : st.hi_d;
+    const float t = x[o] * (MODE == 2 ? gi[o] : st.inv_s);
     const float rq = rintf(t);
     tie |= fabsf(fabsf(t - rq) - 0.5f) <= 1e-6f * fabsf(t);
-    const float d = fminf(fmaxf(rq, st.lo_d), st.hi_d);  // code - zero
-    const float e = (x[o] - st.scale * d) * rd[o];
+    const float d = fminf(fmaxf(rq, lo_d), hi_d);  // code - zero
+    const float e = (x[o] - sc * d) * rd[o];
     err[o] = e;
     dq[o] = d;
     if (o + 1 < L) {
@@ -453,8 +521,11 @@ __device__ __forceinline__ void sq_sub_block(SqState<L>& st, int m, const SqArgs
     for (int o = 0; o < L; ++o) x[o] = x0[o];
 #pragma unroll
     for (int o = 0; o < L; ++o) {
-      const float d = fminf(fmaxf(rint_exact_div(x[o], st.scale), st.lo_d), st.hi_d);
-      const float e = (x[o] - st.scale * d) * rd[o];
+      const float sc = MODE == 2 ? gs[o] : st.scale;
+      const float lo_d = MODE == 2 ? -gz[o] : st.lo_d;
+      const float hi_d = MODE == 2 ? a.maxq - gz[o] : st.hi_d;
+      const float d = fminf(fmaxf(rint_exact_div(x[o], sc), lo_d), hi_d);
+      const float e = (x[o] - sc * d) * rd[o];
       err[o] = e;
       dq[o] = d;
       if (o + 1 < L) {
@@ -487,7 +558,7 @@ __device__ __forceinline__ void sq_sub_block(SqState<L>& st, int m, const SqArgs
     if (l == o) e_own = err[o], d_own = dq[o];
   const int c = L * m + l;
   if (valid && c < a.bw) {
-    a.codes[(int64_t)row * a.k + pcol[c]] = (uint8_t)(d_own + st.zero);
+    a.codes[(int64_t)row * a.k + pcol[c]] = (uint8_t)(d_own + own_zero);
     if (a.Err_lo != nullptr) {
       float h, lo;
       split_tf32(e_own, h, lo);
@@ -506,8 +577,10 @@ __device__ __forceinline__ void sq_sub_block(SqState<L>& st, int m, const SqArgs
 
 // One lazy block [s, s + bw) for 32 / L rows per warp.  MODE 1: groups start
 // inside the block (G <= B, G % L == 0); MODE 0: the block lies inside one
-// group whose grid is already in scales / zeros.  Adds sum_i err_i^2 of the
-// block to loss[row] (the Optimal Brain Surgeon part of the layer loss).
+// group whose grid is already in scales / zeros; MODE 2: static groups, each
+// column's grid read from scales / zeros (group perm[col] / G).  Adds
+// sum_i err_i^2 of the block to loss[row] (the Optimal Brain Surgeon part of
+// the layer loss).
 template <int L, int MODE>
 __global__ void __launch_bounds__(SQ_MAX_WARPS * 32, 1) sweep_block_lane_kernel(SqArgs a) {
   using Ly = SqLayout<L>;
@@ -566,6 +639,7 @@ __global__ void __launch_bounds__(SQ_MAX_WARPS * 32, 1) sweep_block_lane_kernel(
     if (tid == 0 && a.d_status != nullptr) atomicCAS(a.d_status, 0, (int32_t)GPTQ_ERR_TIMEOUT);
     return;
   }
+  if (MODE == 2) sq_fetch_static(st, 0, a, pcol, l, row, valid);  // needs pcol from the record
   constexpr int S = Ly::S;
   const int nsb = (a.bw + L - 1) / L;
   int m = 0;
@@ -678,8 +752,14 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
   double* lossp = want_loss ? loss : nullptr;
   {
     dim3 grid((unsigned)cdiv(k, 1024), (unsigned)r);
-    sweep_init_kernel<T><<<grid, 256, 0, s>>>(W, ldw, r, k, perm, dead, G, sc.Wt, g_idx, lossp,
-                                              d_status);
+    sweep_init_kernel<T><<<grid, 256, 0, s>>>(W, ldw, r, k, perm, dead, G, cfg->static_groups,
+                                              sc.Wt, g_idx, lossp, d_status);
+    GPTQ_CHECK_LAUNCH();
+  }
+  const bool stat = cfg->static_groups != 0;
+  if (stat) {
+    static_grid_kernel<T><<<(unsigned)cdiv((int64_t)r * ngroups * kWarp, 256), 256, 0, s>>>(
+        W, ldw, r, k, dead, G, ngroups, maxq, cfg->sym, scales, zeros);
     GPTQ_CHECK_LAUNCH();
   }
   if (want_loss) {
@@ -696,7 +776,8 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
   // row unless the rows alone fill the SMs with 2 warps per scheduler, or the
   // groups need 4 -- else the 4-threads-per-row kernel
   int lane_mode = -1, lanes = 8;
-  if (G > B) lane_mode = 0;
+  if (stat) lane_mode = 2;  // any group size: grids are looked up per column
+  else if (G > B) lane_mode = 0;
   else if (G % 4 == 0) lane_mode = 1;
   const int nblocks = (int)cdiv(k, B);
   int q_warps = 1;
@@ -723,7 +804,7 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
   float* err_lo = tc ? sc.Err_lo : nullptr;
   for (int s0 = 0, b = 0; s0 < k; s0 += B, ++b) {
     int bw = min(B, k - s0);
-    if (G > B && s0 % G == 0) {
+    if (!stat && G > B && s0 % G == 0) {
       int gw = min(G, k - s0);
       group_grid_kernel<<<(unsigned)cdiv((int64_t)r * kWarp, 256), 256, 0, s>>>(
           sc.Wt, r, k, s0, gw, s0 / G, ngroups, maxq, cfg->sym, scales, zeros);
@@ -743,13 +824,16 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
       a.codes = codes;
       a.loss = lossp;
       a.d_status = d_status;
-      const bool pdl = b > 0 && !(G > B && s0 % G == 0);  // right behind a trailing update
+      // right behind a trailing update (not behind a group grid launch)
+      const bool pdl = b > 0 && !(!stat && G > B && s0 % G == 0);
       if (lanes == 8) {
         if (lane_mode == 0) launch_lane<8, 0>(q_grid, 32 * q_warps, s, a, pdl);
-        else launch_lane<8, 1>(q_grid, 32 * q_warps, s, a, pdl);
+        else if (lane_mode == 1) launch_lane<8, 1>(q_grid, 32 * q_warps, s, a, pdl);
+        else launch_lane<8, 2>(q_grid, 32 * q_warps, s, a, pdl);
       } else {
         if (lane_mode == 0) launch_lane<4, 0>(q_grid, 32 * q_warps, s, a, pdl);
-        else launch_lane<4, 1>(q_grid, 32 * q_warps, s, a, pdl);
+        else if (lane_mode == 1) launch_lane<4, 1>(q_grid, 32 * q_warps, s, a, pdl);
+        else launch_lane<4, 2>(q_grid, 32 * q_warps, s, a, pdl);
       }
     } else {
 #define GPTQ_SWEEP_BLOCK(SBV)                                                                  \

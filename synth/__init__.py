@@ -50,6 +50,8 @@ class LayerSpec:
     block_size: int = 128
     percdamp: float = 0.01
     act_order: bool = False
+    sym: bool = False            # symmetric grid
+    static_groups: bool = False  # grids fixed before the sweep
 
     def scaled(self, r=None, k=None, n=None, **kw):
         """Same distributions at other sizes (for parity runs the oracle can finish)."""

@@ -79,22 +79,23 @@ def compare(gpu, W_np, X_np, cfg, rows=None, H=None):
     Wc = W_np if rows is None else W_np[rows]
     gperm = gpu["perm"].numpy().astype(np.int64)
     sym = bool(getattr(cfg, "sym", False))
+    stat = bool(getattr(cfg, "static_groups", False))
     own = O.gptq(Wc[:1], H, cfg.bits, cfg.group_size, cfg.block_size, cfg.percdamp, cfg.act_order,
-                 sym=sym)
+                 sym=sym, static_groups=stat)
     perm_diff = int((own["perm"] != gperm).sum())
     # the act-order permutation is decided from floating-point diag(H): the
     # oracle takes the GPU's order where (and only where) it is a valid order
     # within the Hessian tolerance; everything downstream is then compared
     fp = gperm if cfg.act_order else None
     ref = O.gptq(Wc, H, cfg.bits, cfg.group_size, cfg.block_size, cfg.percdamp, cfg.act_order,
-                 force_perm=fp, tau_perm=TOL_H_REL_FRO, sym=sym)
+                 force_perm=fp, tau_perm=TOL_H_REL_FRO, sym=sym, static_groups=stat)
     sel = slice(None) if rows is None else rows
     codes = gpu["codes"].numpy().astype(np.int64)[sel]
     zeros = gpu["zeros"].numpy().astype(np.int64)[sel]
     scales = gpu["scales"].numpy()[sel]
     rep = O.gptq(Wc, H, cfg.bits, cfg.group_size, cfg.block_size, cfg.percdamp, cfg.act_order,
                  force_codes=codes, force_zeros=zeros, tau=TIE_TAU, force_perm=fp,
-                 tau_perm=TOL_H_REL_FRO, sym=sym)
+                 tau_perm=TOL_H_REL_FRO, sym=sym, static_groups=stat)
     perm_equal = bool(np.array_equal(gperm, ref["perm"]))
     U = gpu["U"].double().numpy()
     u_rel = float(np.abs(U - ref["U"]).max() / np.abs(ref["U"]).max())

@@ -89,6 +89,13 @@ def test_host_argument_checks(lib):
     bad_sym = _lib.make_config(4, 128, 128, 0.01, False)
     bad_sym.sym = 2
     assert q(ctypes.byref(bad_sym)) == _lib.GPTQ_ERR_INVALID_ARG
+    bad_static = _lib.make_config(4, 128, 128, 0.01, False)
+    bad_static.static_groups = 2
+    assert q(ctypes.byref(bad_static)) == _lib.GPTQ_ERR_INVALID_ARG
+    # groups that straddle lazy blocks are fine once the grids are static: the
+    # call then gets past the config check to the workspace check
+    static_g96 = ctypes.byref(_lib.make_config(4, 96, 128, 0.01, False, static_groups=True))
+    assert q(static_g96, ws=None) == _lib.GPTQ_ERR_WORKSPACE
 
 
 def test_binding_refuses_cpu_tensors():

@@ -23,10 +23,10 @@ def _np(t):
     return t.float().numpy() if t.dtype == torch.bfloat16 else t.numpy()
 
 
-def _cfg(spec, sym=False):
+def _cfg(spec, sym=False, static_groups=False):
     from post_weight_quantization_23_b200 import QuantConfig
     return QuantConfig(spec.bits, spec.group_size, spec.block_size, spec.percdamp, spec.act_order,
-                       sym)
+                       sym, static_groups)
 
 
 CASES = {
@@ -98,6 +98,61 @@ def test_layer_parity_symmetric(name):
     # re-enters its row's compensation and later group grids.  What must hold:
     # the tie-aware replay matches exactly, including the layer loss with the
     # GPU's tie decisions, and the plain match rate stays high.
+    from _parity import TOL_H_REL_FRO, TOL_LOSS_REL, TOL_SCALE_REL
+    assert a.h_rel_fro <= TOL_H_REL_FRO, a
+    assert a.perm_equal and a.gidx_equal, a
+    assert a.replay_mismatch == 0 and a.zero_mismatch_replay == 0, a
+    assert a.scale_rel_replay <= TOL_SCALE_REL, a
+    assert a.loss_rel_replay <= TOL_LOSS_REL, a
+    assert a.code_match >= 0.99, a
+
+
+STATIC_CASES = {
+    # static groups (READING R15): grids fitted before the sweep to the original
+    # columns; with act-order a column keeps its original group
+    "static_q_proj_act": synth.CONFIGS["q_proj"].scaled(r=128, k=512, n=8192, act_order=True),
+    "static_down_act_g16": synth.CONFIGS["down_proj"].scaled(r=64, k=400, n=4096,
+                                                              group_size=16),
+    # groups that straddle lazy blocks (allowed only for static groups)
+    "static_g48_b32": synth.CONFIGS["q_proj"].scaled(r=96, k=480, n=4096, group_size=48,
+                                                     block_size=32, act_order=True),
+    "static_g100_b64_3bit": synth.CONFIGS["tiny"].scaled(r=40, k=300, n=3000, group_size=100,
+                                                         block_size=64, bits=3),
+    "static_per_row_act": synth.CONFIGS["opt175_width"].scaled(r=64, k=384, n=4096,
+                                                               act_order=True),
+    # enough rows for the 4-lanes-per-row kernel
+    "static_4lanes_r9472": synth.CONFIGS["q_proj"].scaled(r=9472, k=256, n=4096, group_size=32,
+                                                          block_size=64, act_order=True),
+}
+
+
+@pytest.mark.parametrize("name", list(STATIC_CASES))
+def test_layer_parity_static_groups(name):
+    spec = STATIC_CASES[name]
+    W, X, Wd, Xd = layer_inputs(spec, seed=6)
+    cfg = _cfg(spec, static_groups=True)
+    gpu = gpu_quantize(Wd, Xd, cfg)
+    G = spec.k if spec.group_size == -1 else spec.group_size
+    assert np.array_equal(gpu["g_idx"].numpy(), np.arange(spec.k) // G)
+    # the grids come from the same fp32 inputs by the same IEEE operations: exact
+    ss, zz = O.static_grids(O.fix_dead_columns(O.hessian(_np(X)), _np(W).astype(np.float64))[1],
+                            spec.bits, spec.group_size)
+    assert np.array_equal(gpu["scales"].numpy(), ss)
+    assert np.array_equal(gpu["zeros"].numpy(), zz.astype(np.int32))
+    a = compare(gpu, _np(W), _np(X), cfg)
+    print(name, a)
+    a.assert_ok()
+
+
+def test_layer_parity_static_symmetric():
+    spec = synth.CONFIGS["q_proj"].scaled(r=128, k=512, n=8192, group_size=64, act_order=True)
+    W, X, Wd, Xd = layer_inputs(spec, seed=7)
+    cfg = _cfg(spec, sym=True, static_groups=True)
+    gpu = gpu_quantize(Wd, Xd, cfg)
+    assert np.all(gpu["zeros"].numpy() == (2 ** cfg.bits) // 2)
+    a = compare(gpu, _np(W), _np(X), cfg)
+    print("static_sym", a)
+    # fixed grids: only code ties can differ, and the replay must match exactly
     from _parity import TOL_H_REL_FRO, TOL_LOSS_REL, TOL_SCALE_REL
     assert a.h_rel_fro <= TOL_H_REL_FRO, a
     assert a.perm_equal and a.gidx_equal, a
