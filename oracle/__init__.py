@@ -47,6 +47,7 @@ from .gptq_oracle import (  # noqa: F401
     pack,
     unpack,
     dequant,
+    dequant_matmul,
     storage_bits_per_weight,
     group_count,
 )

@@ -646,6 +646,25 @@ def dequant(codes, scales, zeros, g_idx, out_dtype=F32):
     return v.astype(out_dtype)
 
 
+def dequant_matmul(X, qweight, scales, zeros, g_idx, bits, k):
+    """The inference product of a quantized layer: Y = X W_hat^T with
+    W_hat[j, c] = scale[j, g_c] * (code[j, c] - zero[j, g_c]), the codes read
+    from the packed words ([GPTQ-tool] *What the output looks like*: a GPU
+    kernel reads the packed data and dequantizes inside the matrix multiply;
+    Step 8: the fused kernel unpacks, scales and multiplies; [What-is-GPTQ]
+    *How it works*: each group is expanded just in time for the multiply).
+    X (m, k), qweight int32 (n, k*bits/32), scales / zeros (n, ngroups),
+    g_idx (k).  Exact fp64 arithmetic on the exact input values (an fp32
+    scale times a small integer is exact in fp64), then one fp64 matrix
+    product.  Returns (m, n) fp64."""
+    codes = unpack(qweight, k, bits)
+    g_idx = np.asarray(g_idx, dtype=np.int64)
+    s = np.asarray(scales, dtype=F32).astype(F64)[:, g_idx]
+    z = np.asarray(zeros, dtype=np.int64)[:, g_idx]
+    W_hat = s * (codes - z).astype(F64)
+    return np.asarray(X, dtype=F64) @ W_hat.T
+
+
 def storage_bits_per_weight(bits, group_size, k, scale_bits=16, zero_bits=None):
     """[GPTQ-tool] *Memory arithmetic*: code bits plus one scale and one zero
     point per group, spread over the group's weights."""

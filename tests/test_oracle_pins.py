@@ -663,3 +663,55 @@ def test_tie_replay_accepts_only_ties():
     rep = O.gptq(W, H, bits=4, group_size=32, block_size=32, force_codes=cand,
                  force_zeros=ref["zeros"], tau=1e-9)
     assert rep["codes"][2, 5] != cand[2, 5]
+
+
+# ---------------------------------------------------------------- inference product
+
+def test_dequant_matmul_worked_word():
+    # One packed word, LSB first: codes 0..7 -> 0x76543210.  scale 0.5, zero 3
+    # gives W_hat = 0.5 * (c - 3) = -1.5, -1, ..., 2.  A token of ones sums it
+    # (0.5 * (28 - 24) = 2.0); the token 1..8 gives 0.5 * sum_i (i + 1)(i - 3)
+    # = 0.5 * (140 - 56 - 24) = 30.
+    qw = np.array([[0x76543210]], dtype=np.int64).astype(np.uint32).view(np.int32)
+    assert O.unpack(qw, 8, 4).tolist() == [list(range(8))]
+    X = np.array([np.ones(8), np.arange(1, 9)], dtype=np.float64)
+    Y = O.dequant_matmul(X, qw, np.array([[0.5]]), np.array([[3]]), np.zeros(8, int), 4, 8)
+    assert Y.tolist() == [[2.0], [30.0]]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_dequant_matmul_identity_and_brute_force(bits):
+    # X = I recovers W_hat^T, exact in fp64, so rounding it to fp32 gives
+    # dequant() of the unpacked codes (one fp32 product, correctly rounded);
+    # a triple loop over plain Python numbers gives the same product.
+    rng = np.random.default_rng(bits)
+    n, k, G = 5, 64, 16
+    codes = rng.integers(0, 2 ** bits, (n, k))
+    scales = (rng.random((n, k // G)) * 0.01 + 1e-3).astype(np.float32)
+    zeros = rng.integers(0, 2 ** bits, (n, k // G))
+    g_idx = rng.permutation(np.arange(k) // G)  # an act-order style g_idx
+    qw = O.pack(codes, bits)
+    Y = O.dequant_matmul(np.eye(k), qw, scales, zeros, g_idx, bits, k)
+    assert np.array_equal(Y.T.astype(np.float32), O.dequant(codes, scales, zeros, g_idx))
+    X = rng.standard_normal((3, k)).astype(np.float16)
+    Y = O.dequant_matmul(X, qw, scales, zeros, g_idx, bits, k)
+    for t in range(3):
+        for j in range(n):
+            acc = 0.0
+            for c in range(k):
+                g = int(g_idx[c])
+                acc += float(X[t, c]) * float(scales[j, g]) * (int(codes[j, c]) - int(zeros[j, g]))
+            assert abs(acc - Y[t, j]) <= 1e-12 * max(1.0, abs(acc))
+
+
+@pytest.mark.parametrize("act,static", [(False, False), (True, False), (True, True)])
+def test_dequant_matmul_of_gptq_output_equals_sweep_weights(act, static):
+    # The packed output of a GPTQ run, multiplied through the inference
+    # product, gives X Qhat^T with the sweep's own dequantized weights (a
+    # different route: the sweep's scale * (code - zero) at quantization time).
+    W, Z, H = _rand_layer(41, 12, 128)
+    res = O.gptq(W, H, 4, 32, 32, 0.01, act, static_groups=static)
+    qw = O.pack(res["codes"], 4)
+    X = Z[:7].astype(np.float16).astype(np.float64)
+    Y = O.dequant_matmul(X, qw, res["scales"], res["zeros"].astype(np.int64), res["g_idx"], 4, 128)
+    assert np.allclose(Y, X @ res["qhat"].T, rtol=1e-13, atol=1e-15)
