@@ -396,6 +396,8 @@ def native_arm(args, spec, world, rank, local):
         "gpu_launches": launches * args.steps if launches is not None else None,
         "gpu_launches_per_step": launches, "clocks": clk, "e2e": e2e,
     }
+    if not args.no_qgemm:
+        line["inference_matmul"] = qgemm_measure(dev, stream, peaks, args.seed + rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_full, wall, sample = oracle_sample(spec, args.seed, args.ref_tokens, args.ref_rows)
         line["cpu_baseline"] = {"value": spec.r * spec.k / t_full / 1e6, "unit": UNIT,
@@ -404,6 +406,82 @@ def native_arm(args, spec, world, rank, local):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+# Linear layers of one Llama-2-7B-shaped block, (out-features n, in-features k)
+QG_BLOCK = [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]
+QG_BLOCKS = 4  # 4 blocks: 405 MB of int4 weights, more than L2
+
+
+def qgemm_measure(dev, stream, peaks, seed, bits=4, G=128, reps=20):
+    """The inference product (gptq_gemm) on one decode token (m = 1) through
+    the linear layers of QG_BLOCKS blocks of a 7B-shaped model, int4 g128,
+    synthetic packed weights resident in HBM; the 28 calls are one CUDA
+    graph, timed with events.  Algorithmic bytes: packed weights + fp32 scales
+    + int32 zeros + X + Y of every layer.  Also m = 16 (a small batch) and
+    m = 2048 (prefill, the tensor-core kernel, against the dense bf16 peak;
+    f16 has the same nominal rate)."""
+    from post_weight_quantization_23_b200 import quant_matmul
+    g = torch.Generator(device=dev).manual_seed(seed)
+    layers = []
+    for _ in range(QG_BLOCKS):
+        for n, k in QG_BLOCK:
+            ng = k // G
+            qw = torch.randint(-2 ** 31, 2 ** 31 - 1, (n, k * bits // 32), generator=g,
+                               dtype=torch.int32, device=dev)
+            sc = torch.rand(n, ng, generator=g, device=dev) * 0.01 + 1e-3
+            z = torch.randint(0, 2 ** bits, (n, ng), generator=g, dtype=torch.int32, device=dev)
+            layers.append((n, k, qw, sc, z))
+    out = {"workload": (f"one token through the linear layers of {QG_BLOCKS} Llama-2-7B-shaped "
+                        f"blocks ({len(layers)} layers: 4x 4096x4096, 2x 11008x4096, "
+                        f"1x 4096x11008 per block), int{bits} g{G}, f16 activations"),
+           "l2": "weights larger than L2, each layer read once per pass", "bound": "hbm",
+           "peak": peaks["hbm"], "unit": "GB/s", "kernel": "qgemv_kernel (gptq_gemm)"}
+    for m in (1, 16, 2048):
+        xs = [torch.randn(m, k, generator=g, device=dev).half() for (_, k, *_r) in layers]
+        ys = [torch.empty(m, n, dtype=torch.float16, device=dev) for (n, *_r) in layers]
+
+        def run():
+            for (n, k, qw, sc, z), x, y in zip(layers, xs, ys):
+                quant_matmul(x, qw, sc, z, bits, G, None, y)
+
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize(dev)
+        s2 = torch.cuda.Stream(dev)
+        s2.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s2):
+            run()
+        torch.cuda.synchronize(dev)
+        for _ in range(3):
+            graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        nbytes = sum(n * k * bits // 8 + n * (k // G) * 8 + m * k * 2 + m * n * 2
+                     for (n, k, *_r) in layers)
+        gbs = nbytes / (us / 1e6) / 1e9
+        tag = f"m{m}"
+        out[f"{tag}_us_per_pass"] = us
+        if m >= 17:  # the tensor-core kernel: bound by the multiply
+            flop = 2.0 * m * sum(n * k for (n, k, *_r) in layers)
+            out[f"{tag}_tflops"] = flop / (us / 1e6) / 1e12
+            out[f"{tag}_frac_of_bf16_dense"] = out[f"{tag}_tflops"] / peaks["bf16"]
+        else:
+            out[f"{tag}_bytes_per_pass"] = nbytes
+            out[f"{tag}_achieved_gbs"] = gbs
+            out[f"{tag}_frac"] = gbs / peaks["hbm"]
+        del graph, xs, ys
+    out["achieved"] = out["m1_achieved_gbs"]
+    out["frac"] = out["m1_frac"]
+    out["launches_per_pass"] = len(layers)
+    return out
 
 
 def sweep_model_bytes(spec):
@@ -476,6 +554,8 @@ def main():
     ap.add_argument("--rows", type=int, default=None, help="override the row count of W")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per Hessian launch from an ncu capture of this kernel")
+    ap.add_argument("--no-qgemm", action="store_true",
+                    help="skip the inference-product measurement")
     ap.add_argument("--act-order", action="store_true", help="variant: act-order")
     ap.add_argument("--sym", action="store_true", help="variant: symmetric grid")
     ap.add_argument("--static-groups", action="store_true", help="variant: static groups")

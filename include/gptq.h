@@ -242,6 +242,33 @@ GPTQ_API gptq_status gptq_dequant(const int32_t* qweight, const float* scales, c
                          int64_t ngroups, gptq_dtype out_dt, void* out,
                          gptq_stream_t stream);
 
+/* The inference product of a quantized layer, read straight from the packed
+ * codes ("GPTQ", ozercemkelahmet.com/tools/gptq: What the output looks like --
+ * a GPU kernel reads the packed data and dequantizes inside the matrix
+ * multiply; How it works, Step 8; "What Is GPTQ?", ai-tldr.dev, How it works:
+ * each group is expanded just in time):
+ *   Y[t, j] = sum_c X[t, c] * scales[j, g] * (code[j, c] - zeros[j, g]),
+ *   g = g_idx[c], or c / group_size when g_idx is NULL,
+ * summed in fp32 and rounded once to dt.
+ *   X       (m, k) f16 or bf16 (dt), row-major, leading dimension ldx >= k.
+ *   qweight int32 (n, k*bits/32) as written by gptq_pack; n = rows of W
+ *           (output features).  k % 32 == 0.
+ *   scales  fp32 (n, ngroups); zeros int32 (n, ngroups).
+ *   g_idx   int32[k] with 0 <= g_idx[c] < ngroups (an entry outside makes the
+ *           affected outputs NaN), or NULL: then group_size (-1 = one group)
+ *           defines the groups and ngroups must be ceil(k / group_size).
+ *   Y       (m, n) out, dt, row-major, leading dimension ldy >= n.
+ *   m <= 131070 tokens.  The library allocates nothing.
+ * With g_idx NULL, bits 2/4/8 and group_size a multiple of 128/bits (or one
+ * group per row), the decode kernel runs (weights streamed once per 2 tokens,
+ * each product exact in fp32); every other case runs the general kernel.
+ * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_UNSUPPORTED (bits, f32 X),
+ * GPTQ_ERR_CUDA. */
+GPTQ_API gptq_status gptq_gemm(const void* X, gptq_dtype dt, int64_t m, int64_t k, int64_t ldx,
+                      const int32_t* qweight, const float* scales, const int32_t* zeros,
+                      const int32_t* g_idx, int64_t n, int bits, int group_size,
+                      int64_t ngroups, void* Y, int64_t ldy, gptq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

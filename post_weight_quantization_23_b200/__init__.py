@@ -14,4 +14,4 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     load,
 )
-from .api import GptqPlan, QuantConfig, quantize_layer  # noqa: F401
+from .api import GptqPlan, QuantConfig, quant_matmul, quantize_layer  # noqa: F401

@@ -38,6 +38,7 @@ EXPORTED = (
     "gptq_quantize_layer",
     "gptq_pack",
     "gptq_dequant",
+    "gptq_gemm",
 )
 
 _DTYPES = {torch.float32: GPTQ_F32, torch.float16: GPTQ_F16, torch.bfloat16: GPTQ_BF16}
@@ -103,6 +104,9 @@ def load(path: str = LIB_PATH):
     lib.gptq_pack.argtypes = [vp, i64, i64, i32, vp, vp]
     lib.gptq_dequant.restype = i32
     lib.gptq_dequant.argtypes = [vp, vp, vp, vp, i64, i64, i32, i64, i32, vp, vp]
+    lib.gptq_gemm.restype = i32
+    lib.gptq_gemm.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, i64, i32, i32, i64, vp, i64,
+                              vp]
     _lib = lib
     return lib
 
@@ -195,3 +199,16 @@ def dequant(qweight, scales, zeros, g_idx, k, bits, out, stream=None):
     st = load().gptq_dequant(_ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(g_idx), r, k, int(bits),
                              scales.shape[1], dtype_code(out.dtype), _ptr(out), _stream(stream))
     _check(st, "gptq_dequant")
+
+
+def gemm(X, qweight, scales, zeros, g_idx, bits, group_size, Y, stream=None):
+    """Y = X W_hat^T from the packed weights (gptq_gemm).  X (m, k) and Y (m, n)
+    f16/bf16 with unit column stride; g_idx None means groups of group_size."""
+    m, k = X.shape
+    n = qweight.shape[0]
+    if X.stride(1) != 1 or Y.stride(1) != 1 or Y.dtype != X.dtype:
+        raise GptqError(GPTQ_ERR_INVALID_ARG, "gptq_gemm", "X, Y: unit column stride, same dtype")
+    st = load().gptq_gemm(_ptr(X), dtype_code(X.dtype), m, k, X.stride(0), _ptr(qweight),
+                          _ptr(scales), _ptr(zeros), _ptr(g_idx), n, int(bits), int(group_size),
+                          scales.shape[1], _ptr(Y), Y.stride(0), _stream(stream))
+    _check(st, "gptq_gemm")

@@ -104,6 +104,14 @@ class GptqPlan:
             _lib.dequant(self.qweight, self.scales, self.zeros, self.g_idx, self.k, self.cfg.bits,
                          self.deq, stream)
 
+    def matmul(self, X: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        """Y = X W_hat^T with this plan's packed weights (after pack()).  The
+        groups are runs of group_size columns unless act-order reordered them
+        with dynamic groups; only then is g_idx passed to the kernel."""
+        g_idx = self.g_idx if (self.cfg.act_order and not self.cfg.static_groups) else None
+        return quant_matmul(X, self.qweight, self.scales, self.zeros, self.cfg.bits,
+                            self.cfg.group_size, g_idx, out, stream)
+
     def run_after_hessian(self, W: torch.Tensor, stream=None):
         """prepare -> quantize -> pack -> dequant, no synchronisation."""
         self.prepare(stream)
@@ -152,6 +160,21 @@ class GptqPlan:
         if self.deq is not None:
             out["deq"] = self.deq
         return out
+
+
+def quant_matmul(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+                 zeros: torch.Tensor, bits: int, group_size: int, g_idx=None,
+                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The inference product Y = X W_hat^T read straight from packed weights
+    (gptq_gemm): X (m, k) f16/bf16 on the device, qweight (n, k*bits/32),
+    scales / zeros (n, ngroups), g_idx (k,) or None for runs of group_size
+    columns.  Returns Y (m, n) in X's dtype (``out`` if given)."""
+    m = X.shape[0]
+    n = qweight.shape[0]
+    if out is None:
+        out = torch.empty(m, n, dtype=X.dtype, device=X.device)
+    _lib.gemm(X, qweight, scales, zeros, g_idx, bits, group_size, out, stream)
+    return out
 
 
 def quantize_layer(W: torch.Tensor, X=None, cfg: QuantConfig | None = None, H=None,

@@ -3,6 +3,8 @@
 // before anything is enqueued.
 #include "common.cuh"
 
+#include <algorithm>
+
 namespace gptq {
 gptq_status hessian_simt(const void* X, gptq_dtype dt, int64_t n, int64_t k, int64_t ldx,
                          float alpha, float* H, cudaStream_t s);
@@ -25,6 +27,10 @@ gptq_status pack_impl(const uint8_t* codes, int64_t r, int64_t k, int bits, int3
 gptq_status dequant_impl(const int32_t* qweight, const float* scales, const int32_t* zeros,
                          const int32_t* g_idx, int64_t r, int64_t k, int bits, int64_t ngroups,
                          gptq_dtype out_dt, void* out, cudaStream_t s);
+gptq_status gemm_impl(const void* X, gptq_dtype dt, int64_t m, int64_t k, int64_t ldx,
+                      const int32_t* qweight, const float* scales, const int32_t* zeros,
+                      const int32_t* g_idx, int64_t n, int bits, int group_size, int64_t ngroups,
+                      void* Y, int64_t ldy, cudaStream_t s);
 }  // namespace gptq
 
 using namespace gptq;
@@ -32,6 +38,7 @@ using namespace gptq;
 namespace {
 
 constexpr int64_t kMaxDim = (int64_t)1 << 20;  // k and r limit (int indexing inside kernels)
+constexpr int64_t kGemmMaxTokens = (int64_t)65535 * 2;  // token pairs on the grid's y axis
 
 bool valid_dtype(gptq_dtype dt) { return dt == GPTQ_F32 || dt == GPTQ_F16 || dt == GPTQ_BF16; }
 
@@ -169,6 +176,30 @@ gptq_status gptq_dequant(const int32_t* qweight, const float* scales, const int3
   if (!aligned(out, dtype_bytes(out_dt))) return GPTQ_ERR_INVALID_ARG;
   return dequant_impl(qweight, scales, zeros, g_idx, r, k, bits, ngroups, out_dt, out,
                       (cudaStream_t)stream);
+}
+
+gptq_status gptq_gemm(const void* X, gptq_dtype dt, int64_t m, int64_t k, int64_t ldx,
+                      const int32_t* qweight, const float* scales, const int32_t* zeros,
+                      const int32_t* g_idx, int64_t n, int bits, int group_size, int64_t ngroups,
+                      void* Y, int64_t ldy, gptq_stream_t stream) {
+  if (!valid_bits(bits)) return GPTQ_ERR_UNSUPPORTED;
+  if (dt == GPTQ_F32) return GPTQ_ERR_UNSUPPORTED;
+  if (!valid_dtype(dt)) return GPTQ_ERR_INVALID_ARG;
+  if (m < 0 || n < 0 || k < 0 || k % 32 != 0 || k > kMaxDim || n > kMaxDim) return GPTQ_ERR_INVALID_ARG;
+  if (m > kGemmMaxTokens) return GPTQ_ERR_INVALID_ARG;
+  if (group_size != -1 && group_size <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (m == 0 || n == 0) return GPTQ_OK;
+  if (ldx < k || ldy < n) return GPTQ_ERR_INVALID_ARG;
+  if (X == nullptr || Y == nullptr || qweight == nullptr || scales == nullptr ||
+      zeros == nullptr || ngroups <= 0)
+    return GPTQ_ERR_INVALID_ARG;
+  if (g_idx == nullptr) {
+    const int64_t G = group_size == -1 ? std::max<int64_t>(k, 1) : group_size;
+    if (ngroups != std::max<int64_t>(cdiv(k, G), 1)) return GPTQ_ERR_INVALID_ARG;
+  }
+  if (!aligned(X, 2) || !aligned(Y, 2) || !aligned(qweight, 4)) return GPTQ_ERR_INVALID_ARG;
+  return gemm_impl(X, dt, m, k, ldx, qweight, scales, zeros, g_idx, n, bits, group_size, ngroups,
+                   Y, ldy, (cudaStream_t)stream);
 }
 
 }  // extern "C"

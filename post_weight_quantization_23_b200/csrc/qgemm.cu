@@ -1,0 +1,324 @@
+// The inference product of a GPTQ-quantized layer, Y = X W_hat^T with
+// W_hat[j, c] = scale[j, g(c)] * (code[j, c] - zero[j, g(c)]), read straight
+// from the packed codes ("GPTQ", ozercemkelahmet.com/tools/gptq: What the
+// output looks like -- a GPU kernel reads the packed data and dequantizes
+// inside the matrix multiply; How it works, Step 8; "What Is GPTQ?",
+// ai-tldr.dev, How it works: each group is expanded just in time).
+//
+// Small token counts (decode) are bound by the bytes of the packed weights,
+// so the decode kernel streams them once with coalesced 16-byte loads and
+// does the arithmetic on the CUDA cores.  Each code c is turned into a float
+// by one logic op: a code sitting at bit b j of a 16-bit half word (b = bits,
+// j = its slot) is kept in place and given the exponent of 2^(23 - b j), which
+// makes the float 2^(23 - b j) + c exactly; subtracting 2^(23 - b j) and the
+// zero point leaves c - zero exactly, so every product x (c - zero) is exact
+// in fp32.  The products are summed in fp32 per 16-byte piece (one group) and
+// multiplied by the group's scale once.
+#include "common.cuh"
+
+#include <type_traits>
+
+namespace gptq {
+
+bool qgemm_tc_supported(const void* X, int64_t ldx, const int32_t* qw, int bits, int64_t k,
+                        int G, bool has_gidx);
+gptq_status qgemm_tc(const void* X, bool bf16, int64_t m, int64_t k, int64_t ldx,
+                     const int32_t* qw, const float* scales, const int32_t* zeros, int64_t n,
+                     int G, int64_t ngroups, void* Y, int64_t ldy, cudaStream_t s);
+
+// Token counts above this use the tensor-core kernel when it applies.
+constexpr int QG_TC_MIN_TOKENS = 17;
+
+namespace {
+
+template <typename T> __device__ __forceinline__ T qg_out(float v);
+template <> __device__ __forceinline__ __half qg_out<__half>(float v) { return __float2half_rn(v); }
+template <> __device__ __forceinline__ __nv_bfloat16 qg_out<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+constexpr int QV_WARPS = 16;   // warps per CTA, each a slice of the columns
+constexpr int QV_ROWS = 32;    // rows of W per CTA: 8 rows per lane, 4 rows per load
+constexpr int QV_KC = 4096;    // columns of X staged in shared memory per pass
+
+template <int BITS>
+struct QvShape {
+  static constexpr int CPW = 32 / BITS;   // codes per 32-bit word
+  static constexpr int HC = CPW / 2;      // codes per 16-bit half word
+  static constexpr int CH = 4 * CPW;      // columns per 16-byte piece
+  static constexpr int SLAB = 8 * CH;     // columns one warp covers per step (8 lanes per row)
+  static constexpr int PAD = 4;           // floats of padding after every CH staged columns
+  static constexpr uint32_t MASK = (1u << BITS) - 1u;
+};
+
+inline int qv_kc(int k, int slab) {
+  const int kc = k < QV_KC ? k : QV_KC;
+  return (int)(cdiv(kc, slab) * slab);
+}
+
+template <int BITS>
+inline size_t qv_smem_bytes(int M, int KC) {
+  using Sh = QvShape<BITS>;
+  const int XS = KC + Sh::PAD * (KC / Sh::CH);
+  return sizeof(float) * ((size_t)M * XS + (size_t)QV_WARPS * M * 32);
+}
+
+// Decode kernel: CTA = 32 rows x M tokens, 16 warps splitting the columns.
+// Lane (q = lane / 8, p = lane % 8) loads, for i = 0..7, the 16-byte piece p
+// of row 4 i + q in the warp's current slab, so each load instruction reads
+// four whole 128-byte row segments.  Needs k % CH == 0 and a group size that
+// is a multiple of CH (or one group per row), so a piece lies in one group.
+template <int BITS, int M, typename T>
+__global__ void __launch_bounds__(QV_WARPS * 32)
+qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
+             const int32_t* __restrict__ qw, const float* __restrict__ scales,
+             const int32_t* __restrict__ zeros, int n, int G, int ngroups, int KC,
+             T* __restrict__ Y, int64_t ldy) {
+  using Sh = QvShape<BITS>;
+  extern __shared__ __align__(16) float qv_smem[];
+  const int XS = KC + Sh::PAD * (KC / Sh::CH);
+  float* xs = qv_smem;            // [M][XS] staged activations (fp32)
+  float* red = xs + M * XS;       // [QV_WARPS][M][32] per-warp row sums
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q = lane >> 3, p = lane & 7;
+  const int r0 = blockIdx.x * QV_ROWS;
+  const int t0 = blockIdx.y * M;
+  const int64_t wpr = (int64_t)k / Sh::CPW;  // words per row
+
+  float y[8][M];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int t = 0; t < M; ++t) y[i][t] = 0.f;
+
+  for (int kc0 = 0; kc0 < k; kc0 += KC) {
+    const int kcw = min(KC, k - kc0);
+    __syncthreads();  // the previous pass is done with xs
+    for (int e = tid; e < M * kcw; e += blockDim.x) {
+      const int t = e / kcw, c = e - t * kcw;
+      float v = 0.f;
+      if (t0 + t < m) v = to_f32(X[(int64_t)(t0 + t) * ldx + kc0 + c]);
+      xs[t * XS + c + Sh::PAD * (c / Sh::CH)] = v;
+    }
+    __syncthreads();
+    for (int sl = warp * Sh::SLAB; sl < kcw; sl += QV_WARPS * Sh::SLAB) {
+      const int cl = sl + p * Sh::CH;  // this lane's piece, local column
+      const bool have = cl < kcw;
+      const int g = (kc0 + cl) / G;
+      uint4 d[8];
+      float sc[8];
+      int zc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = r0 + 4 * i + q;
+        const bool ok = have && row < n;
+        d[i] = ok ? ld_stream_u4(qw + (int64_t)row * wpr + (kc0 + cl) / Sh::CPW)
+                  : make_uint4(0u, 0u, 0u, 0u);
+        sc[i] = ok ? scales[(int64_t)row * ngroups + g] : 0.f;
+        zc[i] = ok ? zeros[(int64_t)row * ngroups + g] : 0;
+      }
+      // lanes past the chunk's end have zero words and scale 0; they read
+      // (and discard) the chunk's first columns instead of past the buffer
+      const int clx = have ? cl : 0;
+      const float* xb = xs + clx + Sh::PAD * (clx / Sh::CH);
+      float nz[8];  // -zero of each row
+#pragma unroll
+      for (int i = 0; i < 8; ++i) nz[i] = -(float)zc[i];
+      float2 acc[8][M];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int t = 0; t < M; ++t) acc[i][t] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int j = 0; j < Sh::HC; j += 2) {
+            // the activations of codes j, j + 1 of this half word, for every token
+            const int col = wi * Sh::CPW + h * Sh::HC + j;
+            float2 x2[M];
+#pragma unroll
+            for (int t = 0; t < M; ++t) x2[t] = *reinterpret_cast<const float2*>(xb + t * XS + col);
+            // -2^(23 - b j) for the two slots (compile-time constants)
+            const float2 nmag = make_float2(-(float)(1 << (23 - BITS * j)),
+                                            -(float)(1 << (23 - BITS * (j + 1))));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t word = wi == 0 ? d[i].x : wi == 1 ? d[i].y : wi == 2 ? d[i].z : d[i].w;
+              const uint32_t hw = h ? (word >> 16) : word;
+              // 2^(23 - b j) + c, exactly
+              const float f0 = __uint_as_float((0x4B000000u - ((uint32_t)(BITS * j) << 23)) |
+                                               (hw & (Sh::MASK << (BITS * j))));
+              const float f1 = __uint_as_float((0x4B000000u - ((uint32_t)(BITS * (j + 1)) << 23)) |
+                                               (hw & (Sh::MASK << (BITS * (j + 1)))));
+              const float2 one = make_float2(1.f, 1.f);
+              const float2 c2 = __ffma2_rn(make_float2(f0, f1), one, nmag);            // c, exact
+              const float2 dd = __ffma2_rn(c2, one, make_float2(nz[i], nz[i]));        // c - zero
+#pragma unroll
+              for (int t = 0; t < M; ++t) acc[i][t] = __ffma2_rn(x2[t], dd, acc[i][t]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int t = 0; t < M; ++t) y[i][t] = fmaf(sc[i], acc[i][t].x + acc[i][t].y, y[i][t]);
+    }
+  }
+  // sum the 8 pieces of each row, then the 16 warps
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int t = 0; t < M; ++t) {
+      float v = y[i][t];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      y[i][t] = v;
+    }
+  if (p == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int t = 0; t < M; ++t) red[(warp * M + t) * 32 + 4 * i + q] = y[i][t];
+  }
+  __syncthreads();
+  for (int e = tid; e < M * 32; e += blockDim.x) {
+    const int t = e / 32, rr = e % 32;
+    float v = 0.f;
+#pragma unroll 4
+    for (int w = 0; w < QV_WARPS; ++w) v += red[(w * M + t) * 32 + rr];
+    if (t0 + t < m && r0 + rr < n) Y[(int64_t)(t0 + t) * ldy + r0 + rr] = qg_out<T>(v);
+  }
+}
+
+// General kernel: any bit width (3-bit codes straddle words), any g_idx, any
+// group size.  One warp per (row, 8 tokens); lanes stride over the columns;
+// W_hat = scale * (code - zero) in fp32 per element.  A g_idx entry outside
+// [0, ngroups) is not read through: it makes the row's outputs NaN.
+template <typename T>
+__global__ void __launch_bounds__(256)
+qgemm_general_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
+                     const int32_t* __restrict__ qw, int bits, const float* __restrict__ scales,
+                     const int32_t* __restrict__ zeros, const int32_t* __restrict__ g_idx, int G,
+                     int ngroups, int n, T* __restrict__ Y, int64_t ldy) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int t0 = blockIdx.y * 8;
+  if (row >= n) return;
+  const int64_t wpr = (int64_t)k * bits / 32;
+  const uint32_t* wr = reinterpret_cast<const uint32_t*>(qw) + (int64_t)row * wpr;
+  const uint32_t mask = (1u << bits) - 1u;
+  float acc[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+  bool bad = false;
+  for (int c = lane; c < k; c += 32) {
+    const int64_t bit = (int64_t)c * bits;
+    const int64_t w = bit >> 5;
+    const int sh = (int)(bit & 31);
+    uint32_t v = wr[w] >> sh;
+    if (sh + bits > 32) v |= wr[w + 1] << (32 - sh);
+    const int code = (int)(v & mask);
+    const int g = g_idx != nullptr ? g_idx[c] : c / G;
+    if (g < 0 || g >= ngroups) {
+      bad = true;
+      continue;
+    }
+    const float wv = scales[(int64_t)row * ngroups + g] *
+                     (float)(code - zeros[(int64_t)row * ngroups + g]);
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      if (t0 + t < m) acc[t] = fmaf(to_f32(X[(int64_t)(t0 + t) * ldx + c]), wv, acc[t]);
+  }
+  bad = __any_sync(0xffffffffu, bad);
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    float v = acc[t];
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0 && t0 + t < m)
+      Y[(int64_t)(t0 + t) * ldy + row] = qg_out<T>(bad ? __int_as_float(0x7fc00000) : v);
+  }
+}
+
+template <int BITS, int M, typename T>
+gptq_status launch_qgemv(const T* X, int64_t ldx, int m, int k, const int32_t* qw,
+                         const float* scales, const int32_t* zeros, int n, int G, int ngroups,
+                         T* Y, int64_t ldy, cudaStream_t s) {
+  using Sh = QvShape<BITS>;
+  const int KC = qv_kc(k, Sh::SLAB);
+  const size_t smem = qv_smem_bytes<BITS>(M, KC);
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(qgemv_kernel<BITS, M, T>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return GPTQ_ERR_CUDA;
+  }
+  const dim3 grid((unsigned)cdiv(n, QV_ROWS), (unsigned)cdiv(m, M));
+  qgemv_kernel<BITS, M, T><<<grid, QV_WARPS * 32, smem, s>>>(X, ldx, m, k, qw, scales, zeros, n,
+                                                             G, ngroups, KC, Y, ldy);
+  GPTQ_CHECK_LAUNCH();
+  return GPTQ_OK;
+}
+
+template <int BITS, typename T>
+gptq_status qgemv_bits(const T* X, int64_t ldx, int m, int k, const int32_t* qw,
+                       const float* scales, const int32_t* zeros, int n, int G, int ngroups, T* Y,
+                       int64_t ldy, cudaStream_t s) {
+  // one token, or pairs of tokens on the grid's y axis (later pairs re-read
+  // the packed weights, mostly from L2)
+  if (m == 1) return launch_qgemv<BITS, 1, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
+  return launch_qgemv<BITS, 2, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
+}
+
+template <typename T>
+gptq_status qgemm_typed(const T* X, int64_t ldx, int m, int k, const int32_t* qw,
+                        const float* scales, const int32_t* zeros, const int32_t* g_idx, int n,
+                        int bits, int G, int ngroups, T* Y, int64_t ldy, cudaStream_t s) {
+  const bool pow2 = bits == 2 || bits == 4 || bits == 8;
+  if (m >= QG_TC_MIN_TOKENS && k > 0 &&
+      qgemm_tc_supported(X, ldx, qw, bits, k, G, g_idx != nullptr))
+    return qgemm_tc(X, std::is_same<T, __nv_bfloat16>::value, m, k, ldx, qw, scales, zeros, n, G,
+                    ngroups, Y, ldy, s);
+  if (pow2 && g_idx == nullptr && ((uintptr_t)qw % 16) == 0 && k > 0) {
+    const int CH = 4 * (32 / bits);
+    if (k % CH == 0 && (G >= k || G % CH == 0)) {
+      switch (bits) {
+        case 2: return qgemv_bits<2, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
+        case 4: return qgemv_bits<4, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
+        default: return qgemv_bits<8, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
+      }
+    }
+  }
+  const dim3 grid((unsigned)cdiv(n, 8), (unsigned)cdiv(m, 8));
+  qgemm_general_kernel<T><<<grid, 256, 0, s>>>(X, ldx, m, k, qw, bits, scales, zeros, g_idx, G,
+                                               ngroups, n, Y, ldy);
+  GPTQ_CHECK_LAUNCH();
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+gptq_status gemm_impl(const void* X, gptq_dtype dt, int64_t m, int64_t k, int64_t ldx,
+                      const int32_t* qweight, const float* scales, const int32_t* zeros,
+                      const int32_t* g_idx, int64_t n, int bits, int group_size, int64_t ngroups,
+                      void* Y, int64_t ldy, cudaStream_t s) {
+  const int G = group_size == -1 ? (int)k : group_size;
+  if (dt == GPTQ_F16)
+    return qgemm_typed<__half>((const __half*)X, ldx, (int)m, (int)k, qweight, scales, zeros,
+                               g_idx, (int)n, bits, G, (int)ngroups, (__half*)Y, ldy, s);
+  return qgemm_typed<__nv_bfloat16>((const __nv_bfloat16*)X, ldx, (int)m, (int)k, qweight, scales,
+                                    zeros, g_idx, (int)n, bits, G, (int)ngroups,
+                                    (__nv_bfloat16*)Y, ldy, s);
+}
+
+}  // namespace gptq

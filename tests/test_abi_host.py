@@ -98,6 +98,29 @@ def test_host_argument_checks(lib):
     assert q(static_g96, ws=None) == _lib.GPTQ_ERR_WORKSPACE
 
 
+def test_gemm_host_checks(lib):
+    fake = ctypes.c_void_p(256)  # never dereferenced: every call below fails a host check
+    F16, F32, BF16 = _lib.GPTQ_F16, _lib.GPTQ_F32, _lib.GPTQ_BF16
+
+    def g(dt=F16, m=2, k=256, ldx=256, bits=4, gs=128, ng=2, gidx=None, n=8, ldy=8, X=fake):
+        return lib.gptq_gemm(X, dt, m, k, ldx, fake, fake, fake, gidx, n, bits, gs, ng, fake,
+                             ldy, None)
+
+    assert g(bits=5) == _lib.GPTQ_ERR_UNSUPPORTED
+    assert g(dt=F32) == _lib.GPTQ_ERR_UNSUPPORTED
+    assert g(dt=9) == _lib.GPTQ_ERR_INVALID_ARG
+    assert g(k=250, ldx=250) == _lib.GPTQ_ERR_INVALID_ARG          # k % 32
+    assert g(m=0) == _lib.GPTQ_OK and g(n=0) == _lib.GPTQ_OK       # empty: no-op
+    assert g(ldx=128) == _lib.GPTQ_ERR_INVALID_ARG                 # ldx < k
+    assert g(ldy=4) == _lib.GPTQ_ERR_INVALID_ARG                   # ldy < n
+    assert g(ng=3) == _lib.GPTQ_ERR_INVALID_ARG                    # ngroups != ceil(k / G)
+    assert g(gs=0) == _lib.GPTQ_ERR_INVALID_ARG
+    assert g(gs=-1, ng=2) == _lib.GPTQ_ERR_INVALID_ARG             # one group per row
+    assert g(X=None) == _lib.GPTQ_ERR_INVALID_ARG
+    assert g(m=131071) == _lib.GPTQ_ERR_INVALID_ARG                # token limit
+    assert g(X=ctypes.c_void_p(257)) == _lib.GPTQ_ERR_INVALID_ARG  # misaligned X
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(P.GptqError):
