@@ -48,6 +48,8 @@ from .gptq_oracle import (  # noqa: F401
     unpack,
     dequant,
     dequant_matmul,
+    rotation_matrix,
+    rotate,
     storage_bits_per_weight,
     group_count,
 )

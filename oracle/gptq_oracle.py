@@ -52,6 +52,13 @@ R15 Static groups (the ``static_groups`` flag of the AutoGPTQ configuration
     and each column is quantized on that group's grid when its turn comes.
     Because no grid depends on the sweep, groups need not align with the
     lazy blocks (READING R10 is not needed).
+R16 Rotation preprocessing ([GPTQ-tool] *Variants and extensions*: weights
+    and activations are multiplied by an orthogonal matrix before quantizing
+    so that outliers spread out; the matrix is not named): Q = D_s H_b / sqrt(b),
+    D_s = diag(s) with random signs s (an input), H_b the block-diagonal
+    Sylvester-Hadamard matrix with blocks of b columns (b a power of two
+    dividing k).  W' = W Q and X' = X Q keep X W^T = X' W'^T, and the
+    Hessian of X' is Q^T H Q.
 """
 
 from __future__ import annotations
@@ -644,6 +651,29 @@ def dequant(codes, scales, zeros, g_idx, out_dtype=F32):
     z = np.asarray(zeros, dtype=np.int64)[:, g_idx]
     v = s * (codes - z).astype(F32)
     return v.astype(out_dtype)
+
+
+def rotation_matrix(signs, block):
+    """READING R16: Q = diag(signs) * blockdiag(H_b, ..., H_b) / sqrt(b), with
+    H_b the Sylvester Hadamard matrix of order b (scipy.linalg.hadamard).
+    Orthogonal: Q Q^T = I."""
+    from scipy.linalg import block_diag, hadamard
+    s = np.where(np.asarray(signs) < 0, -1.0, 1.0)
+    k = s.shape[0]
+    b = int(block)
+    if b <= 0 or b & (b - 1) or k % b:
+        raise ValueError("block must be a power of two dividing k")
+    Hb = hadamard(b).astype(F64) / math.sqrt(b)
+    return s[:, None] * block_diag(*([Hb] * (k // b)))
+
+
+def rotate(x, signs, block, inverse=False):
+    """[GPTQ-tool] *Variants and extensions*, rotation-based preprocessing
+    (READING R16): each row x of ``x`` becomes x Q (``inverse``: x Q^T, which
+    undoes it).  fp64."""
+    Q = rotation_matrix(signs, block)
+    x = np.asarray(x, dtype=F64)
+    return x @ (Q.T if inverse else Q)
 
 
 def dequant_matmul(X, qweight, scales, zeros, g_idx, bits, k):

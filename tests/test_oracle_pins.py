@@ -715,3 +715,48 @@ def test_dequant_matmul_of_gptq_output_equals_sweep_weights(act, static):
     X = Z[:7].astype(np.float16).astype(np.float64)
     Y = O.dequant_matmul(X, qw, res["scales"], res["zeros"].astype(np.int64), res["g_idx"], 4, 128)
     assert np.allclose(Y, X @ res["qhat"].T, rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- rotation (R16)
+
+def test_rotation_worked_values_and_outlier_spread():
+    # b = 4, all signs +1: e_0 Q is the first row of H_4 / 2 = [1, 1, 1, 1] / 2;
+    # e_1 Q = [1, -1, 1, -1] / 2.  One outlier of size A spreads to A / sqrt(b)
+    # in every coordinate ("GPTQ", Variants and extensions: outliers spread out).
+    s = np.ones(4)
+    assert O.rotate(np.eye(4)[:2], s, 4).tolist() == [[0.5, 0.5, 0.5, 0.5],
+                                                      [0.5, -0.5, 0.5, -0.5]]
+    x = np.zeros((1, 256))
+    x[0, 37] = 100.0
+    y = O.rotate(x, np.random.default_rng(0).choice([-1, 1], 256), 256)
+    assert np.allclose(np.abs(y), 100.0 / 16.0)
+
+
+@pytest.mark.parametrize("k,b", [(256, 256), (768, 256), (1024, 512), (4096, 4096)])
+def test_rotation_is_orthogonal_and_keeps_the_layer_function(k, b):
+    rng = np.random.default_rng(k + b)
+    s = rng.choice([-1, 1], k)
+    Q = O.rotation_matrix(s, b)
+    assert np.allclose(Q @ Q.T, np.eye(k), atol=1e-12)
+    X = rng.standard_normal((6, k))
+    W = rng.standard_normal((5, k))
+    Xr, Wr = O.rotate(X, s, b), O.rotate(W, s, b)
+    assert np.allclose(Xr @ Wr.T, X @ W.T, atol=1e-10)           # X W^T = X' W'^T
+    assert np.allclose(O.rotate(Xr, s, b, inverse=True), X, atol=1e-12)
+    assert np.allclose(O.hessian(Xr), Q.T @ O.hessian(X) @ Q, atol=1e-10)
+    # a sign flip or a missing 1/sqrt(b) would break these; so would H_b^T != H_b
+    assert not np.allclose(O.rotate(X, -s, b), Xr)
+
+
+def test_gptq_in_the_rotated_basis_measures_the_same_loss():
+    # Quantizing W' = W Q against H' = Q^T H Q and rotating the result back
+    # (Q_hat = Q_hat' Q^T) gives the same layer loss in the original basis:
+    # tr((W - Q_hat) H (W - Q_hat)^T) = tr((W' - Q_hat') H' (W' - Q_hat')^T).
+    W, Z, H = _rand_layer(51, 8, 256)
+    s = np.random.default_rng(3).choice([-1, 1], 256)
+    Hr = O.rotate(O.rotate(H, s, 256).T, s, 256).T  # Q^T H Q
+    assert np.allclose(Hr, O.hessian(O.rotate(Z, s, 256)), atol=1e-10)
+    res = O.gptq(O.rotate(W, s, 256), Hr, 4, 64, 64, 0.01)
+    back = O.rotate(res["qhat"], s, 256, inverse=True)
+    loss, _ = O.layer_loss(W, back, H)
+    assert abs(loss - res["loss"]) <= 1e-9 * res["loss"]
