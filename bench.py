@@ -398,6 +398,8 @@ def native_arm(args, spec, world, rank, local):
     }
     if not args.no_qgemm:
         line["inference_matmul"] = qgemm_measure(dev, stream, peaks, args.seed + rank)
+    if not args.no_rotation:
+        line["rotation"] = rotation_measure(Xd, dev, stream, peaks, args.seed + rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_full, wall, sample = oracle_sample(spec, args.seed, args.ref_tokens, args.ref_rows)
         line["cpu_baseline"] = {"value": spec.r * spec.k / t_full / 1e6, "unit": UNIT,
@@ -484,6 +486,37 @@ def qgemm_measure(dev, stream, peaks, seed, bits=4, G=128, reps=20):
     return out
 
 
+def rotation_measure(Xd, dev, stream, peaks, seed, reps=10):
+    """Rotation preprocessing (gptq_rotate) of the whole calibration matrix X
+    (n x k, resident in HBM) into a second buffer: algorithmic bytes = X read
+    + X written + the signs, per launch; events around `reps` launches (each
+    launch streams 2 x |X|, more than L2)."""
+    from post_weight_quantization_23_b200 import hadamard_block, rotate, rotation_signs
+    n, k = Xd.shape
+    block = hadamard_block(k)
+    if block == 0:
+        return None
+    signs = rotation_signs(k, seed, dev)
+    out = torch.empty_like(Xd)
+    for _ in range(3):
+        rotate(Xd, signs, block, out=out)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(reps):
+        rotate(Xd, signs, block, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    nbytes = 2 * Xd.numel() * Xd.element_size() + k
+    gbs = nbytes / (us / 1e6) / 1e9
+    del out
+    return {"workload": f"X {n}x{k} {str(Xd.dtype)[6:]} rotated by diag(s) H_{block} / sqrt({block})",
+            "kernel": "rotate_kernel (gptq_rotate)", "bound": "hbm", "us_per_launch": us,
+            "bytes_per_launch": nbytes, "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm"]}
+
+
 def sweep_model_bytes(spec):
     """Algorithmic bytes of the lazy-blocked sweep: per block the trailing fp32
     slice of W in and out (8 r (k-e)), the U panel (4 B (k-e)), plus the W
@@ -556,6 +589,10 @@ def main():
                     help="DRAM bytes per Hessian launch from an ncu capture of this kernel")
     ap.add_argument("--no-qgemm", action="store_true",
                     help="skip the inference-product measurement")
+    ap.add_argument("--no-rotation", action="store_true",
+                    help="skip the rotation-preprocessing measurement")
+    ap.add_argument("--only", choices=["inference", "rotation"], default=None,
+                    help="run one side measurement alone (a short command for profiling)")
     ap.add_argument("--act-order", action="store_true", help="variant: act-order")
     ap.add_argument("--sym", action="store_true", help="variant: symmetric grid")
     ap.add_argument("--static-groups", action="store_true", help="variant: static groups")
@@ -572,6 +609,16 @@ def main():
         # CPU only: rank 0 runs the oracle, other ranks exit without work
         return reference_arm(args, spec, int(os.environ.get("WORLD_SIZE", "1")),
                              int(os.environ.get("RANK", "0")))
+    if args.only is not None:
+        dev = torch.device("cuda", 0)
+        stream = torch.cuda.current_stream(dev)
+        if args.only == "inference":
+            out = qgemm_measure(dev, stream, _peaks(), args.seed, reps=args.steps)
+        else:
+            X = synth.make_x(spec, args.seed).to(dev)
+            out = rotation_measure(X, dev, stream, _peaks(), args.seed)
+        print(json.dumps({"only": args.only, **out}), flush=True)
+        return 0
     world, rank, local = dist_setup(args)
     try:
         return native_arm(args, spec, world, rank, local)

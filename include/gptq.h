@@ -269,6 +269,26 @@ GPTQ_API gptq_status gptq_gemm(const void* X, gptq_dtype dt, int64_t m, int64_t 
                       const int32_t* g_idx, int64_t n, int bits, int group_size,
                       int64_t ngroups, void* Y, int64_t ldy, gptq_stream_t stream);
 
+/* Rotation preprocessing ("GPTQ", ozercemkelahmet.com/tools/gptq, Variants
+ * and extensions: weights and activations multiplied by an orthogonal matrix
+ * before quantizing so that outliers spread out).  Every row x of `in`
+ * becomes
+ *   x Q = (x * s) H_b / sqrt(b),  or with inverse != 0,  x Q^T = (x H_b / sqrt(b)) * s,
+ * Q = diag(s) H_b / sqrt(b) orthogonal, s[c] = -1 where signs[c] < 0 and +1
+ * elsewhere, H_b the block-diagonal Sylvester Hadamard matrix of order b
+ * (block).  Rotating W (r, k) and X (n, k) alike keeps X W^T; the Hessian of
+ * the rotated X is Q^T H Q.  Arithmetic in fp32, rounded once to dt.
+ *   in, out  (rows, k) dt (F32/F16/BF16), row strides ld_in, ld_out >= k
+ *            (elements; rows 16-byte aligned).  in == out with ld_in ==
+ *            ld_out rotates in place; other overlaps are rejected.
+ *   signs    int8[k] device array, 8-byte aligned.
+ *   block    b: a power of two from 256 to 8192 dividing k (else
+ *            GPTQ_ERR_UNSUPPORTED / GPTQ_ERR_INVALID_ARG).
+ * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_UNSUPPORTED, GPTQ_ERR_CUDA. */
+GPTQ_API gptq_status gptq_rotate(const void* in, gptq_dtype dt, int64_t rows, int64_t k,
+                        int64_t ld_in, const int8_t* signs, int block, int inverse, void* out,
+                        int64_t ld_out, gptq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -14,4 +14,5 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     load,
 )
-from .api import GptqPlan, QuantConfig, quant_matmul, quantize_layer  # noqa: F401
+from .api import (GptqPlan, QuantConfig, hadamard_block, quant_matmul,  # noqa: F401
+                  quantize_layer, rotate, rotation_signs)

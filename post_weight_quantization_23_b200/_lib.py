@@ -39,6 +39,7 @@ EXPORTED = (
     "gptq_pack",
     "gptq_dequant",
     "gptq_gemm",
+    "gptq_rotate",
 )
 
 _DTYPES = {torch.float32: GPTQ_F32, torch.float16: GPTQ_F16, torch.bfloat16: GPTQ_BF16}
@@ -107,6 +108,8 @@ def load(path: str = LIB_PATH):
     lib.gptq_gemm.restype = i32
     lib.gptq_gemm.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, i64, i32, i32, i64, vp, i64,
                               vp]
+    lib.gptq_rotate.restype = i32
+    lib.gptq_rotate.argtypes = [vp, i32, i64, i64, i64, vp, i32, i32, vp, i64, vp]
     _lib = lib
     return lib
 
@@ -212,3 +215,14 @@ def gemm(X, qweight, scales, zeros, g_idx, bits, group_size, Y, stream=None):
                           _ptr(scales), _ptr(zeros), _ptr(g_idx), n, int(bits), int(group_size),
                           scales.shape[1], _ptr(Y), Y.stride(0), _stream(stream))
     _check(st, "gptq_gemm")
+
+
+def rotate(x, signs, block, out, inverse=False, stream=None):
+    """Each row of x (rows, k) times Q (or Q^T when inverse), into out (gptq_rotate)."""
+    rows, k = x.shape
+    if x.stride(1) != 1 or out.stride(1) != 1 or out.dtype != x.dtype or signs.dtype != torch.int8:
+        raise GptqError(GPTQ_ERR_INVALID_ARG, "gptq_rotate", "unit column stride, same dtype, int8 signs")
+    st = load().gptq_rotate(_ptr(x), dtype_code(x.dtype), rows, k, x.stride(0), _ptr(signs),
+                            int(block), int(bool(inverse)), _ptr(out), out.stride(0),
+                            _stream(stream))
+    _check(st, "gptq_rotate")

@@ -177,6 +177,33 @@ def quant_matmul(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
     return out
 
 
+def hadamard_block(k: int, largest: int = 8192) -> int:
+    """The largest power of two that divides k, at most ``largest`` (0 if
+    below 256, which gptq_rotate does not take)."""
+    b = k & -k if k > 0 else 0
+    b = min(b, largest)
+    return b if b >= 256 else 0
+
+
+def rotation_signs(k: int, seed: int, device="cuda") -> torch.Tensor:
+    """Seeded random signs (int8, +1 / -1) for rotate()."""
+    g = torch.Generator().manual_seed(int(seed))
+    s = torch.randint(0, 2, (k,), generator=g, dtype=torch.int8) * 2 - 1
+    return s.to(device)
+
+
+def rotate(x: torch.Tensor, signs: torch.Tensor, block: int | None = None, inverse=False,
+           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Rotation preprocessing (gptq_rotate): each row of x becomes
+    x diag(s) H_b / sqrt(b) (or its inverse).  Apply the same signs and block
+    to W and X before quantizing; ``out`` may be x itself (in place)."""
+    block = block or hadamard_block(x.shape[1])
+    if out is None:
+        out = torch.empty_like(x)
+    _lib.rotate(x, signs, block, out, inverse, stream)
+    return out
+
+
 def quantize_layer(W: torch.Tensor, X=None, cfg: QuantConfig | None = None, H=None,
                    chunk_tokens: int = 65536, want_loss=True, deq_dtype=torch.float16) -> dict:
     """Quantize one layer on the GPU: W (r, k) and either calibration inputs X

@@ -31,6 +31,9 @@ gptq_status gemm_impl(const void* X, gptq_dtype dt, int64_t m, int64_t k, int64_
                       const int32_t* qweight, const float* scales, const int32_t* zeros,
                       const int32_t* g_idx, int64_t n, int bits, int group_size, int64_t ngroups,
                       void* Y, int64_t ldy, cudaStream_t s);
+gptq_status rotate_impl(const void* in, gptq_dtype dt, int64_t rows, int64_t k, int64_t ld_in,
+                        const int8_t* signs, int block, int inverse, void* out, int64_t ld_out,
+                        cudaStream_t s);
 }  // namespace gptq
 
 using namespace gptq;
@@ -200,6 +203,30 @@ gptq_status gptq_gemm(const void* X, gptq_dtype dt, int64_t m, int64_t k, int64_
   if (!aligned(X, 2) || !aligned(Y, 2) || !aligned(qweight, 4)) return GPTQ_ERR_INVALID_ARG;
   return gemm_impl(X, dt, m, k, ldx, qweight, scales, zeros, g_idx, n, bits, group_size, ngroups,
                    Y, ldy, (cudaStream_t)stream);
+}
+
+gptq_status gptq_rotate(const void* in, gptq_dtype dt, int64_t rows, int64_t k, int64_t ld_in,
+                        const int8_t* signs, int block, int inverse, void* out, int64_t ld_out,
+                        gptq_stream_t stream) {
+  if (!valid_dtype(dt)) return GPTQ_ERR_INVALID_ARG;
+  if (block < 256 || block > 8192 || (block & (block - 1)) != 0) return GPTQ_ERR_UNSUPPORTED;
+  if (rows < 0 || k <= 0 || k % block != 0 || k > kMaxDim) return GPTQ_ERR_INVALID_ARG;
+  if (rows == 0) return GPTQ_OK;
+  if (in == nullptr || out == nullptr || signs == nullptr) return GPTQ_ERR_INVALID_ARG;
+  if (ld_in < k || ld_out < k) return GPTQ_ERR_INVALID_ARG;
+  const size_t es = dtype_bytes(dt);
+  if (!aligned(in, 16) || !aligned(out, 16) || !aligned(signs, 8) ||
+      ((size_t)ld_in * es) % 16 != 0 || ((size_t)ld_out * es) % 16 != 0)
+    return GPTQ_ERR_INVALID_ARG;
+  if (rows * (k / block) > (int64_t)INT32_MAX) return GPTQ_ERR_INVALID_ARG;
+  if (in != out || ld_in != ld_out) {  // distinct buffers must not overlap
+    const char* a = (const char*)in;
+    const char* b = (const char*)out;
+    const size_t na = ((size_t)(rows - 1) * ld_in + k) * es, nb = ((size_t)(rows - 1) * ld_out + k) * es;
+    if (a < b + nb && b < a + na) return GPTQ_ERR_INVALID_ARG;
+  }
+  return rotate_impl(in, dt, rows, k, ld_in, signs, block, inverse != 0, out, ld_out,
+                     (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -45,9 +45,10 @@ __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
   return v;
 }
 
-constexpr int QV_WARPS = 16;   // warps per CTA, each a slice of the columns
-constexpr int QV_ROWS = 32;    // rows of W per CTA: 8 rows per lane, 4 rows per load
-constexpr int QV_KC = 4096;    // columns of X staged in shared memory per pass
+constexpr int QV_WARPS = 8;     // warps per CTA, each a share of the slabs
+constexpr int QV_RPL = 4;       // rows per lane
+constexpr int QV_ROWS = 4 * QV_RPL;  // rows of W per CTA (4 rows per load instruction)
+constexpr int QV_KC = 8192;     // columns of X staged in shared memory per pass
 
 template <int BITS>
 struct QvShape {
@@ -68,14 +69,88 @@ template <int BITS>
 inline size_t qv_smem_bytes(int M, int KC) {
   using Sh = QvShape<BITS>;
   const int XS = KC + Sh::PAD * (KC / Sh::CH);
-  return sizeof(float) * ((size_t)M * XS + (size_t)QV_WARPS * M * 32);
+  return sizeof(float) * ((size_t)M * XS + (size_t)QV_WARPS * M * QV_ROWS);
 }
 
-// Decode kernel: CTA = 32 rows x M tokens, 16 warps splitting the columns.
-// Lane (q = lane / 8, p = lane % 8) loads, for i = 0..7, the 16-byte piece p
-// of row 4 i + q in the warp's current slab, so each load instruction reads
-// four whole 128-byte row segments.  Needs k % CH == 0 and a group size that
-// is a multiple of CH (or one group per row), so a piece lies in one group.
+// One warp-slab of packed words: lane (q, p) holds piece p of rows 4 i + q.
+template <int BITS>
+struct QvSlab {
+  uint4 d[QV_RPL];
+  float sc[QV_RPL];
+  float nz[QV_RPL];  // -zero
+};
+
+template <int BITS>
+__device__ __forceinline__ void qv_load(QvSlab<BITS>& S, const int32_t* __restrict__ qw,
+                                        const float* __restrict__ scales,
+                                        const int32_t* __restrict__ zeros, int64_t wpr, int r0,
+                                        int q, int n, int c, bool have, int G, int ngroups) {
+  using Sh = QvShape<BITS>;
+  const int g = c / G;
+#pragma unroll
+  for (int i = 0; i < QV_RPL; ++i) {
+    const int row = r0 + 4 * i + q;
+    const bool ok = have && row < n;
+    S.d[i] = ok ? ld_stream_u4(qw + (int64_t)row * wpr + c / Sh::CPW) : make_uint4(0u, 0u, 0u, 0u);
+    S.sc[i] = ok ? scales[(int64_t)row * ngroups + g] : 0.f;
+    S.nz[i] = ok ? -(float)zeros[(int64_t)row * ngroups + g] : 0.f;
+  }
+}
+
+// y[i][t] += scale_i * sum over the lane's piece of x_t (code - zero).
+template <int BITS, int M>
+__device__ __forceinline__ void qv_compute(const QvSlab<BITS>& S, const float* xb, int XS,
+                                           float (&y)[QV_RPL][M]) {
+  using Sh = QvShape<BITS>;
+  float2 acc[QV_RPL][M];
+#pragma unroll
+  for (int i = 0; i < QV_RPL; ++i)
+#pragma unroll
+    for (int t = 0; t < M; ++t) acc[i][t] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int j = 0; j < Sh::HC; j += 2) {
+        const int col = wi * Sh::CPW + h * Sh::HC + j;
+        float2 x2[M];
+#pragma unroll
+        for (int t = 0; t < M; ++t) x2[t] = *reinterpret_cast<const float2*>(xb + t * XS + col);
+        // -2^(23 - b j) for the two slots (compile-time constants)
+        const float2 nmag = make_float2(-(float)(1 << (23 - BITS * j)),
+                                        -(float)(1 << (23 - BITS * (j + 1))));
+        const float2 one = make_float2(1.f, 1.f);
+#pragma unroll
+        for (int i = 0; i < QV_RPL; ++i) {
+          const uint32_t word = wi == 0 ? S.d[i].x : wi == 1 ? S.d[i].y : wi == 2 ? S.d[i].z : S.d[i].w;
+          const uint32_t hw = h ? (word >> 16) : word;
+          // 2^(23 - b j) + c, exactly
+          const float f0 = __uint_as_float((0x4B000000u - ((uint32_t)(BITS * j) << 23)) |
+                                           (hw & (Sh::MASK << (BITS * j))));
+          const float f1 = __uint_as_float((0x4B000000u - ((uint32_t)(BITS * (j + 1)) << 23)) |
+                                           (hw & (Sh::MASK << (BITS * (j + 1)))));
+          const float2 c2 = __ffma2_rn(make_float2(f0, f1), one, nmag);                 // c, exact
+          const float2 dd = __ffma2_rn(c2, one, make_float2(S.nz[i], S.nz[i]));        // c - zero
+#pragma unroll
+          for (int t = 0; t < M; ++t) acc[i][t] = __ffma2_rn(x2[t], dd, acc[i][t]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < QV_RPL; ++i)
+#pragma unroll
+    for (int t = 0; t < M; ++t) y[i][t] = fmaf(S.sc[i], acc[i][t].x + acc[i][t].y, y[i][t]);
+}
+
+// Decode kernel: CTA = 16 rows x M tokens, 8 warps sharing the column slabs.
+// Lane (q = lane / 8, p = lane % 8) loads, for i = 0..3, the 16-byte piece p
+// of row 4 i + q in its warp's slab, so each load instruction reads four whole
+// 128-byte row segments.  The first slab's words are requested before the
+// activations are staged, and each next slab's before the current one is
+// computed.  Needs k % CH == 0 and a group size that is a multiple of CH (or
+// one group per row), so a piece lies in one group.
 template <int BITS, int M, typename T>
 __global__ void __launch_bounds__(QV_WARPS * 32)
 qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
@@ -86,21 +161,28 @@ qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
   extern __shared__ __align__(16) float qv_smem[];
   const int XS = KC + Sh::PAD * (KC / Sh::CH);
   float* xs = qv_smem;            // [M][XS] staged activations (fp32)
-  float* red = xs + M * XS;       // [QV_WARPS][M][32] per-warp row sums
+  float* red = xs + M * XS;       // [QV_WARPS][M][QV_ROWS] per-warp row sums
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int q = lane >> 3, p = lane & 7;
   const int r0 = blockIdx.x * QV_ROWS;
   const int t0 = blockIdx.y * M;
   const int64_t wpr = (int64_t)k / Sh::CPW;  // words per row
 
-  float y[8][M];
+  float y[QV_RPL][M];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < QV_RPL; ++i)
 #pragma unroll
     for (int t = 0; t < M; ++t) y[i][t] = 0.f;
 
   for (int kc0 = 0; kc0 < k; kc0 += KC) {
     const int kcw = min(KC, k - kc0);
+    // this warp's first slab of the chunk, requested before the staging
+    int sl = warp * Sh::SLAB;
+    QvSlab<BITS> cur;
+    {
+      const int cl = sl + p * Sh::CH;
+      qv_load<BITS>(cur, qw, scales, zeros, wpr, r0, q, n, kc0 + cl, cl < kcw, G, ngroups);
+    }
     __syncthreads();  // the previous pass is done with xs
     for (int e = tid; e < M * kcw; e += blockDim.x) {
       const int t = e / kcw, c = e - t * kcw;
@@ -109,75 +191,25 @@ qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
       xs[t * XS + c + Sh::PAD * (c / Sh::CH)] = v;
     }
     __syncthreads();
-    for (int sl = warp * Sh::SLAB; sl < kcw; sl += QV_WARPS * Sh::SLAB) {
+    for (; sl < kcw; sl += QV_WARPS * Sh::SLAB) {
       const int cl = sl + p * Sh::CH;  // this lane's piece, local column
       const bool have = cl < kcw;
-      const int g = (kc0 + cl) / G;
-      uint4 d[8];
-      float sc[8];
-      int zc[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int row = r0 + 4 * i + q;
-        const bool ok = have && row < n;
-        d[i] = ok ? ld_stream_u4(qw + (int64_t)row * wpr + (kc0 + cl) / Sh::CPW)
-                  : make_uint4(0u, 0u, 0u, 0u);
-        sc[i] = ok ? scales[(int64_t)row * ngroups + g] : 0.f;
-        zc[i] = ok ? zeros[(int64_t)row * ngroups + g] : 0;
+      QvSlab<BITS> nxt;
+      const int sn = sl + QV_WARPS * Sh::SLAB;
+      if (sn < kcw) {
+        const int cn = sn + p * Sh::CH;
+        qv_load<BITS>(nxt, qw, scales, zeros, wpr, r0, q, n, kc0 + cn, cn < kcw, G, ngroups);
       }
       // lanes past the chunk's end have zero words and scale 0; they read
       // (and discard) the chunk's first columns instead of past the buffer
       const int clx = have ? cl : 0;
-      const float* xb = xs + clx + Sh::PAD * (clx / Sh::CH);
-      float nz[8];  // -zero of each row
-#pragma unroll
-      for (int i = 0; i < 8; ++i) nz[i] = -(float)zc[i];
-      float2 acc[8][M];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int t = 0; t < M; ++t) acc[i][t] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int wi = 0; wi < 4; ++wi) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int j = 0; j < Sh::HC; j += 2) {
-            // the activations of codes j, j + 1 of this half word, for every token
-            const int col = wi * Sh::CPW + h * Sh::HC + j;
-            float2 x2[M];
-#pragma unroll
-            for (int t = 0; t < M; ++t) x2[t] = *reinterpret_cast<const float2*>(xb + t * XS + col);
-            // -2^(23 - b j) for the two slots (compile-time constants)
-            const float2 nmag = make_float2(-(float)(1 << (23 - BITS * j)),
-                                            -(float)(1 << (23 - BITS * (j + 1))));
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint32_t word = wi == 0 ? d[i].x : wi == 1 ? d[i].y : wi == 2 ? d[i].z : d[i].w;
-              const uint32_t hw = h ? (word >> 16) : word;
-              // 2^(23 - b j) + c, exactly
-              const float f0 = __uint_as_float((0x4B000000u - ((uint32_t)(BITS * j) << 23)) |
-                                               (hw & (Sh::MASK << (BITS * j))));
-              const float f1 = __uint_as_float((0x4B000000u - ((uint32_t)(BITS * (j + 1)) << 23)) |
-                                               (hw & (Sh::MASK << (BITS * (j + 1)))));
-              const float2 one = make_float2(1.f, 1.f);
-              const float2 c2 = __ffma2_rn(make_float2(f0, f1), one, nmag);            // c, exact
-              const float2 dd = __ffma2_rn(c2, one, make_float2(nz[i], nz[i]));        // c - zero
-#pragma unroll
-              for (int t = 0; t < M; ++t) acc[i][t] = __ffma2_rn(x2[t], dd, acc[i][t]);
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int t = 0; t < M; ++t) y[i][t] = fmaf(sc[i], acc[i][t].x + acc[i][t].y, y[i][t]);
+      qv_compute<BITS, M>(cur, xs + clx + Sh::PAD * (clx / Sh::CH), XS, y);
+      if (sn < kcw) cur = nxt;
     }
   }
-  // sum the 8 pieces of each row, then the 16 warps
+  // sum the 8 pieces of each row, then the warps
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < QV_RPL; ++i)
 #pragma unroll
     for (int t = 0; t < M; ++t) {
       float v = y[i][t];
@@ -188,16 +220,16 @@ qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
     }
   if (p == 0) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < QV_RPL; ++i)
 #pragma unroll
-      for (int t = 0; t < M; ++t) red[(warp * M + t) * 32 + 4 * i + q] = y[i][t];
+      for (int t = 0; t < M; ++t) red[(warp * M + t) * QV_ROWS + 4 * i + q] = y[i][t];
   }
   __syncthreads();
-  for (int e = tid; e < M * 32; e += blockDim.x) {
-    const int t = e / 32, rr = e % 32;
+  for (int e = tid; e < M * QV_ROWS; e += blockDim.x) {
+    const int t = e / QV_ROWS, rr = e % QV_ROWS;
     float v = 0.f;
-#pragma unroll 4
-    for (int w = 0; w < QV_WARPS; ++w) v += red[(w * M + t) * 32 + rr];
+#pragma unroll
+    for (int w = 0; w < QV_WARPS; ++w) v += red[(w * M + t) * QV_ROWS + rr];
     if (t0 + t < m && r0 + rr < n) Y[(int64_t)(t0 + t) * ldy + r0 + rr] = qg_out<T>(v);
   }
 }
@@ -258,10 +290,13 @@ gptq_status launch_qgemv(const T* X, int64_t ldx, int m, int k, const int32_t* q
   using Sh = QvShape<BITS>;
   const int KC = qv_kc(k, Sh::SLAB);
   const size_t smem = qv_smem_bytes<BITS>(M, KC);
-  if (smem > 48 * 1024) {
+  static size_t smem_set = 48 * 1024;  // opt-in limit set so far for this instantiation
+  if (smem > smem_set) {
+    const size_t most = qv_smem_bytes<BITS>(M, QV_KC);
     if (cudaFuncSetAttribute(qgemv_kernel<BITS, M, T>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most) != cudaSuccess)
       return GPTQ_ERR_CUDA;
+    smem_set = most;
   }
   const dim3 grid((unsigned)cdiv(n, QV_ROWS), (unsigned)cdiv(m, M));
   qgemv_kernel<BITS, M, T><<<grid, QV_WARPS * 32, smem, s>>>(X, ldx, m, k, qw, scales, zeros, n,

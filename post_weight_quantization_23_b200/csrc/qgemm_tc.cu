@@ -143,11 +143,24 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
     const bool rv = row < a.n;
     const float* srow = a.scales + (int64_t)(rv ? row : 0) * a.ngroups;
     const int32_t* zrow = a.zeros + (int64_t)(rv ? row : 0) * a.ngroups;
-    int gcur = -1;
-    float sc = 0.f, zb = 8388608.f;
+    // the grids of a stage's two 32-column halves (a group holds whole
+    // halves), fetched one stage ahead so no load waits inside the loop
+    auto fetch = [&](int kc, float (&sc)[2], float (&zb)[2]) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int col = kc * QT_K + 32 * hf;
+        const bool ok = rv && kc < nk && col < a.k;
+        const int g = ok ? col / a.G : 0;
+        sc[hf] = ok ? srow[g] : 0.f;
+        zb[hf] = 8388608.f + (ok ? (float)zrow[g] : 0.f);  // 2^23 + zero, exact
+      }
+    };
+    float sc[2], zb[2], sc_n[2], zb_n[2];
+    fetch(0, sc, zb);
     for (int kc = 0; kc < nk; ++kc) {
       const int s = kc % QT_STAGES;
       const uint32_t ph = (uint32_t)(kc / QT_STAGES) & 1u;
+      fetch(kc + 1, sc_n, zb_n);
       if (!tc::mbar_wait(&full_tma[s], ph, abort_flag)) break;
       const uint4* pr = reinterpret_cast<const uint4*>(stage_p(s) + r * 32);
       const uint4 p0 = pr[0], p1 = pr[1];
@@ -155,20 +168,13 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
       uint8_t* arow = stage_a(s) + r * 128;
 #pragma unroll
       for (int wi = 0; wi < 8; ++wi) {
-        const int col = kc * QT_K + 8 * wi;
-        const int g = col < a.k ? col / a.G : -1;
-        if (g != gcur) {
-          gcur = g;
-          const bool ok = rv && g >= 0;
-          sc = ok ? srow[g] : 0.f;
-          zb = 8388608.f + (ok ? (float)zrow[g] : 0.f);  // 2^23 + zero, exact
-        }
+        const float s_w = sc[wi / 4], zb_w = zb[wi / 4];
         float w[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           // 2^23 + c exactly, minus 2^23 + zero: c - zero exactly; times the scale
           const float f = __uint_as_float(0x4B000000u | ((words[wi] >> (4 * j)) & 0xFu));
-          w[j] = (f - zb) * sc;
+          w[j] = (f - zb_w) * s_w;
         }
         uint4 o;
         if (a.bf16) {
@@ -183,6 +189,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
       tc::fence_proxy_async_smem();  // the MMA (async proxy) reads what this thread wrote
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&full_a[s]);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) sc[hf] = sc_n[hf], zb[hf] = zb_n[hf];
     }
     // epilogue
     const bool ok = tc::mbar_wait(done, 0, abort_flag) && !*abort_flag;

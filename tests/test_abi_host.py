@@ -121,6 +121,34 @@ def test_gemm_host_checks(lib):
     assert g(X=ctypes.c_void_p(257)) == _lib.GPTQ_ERR_INVALID_ARG  # misaligned X
 
 
+def test_rotate_host_checks(lib):
+    fake = ctypes.c_void_p(256)  # never dereferenced: every call below fails a host check
+    F16 = _lib.GPTQ_F16
+
+    def r(rows=4, k=512, ld_in=512, block=256, ld_out=512, inp=fake, out=ctypes.c_void_p(1 << 30),
+          signs=fake, dt=F16):
+        return lib.gptq_rotate(inp, dt, rows, k, ld_in, signs, block, 0, out, ld_out, None)
+
+    assert r(block=128) == _lib.GPTQ_ERR_UNSUPPORTED
+    assert r(block=384) == _lib.GPTQ_ERR_UNSUPPORTED
+    assert r(block=16384) == _lib.GPTQ_ERR_UNSUPPORTED
+    assert r(k=640, ld_in=640, ld_out=640) == _lib.GPTQ_ERR_INVALID_ARG   # k % block
+    assert r(rows=0) == _lib.GPTQ_OK
+    assert r(ld_in=256) == _lib.GPTQ_ERR_INVALID_ARG
+    assert r(ld_in=516) == _lib.GPTQ_ERR_INVALID_ARG                      # row not 16-byte aligned
+    assert r(signs=None) == _lib.GPTQ_ERR_INVALID_ARG
+    assert r(signs=ctypes.c_void_p(260)) == _lib.GPTQ_ERR_INVALID_ARG     # signs not 8-byte aligned
+    assert r(out=ctypes.c_void_p(256 + 512)) == _lib.GPTQ_ERR_INVALID_ARG  # overlapping buffers
+    assert r(dt=9) == _lib.GPTQ_ERR_INVALID_ARG
+
+
+def test_hadamard_block_choice():
+    from post_weight_quantization_23_b200 import hadamard_block
+    assert hadamard_block(4096) == 4096 and hadamard_block(11008) == 256
+    assert hadamard_block(12288) == 4096 and hadamard_block(16384) == 8192
+    assert hadamard_block(4160) == 0 and hadamard_block(0) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(P.GptqError):
