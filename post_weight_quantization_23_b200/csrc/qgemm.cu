@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(QV_WARPS * 32)
 qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
              const int32_t* __restrict__ qw, const float* __restrict__ scales,
              const int32_t* __restrict__ zeros, int n, int G, int ngroups, int KC,
-             T* __restrict__ Y, int64_t ldy) {
+             int xvec, T* __restrict__ Y, int64_t ldy) {
   using Sh = QvShape<BITS>;
   extern __shared__ __align__(16) float qv_smem[];
   const int XS = KC + Sh::PAD * (KC / Sh::CH);
@@ -184,11 +184,28 @@ qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
       qv_load<BITS>(cur, qw, scales, zeros, wpr, r0, q, n, kc0 + cl, cl < kcw, G, ngroups);
     }
     __syncthreads();  // the previous pass is done with xs
-    for (int e = tid; e < M * kcw; e += blockDim.x) {
-      const int t = e / kcw, c = e - t * kcw;
-      float v = 0.f;
-      if (t0 + t < m) v = to_f32(X[(int64_t)(t0 + t) * ldx + kc0 + c]);
-      xs[t * XS + c + Sh::PAD * (c / Sh::CH)] = v;
+    if (xvec) {
+      // 8 activations per 16-byte load, all of a thread's loads in flight
+      // together (kcw is a multiple of 8; 8 columns never straddle a pad)
+      const int nv = kcw / 8;
+#pragma unroll 4
+      for (int e = tid; e < M * nv; e += blockDim.x) {
+        const int t = e / nv, c = 8 * (e - t * nv);
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (t0 + t < m) u = *reinterpret_cast<const uint4*>(X + (int64_t)(t0 + t) * ldx + kc0 + c);
+        const T* h = reinterpret_cast<const T*>(&u);
+        float4* dst = reinterpret_cast<float4*>(xs + t * XS + c + Sh::PAD * (c / Sh::CH));
+        dst[0] = make_float4(to_f32(h[0]), to_f32(h[1]), to_f32(h[2]), to_f32(h[3]));
+        dst[1] = make_float4(to_f32(h[4]), to_f32(h[5]), to_f32(h[6]), to_f32(h[7]));
+      }
+    } else {
+#pragma unroll 8
+      for (int e = tid; e < M * kcw; e += blockDim.x) {
+        const int t = e / kcw, c = e - t * kcw;
+        float v = 0.f;
+        if (t0 + t < m) v = to_f32(X[(int64_t)(t0 + t) * ldx + kc0 + c]);
+        xs[t * XS + c + Sh::PAD * (c / Sh::CH)] = v;
+      }
     }
     __syncthreads();
     for (; sl < kcw; sl += QV_WARPS * Sh::SLAB) {
@@ -299,8 +316,10 @@ gptq_status launch_qgemv(const T* X, int64_t ldx, int m, int k, const int32_t* q
     smem_set = most;
   }
   const dim3 grid((unsigned)cdiv(n, QV_ROWS), (unsigned)cdiv(m, M));
+  // 16-byte activation loads when every row of X starts on a 16-byte boundary
+  const int xvec = ((uintptr_t)X % 16) == 0 && ldx % 8 == 0;
   qgemv_kernel<BITS, M, T><<<grid, QV_WARPS * 32, smem, s>>>(X, ldx, m, k, qw, scales, zeros, n,
-                                                             G, ngroups, KC, Y, ldy);
+                                                             G, ngroups, KC, xvec, Y, ldy);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
 }

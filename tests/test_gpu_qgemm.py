@@ -126,6 +126,12 @@ def test_qgemm_strided_and_empty():
     torch.cuda.synchronize()
     _check(Yp[:, :n], X, qw, scales, zeros, g_idx, 4, k, torch.float16)
     assert torch.all(Yp[:, n:] == 7.0)  # the padding is not written
+    # rows of X that do not start on 16-byte boundaries: the scalar staging path
+    Xo = torch.zeros(2, k + 3, dtype=torch.float16, device="cuda")
+    Xo[:, :k] = X.cuda()
+    Yo = quant_matmul(Xo[:, :k], qw.cuda(), scales.cuda(), zeros.cuda(), 4, 128)
+    torch.cuda.synchronize()
+    _check(Yo, X, qw, scales, zeros, g_idx, 4, k, torch.float16)
     # no tokens: nothing to do
     Y0 = quant_matmul(torch.empty(0, k, dtype=torch.float16, device="cuda"), qw.cuda(),
                       scales.cuda(), zeros.cuda(), 4, 128)
