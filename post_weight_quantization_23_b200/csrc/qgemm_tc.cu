@@ -9,11 +9,17 @@
 // One CTA per tile of 128 weight rows x 256 tokens, K in stages of 64:
 //   warp 0      TMA: the packed words of the 128 rows (128 x 32 bytes) and
 //               the 256 x 64 activation box (128-byte swizzle), one barrier;
-//   warps 2..5  thread = weight row: read its 8 packed words, w = s (c - z)
-//               in fp32 (exact c - z, one rounding by the scale), rounded
-//               once to the activations' type, written as the A operand in
-//               the 128-byte-swizzled K-major layout; then, after the last
-//               stage, the epilogue (TMEM lane = weight row, column = token);
+//   warps 2..9  thread = (weight row, 32-column half of the stage): its 4
+//               packed words become 32 weights in the activations' 16-bit
+//               type, two at a time: a byte permute and a mask put codes
+//               c_2i, c_2i+1 into the mantissas of a half2 holding M + c (M =
+//               1024 for f16, 128 for bf16: exact), one packed subtract of
+//               M + zero leaves c - zero exactly, one packed multiply by the
+//               scale (itself rounded to the type) gives the weight; written
+//               as the A operand in the 128-byte-swizzled K-major layout.
+//               After the last stage the same warps are the epilogue (TMEM
+//               lane = weight row, column = token; two warps per lane quarter
+//               split the tokens);
 //   warp 1      one thread issues kind::f16 MMAs D[128 x 256] += A B^T into
 //               TMEM (fp32), one commit per stage frees it.
 // Rows past n and tokens past m are zero-filled by TMA and not stored.  Every
@@ -32,7 +38,8 @@ constexpr int QT_A_BYTES = QT_M * QT_K * 2;          // 16 KB dequantized W tile
 constexpr int QT_B_BYTES = QT_N * QT_K * 2;          // 32 KB activation tile
 constexpr int QT_P_BYTES = QT_M * QT_K / 2;          // 4 KB packed 4-bit tile
 constexpr int QT_STAGE_BYTES = QT_A_BYTES + QT_B_BYTES + QT_P_BYTES;  // 52 KB, 1024-aligned
-constexpr int QT_THREADS = 192;
+constexpr int QT_DQ_WARPS = 8;                        // dequantizing / epilogue warps
+constexpr int QT_THREADS = 64 + 32 * QT_DQ_WARPS;     // + TMA and MMA warps
 constexpr int QT_TMEM_COLS = 256;
 constexpr size_t QT_SMEM = (size_t)QT_STAGES * QT_STAGE_BYTES + 1024 + 256;
 
@@ -42,23 +49,40 @@ struct QtArgs {
   void* Y;
   int64_t ldy;
   int n, m, k, G, ngroups;
-  int bf16;
 };
 
-__device__ __forceinline__ uint32_t pack2_f16(float a, float b) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));  // a in the low half
-  return r;
+// The 16-bit activation type T and its packed pair T2.
+template <bool BF16> struct QtType;
+template <> struct QtType<false> {
+  using T = __half;
+  using T2 = __half2;
+  static constexpr uint32_t MAGIC = 0x64006400u;  // 1024 in both halves: ulp 1 on [1024, 2048)
+  static constexpr float BASE = 1024.f;
+  __device__ static T2 pair(float v) { return __float2half2_rn(v); }
+  __device__ static T out(float v) { return __float2half_rn(v); }
+};
+template <> struct QtType<true> {
+  using T = __nv_bfloat16;
+  using T2 = __nv_bfloat162;
+  static constexpr uint32_t MAGIC = 0x43004300u;  // 128 in both halves: ulp 1 on [128, 256)
+  static constexpr float BASE = 128.f;
+  __device__ static T2 pair(float v) { return __float2bfloat162_rn(v); }
+  __device__ static T out(float v) { return __float2bfloat16_rn(v); }
+};
+
+template <typename T2> __device__ __forceinline__ T2 as_t2(uint32_t u) {
+  return *reinterpret_cast<T2*>(&u);
 }
-__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
-  return r;
+template <typename T2> __device__ __forceinline__ uint32_t as_u32(T2 v) {
+  return *reinterpret_cast<uint32_t*>(&v);
 }
 
+template <bool BF16>
 __global__ void __launch_bounds__(QT_THREADS, 1)
 qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap pmap,
                 QtArgs a) {
+  using Ty = QtType<BF16>;
+  using T2 = typename Ty::T2;
   extern __shared__ uint8_t qt_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)qt_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(smem + QT_STAGES * QT_STAGE_BYTES);
@@ -79,7 +103,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int s = 0; s < QT_STAGES; ++s) {
       tc::mbar_init(&full_tma[s], 1);
-      tc::mbar_init(&full_a[s], 4);
+      tc::mbar_init(&full_a[s], QT_DQ_WARPS);
       tc::mbar_init(&empty[s], 1);
     }
     tc::mbar_init(done, 1);
@@ -116,7 +140,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = tc::instr_desc(a.bf16 ? 1 : 0, QT_M, QT_N, 0, 0);  // both K-major
+      const uint32_t idesc = tc::instr_desc(BF16 ? 1 : 0, QT_M, QT_N, 0, 0);  // both K-major
       for (int kc = 0; kc < nk; ++kc) {
         const int s = kc % QT_STAGES;
         const uint32_t ph = (uint32_t)(kc / QT_STAGES) & 1u;
@@ -136,67 +160,60 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
       tc::mma_commit(done);  // also after a give-up: fires once the issued MMAs finish
     }
   } else {
-    // warps 2..5: thread = tile row (= its TMEM lane in the epilogue)
+    // warps 2..9: thread = (tile row = its TMEM lane, 32-column half of each stage)
+    const int dq = warp - 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    const int hf = dq >> 2;
     const int row = n0 + r;
     const bool rv = row < a.n;
     const float* srow = a.scales + (int64_t)(rv ? row : 0) * a.ngroups;
     const int32_t* zrow = a.zeros + (int64_t)(rv ? row : 0) * a.ngroups;
-    // the grids of a stage's two 32-column halves (a group holds whole
-    // halves), fetched one stage ahead so no load waits inside the loop
-    auto fetch = [&](int kc, float (&sc)[2], float (&zb)[2]) {
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int col = kc * QT_K + 32 * hf;
-        const bool ok = rv && kc < nk && col < a.k;
-        const int g = ok ? col / a.G : 0;
-        sc[hf] = ok ? srow[g] : 0.f;
-        zb[hf] = 8388608.f + (ok ? (float)zrow[g] : 0.f);  // 2^23 + zero, exact
-      }
+    // the grid of this thread's half of stage kc, as (scale, scale) and
+    // (M + zero, M + zero) pairs; fetched two stages ahead
+    auto fetch = [&](int kc, uint32_t& s2, uint32_t& z2) {
+      const int col = kc * QT_K + 32 * hf;
+      const bool ok = rv && kc < nk && col < a.k;
+      const int g = ok ? col / a.G : 0;
+      s2 = as_u32(Ty::pair(ok ? srow[g] : 0.f));
+      z2 = as_u32(Ty::pair(Ty::BASE + (ok ? (float)zrow[g] : 0.f)));  // exact
     };
-    float sc[2], zb[2], sc_n[2], zb_n[2];
-    fetch(0, sc, zb);
+    uint32_t s_c, z_c, s_1, z_1, s_2, z_2;
+    fetch(0, s_c, z_c);
+    fetch(1, s_1, z_1);
     for (int kc = 0; kc < nk; ++kc) {
       const int s = kc % QT_STAGES;
       const uint32_t ph = (uint32_t)(kc / QT_STAGES) & 1u;
-      fetch(kc + 1, sc_n, zb_n);
+      fetch(kc + 2, s_2, z_2);
       if (!tc::mbar_wait(&full_tma[s], ph, abort_flag)) break;
-      const uint4* pr = reinterpret_cast<const uint4*>(stage_p(s) + r * 32);
-      const uint4 p0 = pr[0], p1 = pr[1];
-      const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      const uint4 pw = reinterpret_cast<const uint4*>(stage_p(s) + r * 32)[hf];
+      const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
+      const T2 sc2 = as_t2<T2>(s_c), zz2 = as_t2<T2>(z_c);
       uint8_t* arow = stage_a(s) + r * 128;
 #pragma unroll
-      for (int wi = 0; wi < 8; ++wi) {
-        const float s_w = sc[wi / 4], zb_w = zb[wi / 4];
-        float w[8];
+      for (int wi = 0; wi < 4; ++wi) {
+        const uint32_t w = words[wi], w4 = w >> 4;
+        uint32_t o[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          // 2^23 + c exactly, minus 2^23 + zero: c - zero exactly; times the scale
-          const float f = __uint_as_float(0x4B000000u | ((words[wi] >> (4 * j)) & 0xFu));
-          w[j] = (f - zb_w) * s_w;
+        for (int i = 0; i < 4; ++i) {
+          // byte i of w (c_2i low) into half 0, byte i of w >> 4 (c_2i+1 low) into half 1
+          const uint32_t v = __byte_perm(w, w4, (uint32_t)(i | (i << 4) | ((4 + i) << 8) | (i << 12)));
+          const T2 h = as_t2<T2>((v & 0x000F000Fu) | Ty::MAGIC);     // M + c, exact
+          o[i] = as_u32(__hmul2(__hsub2(h, zz2), sc2));              // (c - z) exact, times s
         }
-        uint4 o;
-        if (a.bf16) {
-          o = make_uint4(pack2_bf16(w[0], w[1]), pack2_bf16(w[2], w[3]), pack2_bf16(w[4], w[5]),
-                         pack2_bf16(w[6], w[7]));
-        } else {
-          o = make_uint4(pack2_f16(w[0], w[1]), pack2_f16(w[2], w[3]), pack2_f16(w[4], w[5]),
-                         pack2_f16(w[6], w[7]));
-        }
-        *reinterpret_cast<uint4*>(arow + ((wi ^ (r & 7)) << 4)) = o;
+        *reinterpret_cast<uint4*>(arow + (((4 * hf + wi) ^ (r & 7)) << 4)) =
+            make_uint4(o[0], o[1], o[2], o[3]);
       }
       tc::fence_proxy_async_smem();  // the MMA (async proxy) reads what this thread wrote
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&full_a[s]);
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) sc[hf] = sc_n[hf], zb[hf] = zb_n[hf];
+      s_c = s_1, z_c = z_1, s_1 = s_2, z_1 = z_2;
     }
-    // epilogue
+    // epilogue: this warp's lane quarter, tokens [128 hf, 128 hf + 128)
     const bool ok = tc::mbar_wait(done, 0, abort_flag) && !*abort_flag;
     tc::tc_fence_after();
     const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
-    for (int c = 0; c < QT_N / 32; ++c) {
+    for (int c = 4 * hf; c < 4 * hf + 4; ++c) {
       float v[32];
       tc::tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), v);
       tc::tmem_ld_wait();
@@ -204,14 +221,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
 #pragma unroll
       for (int t = 0; t < 32; ++t) {
         const int tok = t0 + c * 32 + t;
-        if (tok < a.m) {
-          const float y = ok ? v[t] : __int_as_float(0x7fc00000);
-          if (a.bf16)
-            reinterpret_cast<__nv_bfloat16*>(a.Y)[(int64_t)tok * a.ldy + row] =
-                __float2bfloat16_rn(y);
-          else
-            reinterpret_cast<__half*>(a.Y)[(int64_t)tok * a.ldy + row] = __float2half_rn(y);
-        }
+        if (tok < a.m)
+          reinterpret_cast<typename Ty::T*>(a.Y)[(int64_t)tok * a.ldy + row] =
+              Ty::out(ok ? v[t] : __int_as_float(0x7fc00000));
       }
     }
   }
@@ -283,7 +295,9 @@ gptq_status qgemm_tc(const void* X, bool bf16, int64_t m, int64_t k, int64_t ldx
   }
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(qgemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(qgemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)QT_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(qgemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)QT_SMEM) != cudaSuccess)
       return GPTQ_ERR_CUDA;
     attr = true;
@@ -294,9 +308,11 @@ gptq_status qgemm_tc(const void* X, bool bf16, int64_t m, int64_t k, int64_t ldx
   a.Y = Y;
   a.ldy = ldy;
   a.n = (int)n, a.m = (int)m, a.k = (int)k, a.G = G, a.ngroups = (int)ngroups;
-  a.bf16 = bf16 ? 1 : 0;
   const dim3 grid((unsigned)cdiv(n, QT_M), (unsigned)cdiv(m, QT_N));
-  qgemm_tc_kernel<<<grid, QT_THREADS, QT_SMEM, s>>>(xmap, pmap, a);
+  if (bf16)
+    qgemm_tc_kernel<true><<<grid, QT_THREADS, QT_SMEM, s>>>(xmap, pmap, a);
+  else
+    qgemm_tc_kernel<false><<<grid, QT_THREADS, QT_SMEM, s>>>(xmap, pmap, a);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
 }

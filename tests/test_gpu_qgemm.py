@@ -54,10 +54,12 @@ def _check(Y, X, qw, scales, zeros, g_idx, bits, k, dtype, tc=False):
     # subnormal spacing for outputs that round into the subnormal range
     fp32_err = (k + 2) * 2.0 ** -24 * (np.abs(Xn) @ W_abs.T)
     if tc:
-        # tensor cores: each weight rounded once to the activations' type
-        # (2^-11 or 2^-8 relative), exact products, fp32 sums (counted twice
-        # over in case the adder truncates)
-        fp32_err = U_OUT[dtype] * (np.abs(Xn) @ W_abs.T) + 2 * fp32_err
+        # tensor cores: each weight is the scale rounded to the activations'
+        # type times the exact (code - zero), rounded once more (relative error
+        # at most 2u + u^2), exact products, fp32 sums (counted twice over in
+        # case the adder truncates)
+        u = U_OUT[dtype]
+        fp32_err = (2 * u + u * u) * (np.abs(Xn) @ W_abs.T) + 2 * fp32_err
     bound = U_OUT[dtype] * np.abs(ref) + (1 + U_OUT[dtype]) * fp32_err + 2.0 ** -25
     got = Y.float().cpu().numpy().astype(np.float64)
     err = np.abs(got - ref)
