@@ -48,7 +48,7 @@ class OraclePlan:
     def quantize(self, W, stream=None):
         c = self.cfg
         res = O.gptq(W.numpy(), self.H.numpy(), c.bits, c.group_size, c.block_size, c.percdamp,
-                     c.act_order)
+                     c.act_order, sym=c.sym, static_groups=c.static_groups)
         self.codes = torch.from_numpy(res["codes"].astype(np.uint8))
         self.scales = torch.from_numpy(np.ascontiguousarray(res["scales"], dtype=np.float32))
         self.zeros = torch.from_numpy(np.ascontiguousarray(res["zeros"], dtype=np.int32))
@@ -74,7 +74,8 @@ def _sharded_worker(rank, world, port, tag):
 
         spec = _spec()
         cfg = QuantConfig(spec.bits, spec.group_size, spec.block_size, spec.percdamp,
-                          act_order=(tag == "act"))
+                          act_order=(tag in ("act", "static", "sym_static")),
+                          sym=(tag == "sym_static"), static_groups=(tag in ("static", "sym_static")))
         W = synth.make_w(spec, 3).float()
         X = synth.make_x(spec, 3).float()
         layer = ShardedLayer(spec.r, spec.k, cfg, "cpu", plan_factory=OraclePlan)
@@ -82,7 +83,7 @@ def _sharded_worker(rank, world, port, tag):
         out = layer.run(X[t0:t1], spec.n, W)
         # every rank holds the same H after the all-reduce, and the whole layer after the gather
         ref = O.gptq(W.numpy(), O.hessian(X.numpy()), cfg.bits, cfg.group_size, cfg.block_size,
-                     cfg.percdamp, cfg.act_order)
+                     cfg.percdamp, cfg.act_order, sym=cfg.sym, static_groups=cfg.static_groups)
         assert np.allclose(layer.plan.H.numpy(), O.hessian(X.numpy()), rtol=1e-12, atol=1e-14)
         assert out["codes"].shape == (spec.r, spec.k)
         assert np.array_equal(out["codes"].numpy().astype(np.int64), ref["codes"])
@@ -94,7 +95,7 @@ def _sharded_worker(rank, world, port, tag):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("tag", ["plain", "act"])
+@pytest.mark.parametrize("tag", ["plain", "act", "static", "sym_static"])
 def test_sharded_layer_two_ranks_matches_single_process(tag):
     mp.spawn(_sharded_worker, args=(2, _free_port(), tag), nprocs=2, join=True)
 
