@@ -382,6 +382,8 @@ def native_arm(args, spec, world, rank, local):
         "hessian_ms": phase[0], "prepare_ms": phase[1], "quantize_ms": phase[2],
         "pack_ms": phase[3], "dequant_ms": phase[4],
         "hessian_tflops": achieved,
+        "hessian_issued_tflops": hessian_issued_flop(spec) / t_h / 1e12,
+        "prepare_tflops_algorithmic": (2.0 / 3.0) * float(spec.k) ** 3 / (phase[1] / 1e3) / 1e12,
         "hessian_x_gbs": spec.n * spec.k * 2 / t_h / 1e9,
         "sweep_model_gbs": sweep_bytes / (phase[2] / 1e3) / 1e9,
         "sweep_frac_hbm": sweep_bytes / (phase[2] / 1e3) / 1e9 / peaks["hbm"],
@@ -515,6 +517,15 @@ def rotation_measure(Xd, dev, stream, peaks, seed, reps=10):
             "kernel": "rotate_kernel (gptq_rotate)", "bound": "hbm", "us_per_launch": us,
             "bytes_per_launch": nbytes, "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
             "frac": gbs / peaks["hbm"]}
+
+
+def hessian_issued_flop(spec, tm=128, tn=256):
+    """Flops the Hessian kernel issues: 2 n tm tn per tile of tm x tn that
+    reaches the upper triangle (f16/bf16 path; the algorithmic count is
+    n k (k + 1))."""
+    ntm, ntn = -(-spec.k // tm), -(-spec.k // tn)
+    tiles = sum(1 for i in range(ntm) for j in range(ntn) if (j + 1) * tn > i * tm)
+    return 2.0 * spec.n * tiles * tm * tn
 
 
 def sweep_model_bytes(spec):
