@@ -257,12 +257,12 @@ EncodeTiledFn qt_encode_fn() {
 
 }  // namespace
 
-// The tensor-core path takes 4-bit codes, groups of whole 32-column runs (or
-// one per row), 16-byte aligned X and qweight and an X row stride that is a
-// multiple of 8 elements (the TMA rules).
+// The tensor-core path takes 4-bit codes, at least one full K stage (k >= 64),
+// groups of whole 32-column runs (or one per row), 16-byte aligned X and
+// qweight and an X row stride that is a multiple of 8 elements (the TMA rules).
 bool qgemm_tc_supported(const void* X, int64_t ldx, const int32_t* qw, int bits, int64_t k,
                         int G, bool has_gidx) {
-  return bits == 4 && !has_gidx && (G >= k || G % 32 == 0) && ((uintptr_t)X % 16) == 0 &&
+  return bits == 4 && !has_gidx && k >= QT_K && (G >= k || G % 32 == 0) && ((uintptr_t)X % 16) == 0 &&
          ((uintptr_t)qw % 16) == 0 && ldx % 8 == 0 && qt_encode_fn() != nullptr;
 }
 

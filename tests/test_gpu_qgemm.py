@@ -39,7 +39,7 @@ def _inputs(n, k, bits, G, m, dtype, seed, act_perm=False):
 
 def _tc_path(bits, G, k, m, pass_gidx):
     """Whether gptq_gemm takes the tensor-core kernel (contiguous inputs)."""
-    return bits == 4 and not pass_gidx and (G >= k or G % 32 == 0) and m >= 17
+    return bits == 4 and not pass_gidx and k >= 64 and (G >= k or G % 32 == 0) and m >= 17
 
 
 def _check(Y, X, qw, scales, zeros, g_idx, bits, k, dtype, tc=False):
