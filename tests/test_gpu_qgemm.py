@@ -150,3 +150,34 @@ def test_qgemm_bad_g_idx_gives_nan_not_a_fault():
     Y = quant_matmul(X.cuda(), qw.cuda(), scales.cuda(), zeros.cuda(), 4, 128, bad.cuda())
     torch.cuda.synchronize()
     assert torch.all(torch.isnan(Y.float()))
+
+
+@pytest.mark.parametrize("act,static,m", [(True, False, 3), (True, True, 1), (False, False, 32)])
+def test_plan_matmul_matches_its_own_dequantized_weights(act, static, m):
+    # A consistency property of the plan's glue (which g_idx it passes): Y from
+    # the packed codes equals X W_hat^T with the plan's own fp32 dequantized
+    # weights, up to the kernels' rounding (bounds as in _check).
+    from post_weight_quantization_23_b200 import GptqPlan, QuantConfig
+    spec = synth.CONFIGS["q_proj"].scaled(r=256, k=512, n=4096)
+    W = synth.make_w(spec, 8).cuda()
+    X = synth.make_x(spec, 8).cuda()
+    cfg = QuantConfig(4, 128, 128, 0.01, act, static_groups=static)
+    plan = GptqPlan(spec.r, spec.k, cfg, "cuda", deq_dtype=torch.float32)
+    plan.hessian_add(X, spec.n)
+    plan.run_after_hessian(W)
+    plan.check()
+    Xm = X[:m].contiguous()
+    Y = plan.matmul(Xm)
+    torch.cuda.synchronize()
+    Wd = plan.deq.double().cpu().numpy()
+    Xn = Xm.double().cpu().numpy()
+    ref = Xn @ Wd.T
+    k = spec.k
+    u = U_OUT[torch.float16]
+    # + 2 roundings: the plan's fp32 weights are themselves rounded s (c - z)
+    e = (k + 4) * 2.0 ** -24 * (np.abs(Xn) @ np.abs(Wd).T)
+    if _tc_path(4, 128, k, m, cfg.act_order and not cfg.static_groups):
+        e = (2 * u + u * u) * (np.abs(Xn) @ np.abs(Wd).T) + 2 * e
+    bound = u * np.abs(ref) + (1 + u) * e + 2.0 ** -25
+    err = np.abs(Y.double().cpu().numpy() - ref)
+    assert np.all(err <= bound), float((err / bound).max())
