@@ -259,9 +259,15 @@ GPTQ_API gptq_status gptq_dequant(const int32_t* qweight, const float* scales, c
  *           defines the groups and ngroups must be ceil(k / group_size).
  *   Y       (m, n) out, dt, row-major, leading dimension ldy >= n.
  *   m <= 131070 tokens.  The library allocates nothing.
- * With g_idx NULL, bits 2/4/8 and group_size a multiple of 128/bits (or one
- * group per row), the decode kernel runs (weights streamed once per 2 tokens,
- * each product exact in fp32); every other case runs the general kernel.
+ * Kernel choice (all results within the same bounds of the exact product):
+ *   m >= 17, 4-bit, g_idx NULL, k >= 64, group_size a multiple of 32 (or one
+ *     group per row), X and qweight 16-byte aligned, ldx % 8 == 0: the
+ *     tensor-core kernel (each weight formed in dt: the scale rounded to dt
+ *     times the exact code - zero, rounded once more; fp32 accumulation);
+ *   else g_idx NULL, bits 2/4/8 and group_size a multiple of 128/bits (or one
+ *     group per row): the decode kernel (weights streamed once per 2 tokens,
+ *     each product x (code - zero) exact in fp32);
+ *   every other case: the general kernel (fp32 weights per element).
  * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_UNSUPPORTED (bits, f32 X),
  * GPTQ_ERR_CUDA. */
 GPTQ_API gptq_status gptq_gemm(const void* X, gptq_dtype dt, int64_t m, int64_t k, int64_t ldx,
