@@ -726,6 +726,12 @@ def test_rotation_worked_values_and_outlier_spread():
     s = np.ones(4)
     assert O.rotate(np.eye(4)[:2], s, 4).tolist() == [[0.5, 0.5, 0.5, 0.5],
                                                       [0.5, -0.5, 0.5, -0.5]]
+    # the signs act on the input coordinates (Q = diag(s) H / sqrt(b)): with s_1 = -1,
+    # e_1 Q = -[1, -1, 1, -1] / 2, while signs on the outputs would give
+    # [1, -1, 1, -1] / 2 * s = [0.5, 0.5, 0.5, -0.5]
+    s = np.array([1, -1, 1, 1])
+    assert O.rotate(np.eye(4)[1:2], s, 4).tolist() == [[-0.5, 0.5, -0.5, 0.5]]
+    assert O.rotate(np.array([[-0.5, 0.5, -0.5, 0.5]]), s, 4, inverse=True).tolist() == [[0, 1, 0, 0]]
     x = np.zeros((1, 256))
     x[0, 37] = 100.0
     y = O.rotate(x, np.random.default_rng(0).choice([-1, 1], 256), 256)
