@@ -18,9 +18,13 @@
  * Pointers.   Every array argument is a DEVICE pointer (memory the caller
  *             allocated with cudaMalloc or a caching allocator on the device
  *             the call runs on) unless its comment says otherwise.  The
- *             library allocates nothing and keeps no state between calls;
+ *             library allocates no memory and keeps no per-call state;
  *             scratch memory is the caller's workspace `ws` of at least
- *             gptq_workspace_size(...) bytes, 256-byte aligned.
+ *             gptq_workspace_size(...) bytes, 256-byte aligned.  Process-
+ *             wide it only caches the driver's tensor-map encoder entry
+ *             point and each kernel's shared-memory opt-in (set on first
+ *             use); gptq_prepare_hinv_noalloc alone uses a file-scope device
+ *             scratch array (see there).
  * Layout.     Row-major.  W is (r, k): r = out-features (rows), k =
  *             in-features (columns); X is (n, k): n calibration tokens.
  *             Leading dimensions are in elements.
@@ -32,7 +36,9 @@
  *             Failures that only the device can see are written to device
  *             status words (`d_info`, `d_status`) that the caller reads after
  *             synchronising; no kernel traps, asserts or waits without bound.
- * Inputs.     W, X and H are never modified.
+ * Inputs.     W and X are never modified (gptq_rotate writes `out`, which
+ *             is `in` only when the caller asks for an in-place rotation);
+ *             H is written only by gptq_hessian_accumulate (H += ...).
  */
 #ifndef GPTQ_B200_H
 #define GPTQ_B200_H
