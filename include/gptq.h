@@ -63,7 +63,7 @@ typedef enum {
   GPTQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, leading dimension, alignment */
   GPTQ_ERR_NOT_PD = 2,      /* damped Hessian not positive definite (device: d_info) */
   GPTQ_ERR_CUDA = 3,        /* a kernel launch failed */
-  GPTQ_ERR_UNSUPPORTED = 4, /* valid request this build does not implement (bits, dtype) */
+  GPTQ_ERR_UNSUPPORTED = 4, /* valid request the library does not implement (bits, dtype) */
   GPTQ_ERR_WORKSPACE = 5,   /* workspace null, too small or misaligned */
   GPTQ_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
   GPTQ_ERR_NONFINITE = 7    /* NaN/Inf met in the weights being quantized (device: d_status) */
