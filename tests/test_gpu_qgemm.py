@@ -181,3 +181,26 @@ def test_plan_matmul_matches_its_own_dequantized_weights(act, static, m):
     bound = u * np.abs(ref) + (1 + u) * e + 2.0 ** -25
     err = np.abs(Y.double().cpu().numpy() - ref)
     assert np.all(err <= bound), float((err / bound).max())
+
+
+@pytest.mark.parametrize("n,k", [(11008, 4096), (4096, 11008)])
+@pytest.mark.parametrize("m", [1, 2048])
+def test_qgemm_full_size_7b_mlp_shapes(n, k, m):
+    # The other layer shapes the bench times (gate/up and down of a 7B block),
+    # int4 g128, in full on the device (decode kernel at 1 token, tensor cores
+    # at 2048).  The packed words are seeded random int32 (every code pattern),
+    # and the oracle checks 512 sampled output features.
+    from post_weight_quantization_23_b200 import quant_matmul
+    G = 128
+    g = torch.Generator().manual_seed(n + m)
+    qw = torch.randint(-2 ** 31, 2 ** 31 - 1, (n, k // 8), generator=g, dtype=torch.int32)
+    scales = (torch.rand(n, k // G, generator=g) * 0.02 + 1e-3).float()
+    zeros = torch.randint(0, 16, (n, k // G), generator=g, dtype=torch.int32)
+    g_idx = (torch.arange(k) // G).to(torch.int32)
+    spec = synth.CONFIGS["q_proj"].scaled(r=n, k=k, n=m)
+    X = synth.make_x(spec, n + m)[:m].to(torch.float16)
+    Y = quant_matmul(X.cuda(), qw.cuda(), scales.cuda(), zeros.cuda(), 4, G)
+    torch.cuda.synchronize()
+    rows = torch.randperm(n, generator=g)[:512]
+    _check(Y.cpu()[:, rows], X, qw[rows], scales[rows], zeros[rows], g_idx, 4, k, torch.float16,
+           _tc_path(4, G, k, m, False))
