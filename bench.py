@@ -15,7 +15,12 @@ value  = weights quantized per second over all ranks (Mweights/s), inputs
 e2e    = the same metric through the host-buffer API (pinned X and W copied in,
          packed result and loss copied out, inside the timed region).
 N > 1  = weak scaling: every rank quantizes its own independent layer (a
-         different seed); no collective is on the data path.
+         different seed); no collective is on the data path.  --mode sharded
+         instead splits ONE layer over the ranks (tokens for H + all-reduce,
+         rows for the sweep + all-gather): strong scaling.
+other_configs = the other layer shapes (down_proj 4096 x 11008 act-order, the
+         OPT-175B-width 12288 x 12288 3-bit layer, one decoder layer of the 7B
+         stack), per phase, inputs drawn on the device (N = 1 only).
 --impl reference runs the fp64 CPU oracle on a bounded sample of the same
 workload (rank 0 only) and prints the same line with "impl": "reference".
 """
@@ -42,12 +47,15 @@ METRIC = "GPTQ layer quantize Mweights/s end-to-end"
 UNIT = "Mweights/s"
 
 
-# DRAM traffic of hessian_tc_kernel from one ncu capture (32768 tokens, k = 4096,
-# units of 15104 tokens): 645.9 MB read + 65.9 MB written.  Scaled by tokens to a
-# full launch -- an estimate: a full q_proj launch runs 65536-token units, whose
-# reuse of X in L2 differs.
-HESS_TRAFFIC_K = 4096
-HESS_TRAFFIC_BYTES_PER_TOKEN = (645.9e6 + 65.9e6) / 32768
+# DRAM traffic of hessian_tc_kernel per calibration token, by k, from ncu
+# captures (dram__bytes_read.sum + dram__bytes_write.sum of one launch on a
+# smaller token count, scaled by tokens to a full launch: an estimate).  Only
+# the widths a capture exists for; the line reports null elsewhere.
+HESS_TRAFFIC = {
+    4096: ((645.9e6 + 65.9e6) / 32768,
+           "estimate: ncu dram bytes of hessian_tc_kernel on a 32768 x 4096 capture, scaled by "
+           "tokens (profiles/hessian_tc_kernel_q_proj_32k_tokens.md)"),
+}
 
 
 def _peaks():
@@ -255,84 +263,162 @@ def workload_config(spec):
 
 # --------------------------------------------------------------------------- native arm
 
+def _cfg_of(spec):
+    from post_weight_quantization_23_b200 import QuantConfig
+    return QuantConfig(spec.bits, spec.group_size, spec.block_size, spec.percdamp, spec.act_order,
+                       spec.sym, spec.static_groups)
+
+
+class LayerRun:
+    """One layer's plan and its device-resident inputs; ``step`` issues the
+    whole hot path (H reset, Hessian over all tokens, factor, sweep with the
+    loss, pack, dequant), optionally with events between the phases."""
+
+    PHASES = ("hessian", "prepare", "quantize", "pack", "dequant")
+
+    def __init__(self, spec, Xd, Wd, dev):
+        from post_weight_quantization_23_b200 import GptqPlan
+        self.spec, self.Xd, self.Wd, self.dev = spec, Xd, Wd, dev
+        self.plan = GptqPlan(spec.r, spec.k, _cfg_of(spec), dev, want_loss=True,
+                             deq_dtype=torch.float16, hessian_tokens_hint=spec.n)
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+
+    def lib_calls(self):
+        p = self.plan
+        p.hessian_add(self.Xd, self.spec.n)
+        p.prepare()
+        p.quantize(self.Wd)
+        p.pack()
+        p.dequant()
+
+    def step(self, record=False, stream=None):
+        p, ev = self.plan, self.ev
+        stream = stream or torch.cuda.current_stream(self.dev)
+        if record:
+            ev[0].record(stream)
+        p.hessian_reset()
+        p.hessian_add(self.Xd, self.spec.n)
+        for i, fn in enumerate((p.prepare, lambda: p.quantize(self.Wd), p.pack, p.dequant)):
+            if record:
+                ev[i + 1].record(stream)
+            fn()
+        if record:
+            ev[5].record(stream)
+
+    def phase_ms(self, reps):
+        """Per-phase device times (CUDA events between phases), mean of reps."""
+        acc = np.zeros(5)
+        for _ in range(reps):
+            self.step(record=True)
+            torch.cuda.synchronize(self.dev)
+            acc += [self.ev[i].elapsed_time(self.ev[i + 1]) for i in range(5)]
+        return acc / reps
+
+
+def timed_replays(graph, steps, dev, stream):
+    """Device ms per replay of ``graph`` over ``steps`` back-to-back replays."""
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    return t0.elapsed_time(t1) / steps
+
+
+def phase_figures(spec, phase, peaks):
+    """Absolute and roofline figures of one layer's per-phase times (ms)."""
+    flops = float(spec.n) * spec.k * (spec.k + 1)  # symmetric triangle, algorithmic
+    t_h = phase[0] / 1e3
+    sweep_bytes = sweep_model_bytes(spec)
+    hess = flops / t_h / 1e12
+    return {
+        "hessian_ms": phase[0], "prepare_ms": phase[1], "quantize_ms": phase[2],
+        "pack_ms": phase[3], "dequant_ms": phase[4],
+        "hessian_tflops": hess,
+        "hessian_frac_bf16_burst": hess / peaks["bf16"],
+        "hessian_frac_bf16_sustained": hess / peaks["bf16_sustained"],
+        "hessian_issued_tflops": hessian_issued_flop(spec) / t_h / 1e12,
+        "prepare_tflops_algorithmic": (2.0 / 3.0) * float(spec.k) ** 3 / (phase[1] / 1e3) / 1e12,
+        "hessian_x_gbs": spec.n * spec.k * 2 / t_h / 1e9,
+        "sweep_model_bytes": sweep_bytes,
+        "sweep_model_gbs": sweep_bytes / (phase[2] / 1e3) / 1e9,
+        "sweep_frac_hbm": sweep_bytes / (phase[2] / 1e3) / 1e9 / peaks["hbm"],
+    }
+
+
+def other_configs(dev, stream, peaks, seed, steps, names):
+    """The other layer shapes of the pages (down_proj, the OPT-175B-width
+    layer, one decoder layer of the 7B stack), each measured alone with inputs
+    drawn on the device (same distributions as the CPU generator; timing
+    only): per-phase device times, Mweights/s over one CUDA graph per step."""
+    out = {}
+    for name in names:
+        subs = ([n for n in synth.CONFIGS if n.startswith("stack_")] if name == "stack_layer"
+                else [name])
+        runs = []
+        for sub in subs:
+            spec = synth.CONFIGS[sub]
+            runs.append(LayerRun(spec, synth.make_x_device(spec, seed, dev),
+                                 synth.make_w_device(spec, seed, dev), dev))
+        for run in runs:
+            for _ in range(2):
+                run.step()
+            run.plan.check()
+        entry = {}
+        for run in runs:
+            ph = run.phase_ms(3)
+            entry[run.spec.name] = {"workload": workload_config(run.spec)["workload"],
+                                    **phase_figures(run.spec, ph, peaks)}
+        graph = runs[0].plan.capture(lambda: [r.step() for r in runs])
+        ms = timed_replays(graph, steps, dev, stream)
+        for run in runs:
+            run.plan.check()
+        weights = sum(r.spec.r * r.spec.k for r in runs)
+        out[name] = {"value": weights / (ms / 1e3) / 1e6, "unit": UNIT, "ms_per_step": ms,
+                     "steps": steps, "layers": entry,
+                     "data": "synthetic, drawn on the device (same distributions)"}
+        if name == "stack_layer":
+            out[name]["note"] = ("one decoder layer of the 32-layer 7B-shaped stack (qkv and "
+                                 "gate/up stacked on their shared Hessians); the 32 layers are "
+                                 "identical in shape and independent")
+        del graph, runs
+        torch.cuda.empty_cache()
+    return out
+
+
 def native_arm(args, spec, world, rank, local):
-    from post_weight_quantization_23_b200 import GptqPlan, QuantConfig
     from post_weight_quantization_23_b200.api import HostPipeline
 
     dev = torch.device("cuda", local if world > 1 else 0)
     seed = args.seed + rank  # independent layer per rank (weak scaling)
-    cfg = QuantConfig(spec.bits, spec.group_size, spec.block_size, spec.percdamp, spec.act_order,
-                      spec.sym, spec.static_groups)
     xdt = synth.dtype_of(spec.x_dtype)
     X_host = torch.empty(spec.n, spec.k, dtype=xdt, pin_memory=True)
     synth.make_x(spec, seed, out=X_host)
     W_host = synth.make_w(spec, seed).pin_memory()
-    Xd = X_host.to(dev)
-    Wd = W_host.to(dev)
-    plan = GptqPlan(spec.r, spec.k, cfg, dev, want_loss=True, deq_dtype=torch.float16,
-                    hessian_tokens_hint=spec.n)
+    run = LayerRun(spec, X_host.to(dev), W_host.to(dev), dev)
+    plan = run.plan
     stream = torch.cuda.current_stream(dev)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-
-    def lib_calls():
-        plan.hessian_add(Xd, spec.n)
-        plan.prepare()
-        plan.quantize(Wd)
-        plan.pack()
-        plan.dequant()
-
-    def step(record=False):
-        if record:
-            ev[0].record(stream)
-        plan.hessian_reset()
-        plan.hessian_add(Xd, spec.n)
-        if record:
-            ev[1].record(stream)
-        plan.prepare()
-        if record:
-            ev[2].record(stream)
-        plan.quantize(Wd)
-        if record:
-            ev[3].record(stream)
-        plan.pack()
-        if record:
-            ev[4].record(stream)
-        plan.dequant()
-        if record:
-            ev[5].record(stream)
 
     for _ in range(args.warmup):
-        step()
+        run.step()
     plan.check()
+    phase = run.phase_ms(max(2, min(args.steps, 5)))
 
-    # per-phase device times (separate pass, events between phases)
-    phase = np.zeros(5)
-    n_phase = max(2, min(args.steps, 5))
-    for _ in range(n_phase):
-        step(record=True)
-        torch.cuda.synchronize(dev)
-        phase += [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
-    phase /= n_phase
-
-    launches = count_launches(lib_calls, dev)  # the H reset is a torch fill, not ours
+    launches = count_launches(run.lib_calls, dev)  # the H reset is a torch fill, not ours
     plan.check()
-    graph = plan.capture(step)  # the timed steps replay one CUDA graph per step
+    graph = plan.capture(run.step)  # the timed steps replay one CUDA graph per step
 
     clocks = ClockSampler(dev.index)
     barrier(world)
     torch.cuda.synchronize(dev)
     clocks.start()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for _ in range(args.steps):
-        graph.replay()
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
+    ms = timed_replays(graph, args.steps, dev, stream)
     barrier(world)
     clk = clocks.stop()
     plan.check()
-    ms = t_start.elapsed_time(t_end) / args.steps
     ms = max_over_ranks(ms, world)
     value = world * spec.r * spec.k / (ms / 1e3) / 1e6
 
@@ -361,33 +447,22 @@ def native_arm(args, spec, world, rank, local):
                "d2h_bytes_per_step": pipe.d2h_bytes()}
 
     peaks = _peaks()
-    flops = float(spec.n) * spec.k * (spec.k + 1)  # symmetric triangle, algorithmic
-    t_h = phase[0] / 1e3
-    achieved = flops / t_h / 1e12
-    traffic = args.traffic
-    if traffic is None and spec.k == HESS_TRAFFIC_K:
-        # DRAM bytes of one capture of this kernel at k = 4096, scaled to n tokens
-        traffic = HESS_TRAFFIC_BYTES_PER_TOKEN * spec.n
+    phases = phase_figures(spec, phase, peaks)
+    flops = float(spec.n) * spec.k * (spec.k + 1)
+    traffic, tsrc = None, None
+    if args.traffic is not None:
+        traffic, tsrc = args.traffic, "given on the command line (ncu capture of this workload)"
+    elif spec.k in HESS_TRAFFIC:
+        per_tok, src = HESS_TRAFFIC[spec.k]
+        traffic, tsrc = per_tok * spec.n, src
     roofline = {"bound": "tensor", "kernel": "gptq_hessian_accumulate (X^T X)",
-                "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_sustained"], "traffic": traffic,
-                "traffic_source": ("estimate: ncu dram__bytes_read.sum + dram__bytes_write.sum "
-                                   "of hessian_tc_kernel on a 32768 x 4096 capture, scaled by "
-                                   "tokens (profiles/hessian_tc_kernel_q_proj_32k_tokens.md)")
-                if traffic is not None and args.traffic is None else None,
-                "peak_kind": f"bf16 dense sustained ({peaks['source']}); f16 has the same nominal rate",
+                "achieved": phases["hessian_tflops"], "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": phases["hessian_tflops"] / peaks["bf16"], "traffic": traffic,
+                "traffic_source": tsrc,
+                "peak_kind": (f"bf16 dense burst ({peaks['source']}); f16 has the same nominal "
+                              f"rate"),
+                "frac_of_sustained": phases["hessian_tflops"] / peaks["bf16_sustained"],
                 "algorithmic": f"n*k*(k+1) = {flops:.4g} flop per launch"}
-    sweep_bytes = sweep_model_bytes(spec)
-    phases = {
-        "hessian_ms": phase[0], "prepare_ms": phase[1], "quantize_ms": phase[2],
-        "pack_ms": phase[3], "dequant_ms": phase[4],
-        "hessian_tflops": achieved,
-        "hessian_issued_tflops": hessian_issued_flop(spec) / t_h / 1e12,
-        "prepare_tflops_algorithmic": (2.0 / 3.0) * float(spec.k) ** 3 / (phase[1] / 1e3) / 1e12,
-        "hessian_x_gbs": spec.n * spec.k * 2 / t_h / 1e9,
-        "sweep_model_gbs": sweep_bytes / (phase[2] / 1e3) / 1e9,
-        "sweep_frac_hbm": sweep_bytes / (phase[2] / 1e3) / 1e9 / peaks["hbm"],
-    }
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -398,10 +473,14 @@ def native_arm(args, spec, world, rank, local):
         "gpu_launches": launches * args.steps if launches is not None else None,
         "gpu_launches_per_step": launches, "clocks": clk, "e2e": e2e,
     }
+    del graph
+    if not args.no_other_configs and world == 1:
+        names = [n for n in ("down_proj", "opt175_width", "stack_layer") if n != spec.name]
+        line["other_configs"] = other_configs(dev, stream, peaks, seed, args.other_steps, names)
     if not args.no_qgemm:
         line["inference_matmul"] = qgemm_measure(dev, stream, peaks, args.seed + rank)
     if not args.no_rotation:
-        line["rotation"] = rotation_measure(Xd, dev, stream, peaks, args.seed + rank)
+        line["rotation"] = rotation_measure(run.Xd, dev, stream, peaks, args.seed + rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_full, wall, sample = oracle_sample(spec, args.seed, args.ref_tokens, args.ref_rows)
         line["cpu_baseline"] = {"value": spec.r * spec.k / t_full / 1e6, "unit": UNIT,
@@ -409,6 +488,69 @@ def native_arm(args, spec, world, rank, local):
                                 "sample": sample + f"; wall {wall:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    return 0
+
+
+def sharded_arm(args, spec, world, rank, local):
+    """One layer split over the ranks (strong scaling): each rank accumulates
+    the Hessian of its share of the tokens, one all-reduce sums H, every rank
+    computes the factor, each sweeps its block of rows, and the codes,
+    scales, zeros and per-row losses are all-gathered.  Eager launches (the
+    collectives are not captured); device time, max over ranks."""
+    from post_weight_quantization_23_b200.sharded import ShardedLayer
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    own_group = False
+    if not torch.distributed.is_initialized():  # N = 1: a one-rank group
+        import datetime
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        torch.distributed.init_process_group(
+            "nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+            timeout=datetime.timedelta(seconds=300), device_id=dev)
+        own_group = True
+    group = torch.distributed.group.WORLD
+    layer = ShardedLayer(spec.r, spec.k, _cfg_of(spec), dev, group=group, want_loss=True,
+                         deq_dtype=None, hessian_tokens_hint=spec.n)
+    t0, t1 = layer.token_range(spec.n)
+    X_all = synth.make_x_device(spec, args.seed, dev)
+    X_local = X_all[t0:t1].contiguous()
+    del X_all
+    W = synth.make_w_device(spec, args.seed, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.plan.hessian_reset()
+        return layer.run(X_local, spec.n, W)
+
+    for _ in range(args.warmup):
+        step()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    line = {
+        "metric": METRIC, "value": spec.r * spec.k / (ms / 1e3) / 1e6, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic, drawn on the device",
+        "config": dict(workload_config(spec), parallelism=(
+            f"one layer over {world} ranks: tokens sharded for H + all-reduce, factor "
+            f"replicated, rows sharded for the sweep + all-gather"),
+            launch="eager (collectives between the library calls)"),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if own_group:
+        torch.distributed.destroy_process_group()
     return 0
 
 
@@ -607,6 +749,13 @@ def main():
     ap.add_argument("--act-order", action="store_true", help="variant: act-order")
     ap.add_argument("--sym", action="store_true", help="variant: symmetric grid")
     ap.add_argument("--static-groups", action="store_true", help="variant: static groups")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the down_proj / OPT-175B-width / stack-layer measurements")
+    ap.add_argument("--other-steps", type=int, default=5,
+                    help="timed steps of each other config")
+    ap.add_argument("--mode", choices=["layers", "sharded"], default="layers",
+                    help="layers: every rank its own layer (weak scaling); sharded: one layer "
+                         "split over the ranks (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -632,6 +781,8 @@ def main():
         return 0
     world, rank, local = dist_setup(args)
     try:
+        if args.mode == "sharded":
+            return sharded_arm(args, spec, world, rank, local)
         return native_arm(args, spec, world, rank, local)
     finally:
         if world > 1:

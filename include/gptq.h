@@ -22,9 +22,11 @@
  *             scratch memory is the caller's workspace `ws` of at least
  *             gptq_workspace_size(...) bytes, 256-byte aligned.  Process-
  *             wide it only caches the driver's tensor-map encoder entry
- *             point and each kernel's shared-memory opt-in (set on first
- *             use); gptq_prepare_hinv_noalloc alone uses a file-scope device
- *             scratch array (see there).
+ *             point, each kernel's shared-memory opt-in (per device, under a
+ *             lock, set on first use) and the wait limit of
+ *             gptq_set_wait_limit; gptq_prepare_hinv_noalloc alone uses a
+ *             file-scope device scratch array (see there).  Calls may come
+ *             from several host threads and for several devices.
  * Layout.     Row-major.  W is (r, k): r = out-features (rows), k =
  *             in-features (columns); X is (n, k): n calibration tokens.
  *             Leading dimensions are in elements.
@@ -131,7 +133,14 @@ GPTQ_API const char* gptq_status_string(gptq_status s);
  *          ldx % 8 == 0 and a 16-byte aligned X.
  *   H      (k, k) fp32, symmetric on entry (zero it before the first chunk);
  *          both triangles are updated.  Must not alias X.
- *   ws     GPTQ_OP_HESSIAN workspace (may be NULL when that size is 0).
+ *   ws     GPTQ_OP_HESSIAN workspace (256 bytes, 256-byte aligned).  Its
+ *          second int32, ((int32_t*)ws)[1], is a device status word the
+ *          library only ever sets: GPTQ_ERR_TIMEOUT once a bounded wait of
+ *          the tensor-core kernel gave up in this call or an earlier one on
+ *          the same workspace (H[0][0] is then NaN as well, so a caller who
+ *          never reads the word meets the failure in gptq_prepare_hinv).
+ *          Zero it with H before the first chunk; read it after
+ *          synchronising.  The first int32 is the library's own.
  * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_WORKSPACE, GPTQ_ERR_CUDA.
  * n == 0 or k == 0 is a no-op. */
 GPTQ_API gptq_status gptq_hessian_accumulate(const void* X, gptq_dtype dt, int64_t n, int64_t k,
@@ -155,7 +164,9 @@ GPTQ_API gptq_status gptq_hessian_accumulate(const void* X, gptq_dtype dt, int64
  *   dead    uint8[k] out (original column order): 1 = dead column.
  *   d_info  int32 device scalar out: 0, or 1 + the processing-order index
  *           of the first pivot found non-positive or non-finite (then U is
- *           unspecified; retry with a larger percdamp).
+ *           unspecified; retry with a larger percdamp), or k + 1 when a
+ *           bounded wait of a tensor-core update gave up (GPTQ_ERR_TIMEOUT;
+ *           U is unspecified).
  *   ws      GPTQ_OP_PREPARE_HINV workspace.
  * Returns GPTQ_OK (the device may still report NOT_PD in d_info),
  * GPTQ_ERR_INVALID_ARG, GPTQ_ERR_WORKSPACE, GPTQ_ERR_CUDA. */
@@ -164,21 +175,44 @@ GPTQ_API gptq_status gptq_prepare_hinv(const float* H, int64_t k, const gptq_con
                               int32_t* d_info, void* ws, size_t ws_bytes,
                               gptq_stream_t stream);
 
+/* Test hook: the number of polls after which a pipeline wait inside the
+ * tensor-core kernels (Hessian, factor and sweep updates, lane sweep, the
+ * tensor-core inference product) gives up and takes its error path.  It
+ * applies to launches made after the call, from any thread; the waits that
+ * let a CTA's own copies and MMAs land before it exits keep their full bound.
+ * 0 makes every such wait give up at once (each stage then reports
+ * GPTQ_ERR_TIMEOUT as its comment says); GPTQ_WAIT_LIMIT_DEFAULT restores the
+ * default (2^26 polls, far beyond any correct wait).  Not for production use:
+ * a small limit turns slow waits into failures. */
+#define GPTQ_WAIT_LIMIT_DEFAULT 0xFFFFFFFFu
+GPTQ_API void gptq_set_wait_limit(uint32_t polls);
+
 /* gptq_prepare_hinv without a workspace, for callers that cannot allocate
  * device memory (the pages have no counterpart: this is an interface
  * convenience, not part of the method).
  * Some callers cannot call cudaMalloc or hand over a workspace: a plugin
  * whose host passes it only its input and output buffers, a process that has
  * carved all device memory into its own arena, or a runtime that forbids
- * allocation after start-up.  This call computes exactly what
- * gptq_prepare_hinv computes (same arguments minus ws / ws_bytes) with its
- * scratch in a 4 MiB array of the library's device code, which every device
- * that loads the library holds until the process exits.
+ * allocation after start-up.  This call takes the arguments of
+ * gptq_prepare_hinv minus ws / ws_bytes and keeps its scratch in a 4 MiB
+ * array of the library's device code, which every device that loads the
+ * library holds until the process exits.
  *   k        1 .. 12288; a larger k returns GPTQ_ERR_WORKSPACE (the built-in
  *            scratch is too small) before anything is enqueued.
- *   Setup.   The first call on a device, with that device current, looks up
- *            the array's device address (cudaGetSymbolAddress); make that
- *            first call before any stream capture.
+ *   Result.  Up to k = 4060 the tensor-core rank updates' operand splits
+ *            (1 KiB per column) fit in the array and the call runs exactly the
+ *            kernels of gptq_prepare_hinv: the outputs are bit for bit the
+ *            same.  From k = 4064 to 12288 it runs the fp32 CUDA-core rank
+ *            update instead: perm, invperm, dead and d_info are the same and
+ *            U agrees with gptq_prepare_hinv's within fp32 rounding (1e-5
+ *            relative to max |U|), not bit for bit, and the call is slower
+ *            (at k = 4096 about 4x; the CUDA-core update is the cost).
+ *   Setup.   Host code cannot hand the array's name to a kernel; its device
+ *            address comes from cudaGetSymbolAddress, looked up with the
+ *            device current on every call made outside stream capture (so a
+ *            device reset or a new context is picked up).  A call made while
+ *            `stream` is capturing reuses the address of the last call on that
+ *            device: make the first call on a device before any capture.
  *   Sharing. All calls share the array and it keeps the last call's
  *            contents (every word is written before it is read, nothing needs
  *            clearing).  Calls whose work overlaps on the GPU (other streams,
@@ -211,8 +245,10 @@ GPTQ_API gptq_status gptq_prepare_hinv_noalloc(const float* H, int64_t k, const 
  *   loss    fp64 device array of r+1 out (may be NULL; ignored when H0 is
  *           NULL): loss[0..r-1] = per-row (w0-q) H0 (w0-q)^T, loss[r] = their
  *           sum ([GPTQ-tool] Step 2 objective; Reading a quantization log).
- *   d_status int32 device scalar out (may be NULL): 0, or GPTQ_ERR_NONFINITE
- *           if a non-finite weight was met (its code is then the zero point).
+ *   d_status int32 device scalar out (may be NULL): 0, GPTQ_ERR_NONFINITE
+ *           if a non-finite weight was met (its code is then the zero point),
+ *           or GPTQ_ERR_TIMEOUT if a bounded device wait gave up (the outputs
+ *           are then unspecified).
  *   ws      GPTQ_OP_QUANTIZE workspace (holds the fp32 working copy of W).
  * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_UNSUPPORTED,
  * GPTQ_ERR_WORKSPACE, GPTQ_ERR_CUDA. */

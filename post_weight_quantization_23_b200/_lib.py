@@ -40,7 +40,10 @@ EXPORTED = (
     "gptq_dequant",
     "gptq_gemm",
     "gptq_rotate",
+    "gptq_set_wait_limit",
 )
+
+WAIT_LIMIT_DEFAULT = 0xFFFFFFFF
 
 _DTYPES = {torch.float32: GPTQ_F32, torch.float16: GPTQ_F16, torch.bfloat16: GPTQ_BF16}
 
@@ -110,6 +113,8 @@ def load(path: str = LIB_PATH):
                               vp]
     lib.gptq_rotate.restype = i32
     lib.gptq_rotate.argtypes = [vp, i32, i64, i64, i64, vp, i32, i32, vp, i64, vp]
+    lib.gptq_set_wait_limit.restype = None
+    lib.gptq_set_wait_limit.argtypes = [ctypes.c_uint32]
     _lib = lib
     return lib
 
@@ -167,6 +172,12 @@ def prepare_hinv(H, cfg, U, perm, invperm, dead, d_info, ws, stream=None):
                                   _ptr(dead), _ptr(d_info), _ptr(ws), ws.numel() * ws.element_size(),
                                   _stream(stream))
     _check(st, "gptq_prepare_hinv")
+
+
+def set_wait_limit(polls: int):
+    """Test hook (gptq_set_wait_limit): polls before a pipeline wait of the
+    tensor-core kernels gives up; WAIT_LIMIT_DEFAULT restores the default."""
+    load().gptq_set_wait_limit(int(polls) & 0xFFFFFFFF)
 
 
 def prepare_hinv_noalloc(H, cfg, U, perm, invperm, dead, d_info, stream=None):

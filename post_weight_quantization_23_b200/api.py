@@ -73,13 +73,19 @@ class GptqPlan:
             return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev) if nbytes else None
 
         self.ws_h = ws(_lib.OP_HESSIAN, hessian_tokens_hint)
+        if self.ws_h is not None:
+            self.ws_h.zero_()
         self.ws_p = ws(_lib.OP_PREPARE_HINV)
         self.ws_q = ws(_lib.OP_QUANTIZE)
         self.n_seen = 0
 
     # -- stages -----------------------------------------------------------
     def hessian_reset(self):
+        """Zero H and the Hessian workspace (whose second int32 is the sticky
+        device status word of gptq_hessian_accumulate)."""
         self.H.zero_()
+        if self.ws_h is not None:
+            self.ws_h.zero_()
         self.n_seen = 0
 
     def hessian_add(self, X: torch.Tensor, n_total: int, stream=None):
@@ -139,16 +145,29 @@ class GptqPlan:
             fn()
         return g
 
-    def check(self):
-        """Synchronise and raise on a device-reported failure."""
+    def status(self) -> dict:
+        """Synchronise and read the device status words of the three stages:
+        the Hessian workspace's status, d_info of the factor and d_status of
+        the sweep."""
         torch.cuda.synchronize(self.device)
-        info = int(self.d_info.item())
+        hs = int(self.ws_h[4:8].view(torch.int32).item()) if self.ws_h is not None else 0
+        return {"hessian": hs, "d_info": int(self.d_info.item()),
+                "d_status": int(self.d_status.item())}
+
+    def check(self):
+        """Synchronise and raise on a device-reported failure (the earliest
+        stage first: a Hessian that gave up also poisons the factor)."""
+        st = self.status()
+        if st["hessian"] != 0:
+            raise GptqError(st["hessian"], "gptq_hessian_accumulate", "bounded wait gave up")
+        info = st["d_info"]
+        if info == self.k + 1:
+            raise GptqError(_lib.GPTQ_ERR_TIMEOUT, "gptq_prepare_hinv", "bounded wait gave up")
         if info != 0:
             raise NotPositiveDefinite(_lib.GPTQ_ERR_NOT_PD, "gptq_prepare_hinv",
                                       f"pivot {info - 1} (processing order) not positive")
-        st = int(self.d_status.item())
-        if st != 0:
-            raise GptqError(st, "gptq_quantize_layer")
+        if st["d_status"] != 0:
+            raise GptqError(st["d_status"], "gptq_quantize_layer")
 
     def result(self) -> dict:
         out = dict(codes=self.codes, scales=self.scales, zeros=self.zeros, g_idx=self.g_idx,
@@ -251,7 +270,7 @@ class HostPipeline:
         self.out_zeros = torch.empty(plan.zeros.shape, dtype=plan.zeros.dtype, **pin)
         self.out_gidx = torch.empty(plan.g_idx.shape, dtype=plan.g_idx.dtype, **pin)
         self.out_loss = torch.empty(1, dtype=torch.float64, **pin)
-        self.out_status = torch.empty(2, dtype=torch.int32, **pin)
+        self.out_status = torch.empty(3, dtype=torch.int32, **pin)
 
     def h2d_bytes(self, X_host, W_host) -> int:
         return X_host.numel() * X_host.element_size() + W_host.numel() * W_host.element_size()
@@ -292,10 +311,16 @@ class HostPipeline:
                 self.out_loss.copy_(plan.loss[-1:], non_blocking=True)
             self.out_status[0:1].copy_(plan.d_info, non_blocking=True)
             self.out_status[1:2].copy_(plan.d_status, non_blocking=True)
+            if plan.ws_h is not None:
+                self.out_status[2:3].copy_(plan.ws_h[4:8].view(torch.int32), non_blocking=True)
         torch.cuda.current_stream(plan.device).wait_stream(ks)
 
     def wait(self):
         self.compute_stream.synchronize()
+        if self.plan.ws_h is not None and int(self.out_status[2]) != 0:
+            raise GptqError(int(self.out_status[2]), "gptq_hessian_accumulate")
+        if int(self.out_status[0]) == self.plan.k + 1:
+            raise GptqError(_lib.GPTQ_ERR_TIMEOUT, "gptq_prepare_hinv")
         if int(self.out_status[0]) != 0:
             raise NotPositiveDefinite(_lib.GPTQ_ERR_NOT_PD, "gptq_prepare_hinv")
         if int(self.out_status[1]) != 0:

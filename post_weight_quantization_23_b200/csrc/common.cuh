@@ -1,6 +1,7 @@
 // Shared device helpers for libgptq_b200 (sm_100a).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -44,6 +45,22 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
+
+// Process-wide runtime helpers (runtime.cu); all thread-safe.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+// The driver's cuTensorMapEncodeTiled, or nullptr when the driver lacks it.
+EncodeTiledFn tensormap_encoder();
+// Opt the kernel `func` into `bytes` of dynamic shared memory on the current
+// device (once per device and size; the error of a failed opt-in is returned).
+cudaError_t smem_optin(const void* func, size_t bytes);
+// SM count of the current device.
+int sm_count();
+// Polls after which a pipeline wait of a tensor-core kernel gives up
+// (gptq_set_wait_limit); passed to each kernel at launch.
+uint32_t wait_limit();
 
 __host__ __device__ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

@@ -81,11 +81,18 @@ hessian_simt_kernel(const T* __restrict__ X, int64_t n, int k, int64_t ldx, floa
 // H[j][i] = H[i][j] for j > i.  A nonzero *poison_flag (a device-side wait
 // of the tensor-core pass gave up) writes NaN into H[0][0] instead, so the
 // Cholesky of the next stage reports the failure.
-__global__ void mirror_upper_kernel(float* __restrict__ H, int k, const int32_t* poison_flag) {
+// Copies the upper triangle of H into the lower one.  status (may be NULL):
+// the tensor-core kernel's workspace words; when its per-call flag status[0]
+// is set (a bounded wait gave up), H[0][0] becomes NaN and the caller's
+// status word status[1] GPTQ_ERR_TIMEOUT instead.
+__global__ void mirror_upper_kernel(float* __restrict__ H, int k, int32_t* status) {
   __shared__ float tile[32][33];
   int bi = blockIdx.y, bj = blockIdx.x;
-  if (poison_flag != nullptr && *poison_flag != 0) {
-    if (bi == 0 && bj == 0 && threadIdx.x == 0 && threadIdx.y == 0) H[0] = __int_as_float(0x7fc00000);
+  if (status != nullptr && status[0] != 0) {
+    if (bi == 0 && bj == 0 && threadIdx.x == 0 && threadIdx.y == 0) {
+      H[0] = __int_as_float(0x7fc00000);
+      status[1] = (int32_t)GPTQ_ERR_TIMEOUT;
+    }
     return;
   }
   if (bj < bi) return;

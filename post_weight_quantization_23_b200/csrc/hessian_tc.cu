@@ -25,14 +25,16 @@
 //
 // Every mbarrier wait is bounded.  If one gives up, the CTA stops, waits for
 // its own copies and MMAs in flight, frees TMEM and raises a flag in the
-// workspace; the mirror pass then writes NaN into H[0][0] so that the next
-// stage (the Cholesky in gptq_prepare_hinv) reports the failure.
+// workspace; the mirror pass then sets the caller's status word (the
+// workspace's second int32) to GPTQ_ERR_TIMEOUT and writes NaN into H[0][0],
+// so that a caller who never reads the word still sees the failure in the next
+// stage (the Cholesky in gptq_prepare_hinv).
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
 namespace gptq {
 
-__global__ void mirror_upper_kernel(float* __restrict__ H, int k, const int32_t* poison_flag);
+__global__ void mirror_upper_kernel(float* __restrict__ H, int k, int32_t* status);
 
 namespace {
 
@@ -57,6 +59,7 @@ struct HtArgs {
   float alpha;
   float* H;
   int32_t* status;
+  uint32_t spin;  // polls before a pipeline wait gives up
 };
 
 __device__ __forceinline__ void decode_tile(int t, int nI, int nJ, int& I, int& J) {
@@ -128,7 +131,7 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HtArgs a, int fmt_bf
         const int64_t t_end = min(a.n, t_beg + a.chunk);
         const int nst = (int)((t_end - t_beg + HT_KT - 1) / HT_KT);
         for (int st = 0; st < nst; ++st) {
-          if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.spin)) { ok = false; break; }
           uint8_t* sb = stages + (size_t)stage * HT_STAGE_BYTES;
           tc::mbar_arrive_expect_tx(&full[stage], a_in_b ? HT_B_BYTES : HT_STAGE_BYTES);
           const int32_t tok = (int32_t)(t_beg + (int64_t)st * HT_KT);
@@ -174,12 +177,12 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HtArgs a, int fmt_bf
         const int64_t t_end = min(a.n, t_beg + a.chunk);
         const int nst = (int)((t_end - t_beg + HT_KT - 1) / HT_KT);
         for (int s0 = 0; s0 < nst && ok; s0 += HT_SUB_STAGES) {
-          if (!tc::mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!tc::mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, a.spin)) { ok = false; break; }
           tc::tc_fence_after();
           const uint32_t dcol = tmem + (uint32_t)(tb * HT_N);
           const int s1 = min(nst, s0 + HT_SUB_STAGES);
           for (int st = s0; st < s1; ++st) {
-            if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+            if (!tc::mbar_wait(&full[stage], phase, abort_flag, a.spin)) { ok = false; break; }
             tc::tc_fence_after();
             const uint32_t sb = tc::smem_u32(stages + (size_t)stage * HT_STAGE_BYTES);
             const uint32_t a_base = a_in_b ? sb + (uint32_t)((i0 - j0) / 64) * HT_BOX_BYTES
@@ -226,7 +229,7 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HtArgs a, int fmt_bf
 #pragma unroll
       for (int q = 0; q < 128; ++q) acc[q] = 0.f;
       for (int sub = 0; sub < nsub; ++sub) {
-        if (!tc::mbar_wait(&tfull[tb], tphase, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(&tfull[tb], tphase, abort_flag, a.spin)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t base =
             tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(tb * HT_N + half * 128);
@@ -263,38 +266,20 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HtArgs a, int fmt_bf
   if (warp == 1) tc::tmem_dealloc(tmem, HT_TMEM_COLS);
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)p;
-  }
-  return fn;
-}
-
 }  // namespace
 
 bool hessian_tc_supported(gptq_dtype dt, int64_t n, int64_t k, int64_t ldx, const void* X) {
   if (dt != GPTQ_F16 && dt != GPTQ_BF16) return false;
   if (k < 64 || k % 8 != 0 || ldx % 8 != 0 || ((uintptr_t)X % 16) != 0) return false;
   if (n <= 0 || n > ((int64_t)1 << 31) - HT_MAX_CHUNK) return false;
-  return encode_fn() != nullptr;
+  return tensormap_encoder() != nullptr;
 }
 
 size_t hessian_tc_workspace_bytes(int64_t, int64_t) { return 256; }
 
 gptq_status hessian_tc(const void* X, gptq_dtype dt, int64_t n, int64_t k, int64_t ldx,
                        float alpha, float* H, void* ws, cudaStream_t s) {
-  EncodeTiledFn enc = encode_fn();
+  EncodeTiledFn enc = tensormap_encoder();
   if (enc == nullptr) return GPTQ_ERR_UNSUPPORTED;
   CUtensorMap map;
   cuuint64_t gdim[2] = {(cuuint64_t)k, (cuuint64_t)n};
@@ -308,16 +293,8 @@ gptq_status hessian_tc(const void* X, gptq_dtype dt, int64_t n, int64_t k, int64
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return GPTQ_ERR_INVALID_ARG;
 
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)HT_SMEM) != cudaSuccess)
-      return GPTQ_ERR_CUDA;
-    attr_set = true;
-  }
+  const int nsm = sm_count();
+  if (smem_optin((const void*)hessian_tc_kernel, HT_SMEM) != cudaSuccess) return GPTQ_ERR_CUDA;
   HtArgs a;
   a.k = (int)k;
   a.n = n;
@@ -334,12 +311,14 @@ gptq_status hessian_tc(const void* X, gptq_dtype dt, int64_t n, int64_t k, int64
   a.alpha = alpha;
   a.H = H;
   a.status = (int32_t*)ws;
-  cudaMemsetAsync(ws, 0, sizeof(int32_t), s);
+  a.spin = wait_limit();
+  // word 0: this call's give-up flag; word 1 (the caller's status) is only ever set
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), s) != cudaSuccess) return GPTQ_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(a.nunits, nsm);
   hessian_tc_kernel<<<grid, HT_THREADS, HT_SMEM, s>>>(map, a, dt == GPTQ_BF16 ? 1 : 0);
   GPTQ_CHECK_LAUNCH();
   int nb = (int)cdiv(k, 32);
-  mirror_upper_kernel<<<dim3(nb, nb), dim3(32, 8), 0, s>>>(H, (int)k, (const int32_t*)ws);
+  mirror_upper_kernel<<<dim3(nb, nb), dim3(32, 8), 0, s>>>(H, (int)k, (int32_t*)ws);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
 }

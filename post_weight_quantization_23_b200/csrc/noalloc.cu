@@ -12,16 +12,21 @@
 //
 // The array is `kScratchBytes` (4 MiB) on every device that loads the
 // library and is held until the process exits; it covers k up to
-// kNoAllocMaxK = 12288 (when the tensor-core update's operand splits do not
-// fit as well, the CUDA-core update is used).  All calls share it and it keeps the previous call's
+// kNoAllocMaxK = 12288.  Up to k = 4060 the tensor-core rank updates' operand
+// splits fit beside the rest and the kernels are those of gptq_prepare_hinv
+// (bit-identical results); above, the fp32 CUDA-core rank update runs instead
+// (same result within fp32 rounding, slower).  All calls share it and it keeps the previous call's
 // contents; the Cholesky stages write every scratch word before reading it,
 // so nothing needs clearing.  Calls whose work overlaps on the GPU (two
 // streams, or two host threads) race on the array: serialise them.
 //
 // Host code cannot pass the array's name to a kernel (on the host it is only
-// a stand-in for the device symbol).  The device address is looked up once
-// per device with cudaGetSymbolAddress, with that device current, on the
-// first call made on it; make that first call before any stream capture.
+// a stand-in for the device symbol).  The device address comes from
+// cudaGetSymbolAddress with the device current, on every call made outside
+// stream capture (so a device reset or a context re-created since the last
+// call gets the fresh address); a call made while its stream is capturing
+// reuses the address of the last call on that device, so the first call on a
+// device must come before any capture.
 #include <mutex>
 
 #include "common.cuh"
@@ -44,16 +49,20 @@ constexpr int kMaxDevices = 128;
 void* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-gptq_status scratch_address(void** out) {
+gptq_status scratch_address(cudaStream_t stream, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return GPTQ_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return GPTQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_hinv_scratch) != cudaSuccess || p == nullptr)
       return GPTQ_ERR_CUDA;
     g_scratch_addr[dev] = p;
+  } else if (g_scratch_addr[dev] == nullptr) {
+    return GPTQ_ERR_CUDA;  // first call on this device inside a capture
   }
   *out = g_scratch_addr[dev];
   return GPTQ_OK;
@@ -74,7 +83,7 @@ extern "C" gptq_status gptq_prepare_hinv_noalloc(const float* H, int64_t k,
   // sizes beyond the built-in scratch
   if (k > kNoAllocMaxK || gptq::hinv_workspace_min_bytes(k) > kScratchBytes) return GPTQ_ERR_WORKSPACE;
   void* ws = nullptr;
-  gptq_status st = scratch_address(&ws);
+  gptq_status st = scratch_address((cudaStream_t)stream, &ws);
   if (st != GPTQ_OK) return st;
   return gptq::prepare_hinv_impl(H, k, cfg, U, perm, invperm, dead, d_info, ws, kScratchBytes,
                                  (cudaStream_t)stream);

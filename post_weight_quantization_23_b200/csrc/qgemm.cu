@@ -307,14 +307,10 @@ gptq_status launch_qgemv(const T* X, int64_t ldx, int m, int k, const int32_t* q
   using Sh = QvShape<BITS>;
   const int KC = qv_kc(k, Sh::SLAB);
   const size_t smem = qv_smem_bytes<BITS>(M, KC);
-  static size_t smem_set = 48 * 1024;  // opt-in limit set so far for this instantiation
-  if (smem > smem_set) {
-    const size_t most = qv_smem_bytes<BITS>(M, QV_KC);
-    if (cudaFuncSetAttribute(qgemv_kernel<BITS, M, T>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most) != cudaSuccess)
-      return GPTQ_ERR_CUDA;
-    smem_set = most;
-  }
+  // opt in once per device to the most this instantiation can ask for
+  if (smem > 48 * 1024 &&
+      smem_optin((const void*)qgemv_kernel<BITS, M, T>, qv_smem_bytes<BITS>(M, QV_KC)) != cudaSuccess)
+    return GPTQ_ERR_CUDA;
   const dim3 grid((unsigned)cdiv(n, QV_ROWS), (unsigned)cdiv(m, M));
   // 16-byte activation loads when every row of X starts on a 16-byte boundary
   const int xvec = ((uintptr_t)X % 16) == 0 && ldx % 8 == 0;

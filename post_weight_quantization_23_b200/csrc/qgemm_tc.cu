@@ -49,6 +49,7 @@ struct QtArgs {
   void* Y;
   int64_t ldy;
   int n, m, k, G, ngroups;
+  uint32_t spin;  // polls before a pipeline wait gives up
 };
 
 // The 16-bit activation type T and its packed pair T2.
@@ -125,7 +126,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
       for (int kc = 0; kc < nk && ok; ++kc) {
         const int s = kc % QT_STAGES;
         const uint32_t ph = (uint32_t)(kc / QT_STAGES) & 1u;
-        if (!tc::mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.spin)) { ok = false; break; }
         tc::mbar_arrive_expect_tx(&full_tma[s], QT_P_BYTES + QT_B_BYTES);
         tc::tma_load_2d(stage_p(s), &pmap, &full_tma[s], kc * (QT_K / 8), n0);
         tc::tma_load_2d(stage_b(s), &xmap, &full_tma[s], kc * QT_K, t0);
@@ -144,8 +145,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
       for (int kc = 0; kc < nk; ++kc) {
         const int s = kc % QT_STAGES;
         const uint32_t ph = (uint32_t)(kc / QT_STAGES) & 1u;
-        if (!tc::mbar_wait(&full_tma[s], ph, abort_flag)) break;
-        if (!tc::mbar_wait(&full_a[s], ph, abort_flag)) break;
+        if (!tc::mbar_wait(&full_tma[s], ph, abort_flag, a.spin)) break;
+        if (!tc::mbar_wait(&full_a[s], ph, abort_flag, a.spin)) break;
         tc::tc_fence_after();
         const uint32_t sa = tc::smem_u32(stage_a(s)), sb = tc::smem_u32(stage_b(s));
 #pragma unroll
@@ -185,7 +186,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
       const int s = kc % QT_STAGES;
       const uint32_t ph = (uint32_t)(kc / QT_STAGES) & 1u;
       fetch(kc + 2, s_2, z_2);
-      if (!tc::mbar_wait(&full_tma[s], ph, abort_flag)) break;
+      if (!tc::mbar_wait_warp(&full_tma[s], ph, abort_flag, a.spin)) break;
       const uint4 pw = reinterpret_cast<const uint4*>(stage_p(s) + r * 32)[hf];
       const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
       const T2 sc2 = as_t2<T2>(s_c), zz2 = as_t2<T2>(z_c);
@@ -210,7 +211,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
       s_c = s_1, z_c = z_1, s_1 = s_2, z_1 = z_2;
     }
     // epilogue: this warp's lane quarter, tokens [128 hf, 128 hf + 128)
-    const bool ok = tc::mbar_wait(done, 0, abort_flag) && !*abort_flag;
+    const bool ok = tc::mbar_wait_warp(done, 0, abort_flag, a.spin) && !*abort_flag;
     tc::tc_fence_after();
     const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
     for (int c = 4 * hf; c < 4 * hf + 4; ++c) {
@@ -237,23 +238,6 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
   if (warp == 1) tc::tmem_dealloc(tmem, QT_TMEM_COLS);
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn qt_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)p;
-  }
-  return fn;
-}
 
 }  // namespace
 
@@ -263,13 +247,13 @@ EncodeTiledFn qt_encode_fn() {
 bool qgemm_tc_supported(const void* X, int64_t ldx, const int32_t* qw, int bits, int64_t k,
                         int G, bool has_gidx) {
   return bits == 4 && !has_gidx && k >= QT_K && (G >= k || G % 32 == 0) && ((uintptr_t)X % 16) == 0 &&
-         ((uintptr_t)qw % 16) == 0 && ldx % 8 == 0 && qt_encode_fn() != nullptr;
+         ((uintptr_t)qw % 16) == 0 && ldx % 8 == 0 && tensormap_encoder() != nullptr;
 }
 
 gptq_status qgemm_tc(const void* X, bool bf16, int64_t m, int64_t k, int64_t ldx,
                      const int32_t* qw, const float* scales, const int32_t* zeros, int64_t n,
                      int G, int64_t ngroups, void* Y, int64_t ldy, cudaStream_t s) {
-  EncodeTiledFn enc = qt_encode_fn();
+  EncodeTiledFn enc = tensormap_encoder();
   if (enc == nullptr) return GPTQ_ERR_CUDA;
   CUtensorMap xmap, pmap;
   {
@@ -293,21 +277,16 @@ gptq_status qgemm_tc(const void* X, bool bf16, int64_t m, int64_t k, int64_t ldx
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return GPTQ_ERR_CUDA;
   }
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(qgemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)QT_SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(qgemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)QT_SMEM) != cudaSuccess)
-      return GPTQ_ERR_CUDA;
-    attr = true;
-  }
+  if (smem_optin(bf16 ? (const void*)qgemm_tc_kernel<true> : (const void*)qgemm_tc_kernel<false>,
+                 QT_SMEM) != cudaSuccess)
+    return GPTQ_ERR_CUDA;
   QtArgs a;
   a.scales = scales;
   a.zeros = zeros;
   a.Y = Y;
   a.ldy = ldy;
   a.n = (int)n, a.m = (int)m, a.k = (int)k, a.G = G, a.ngroups = (int)ngroups;
+  a.spin = wait_limit();
   const dim3 grid((unsigned)cdiv(n, QT_M), (unsigned)cdiv(m, QT_N));
   if (bf16)
     qgemm_tc_kernel<true><<<grid, QT_THREADS, QT_SMEM, s>>>(xmap, pmap, a);

@@ -411,6 +411,7 @@ struct SqArgs {
   uint8_t* codes;
   double* loss;
   int32_t* d_status;
+  uint32_t spin;  // polls before the record wait gives up
 };
 
 template <int L>
@@ -632,7 +633,7 @@ __global__ void __launch_bounds__(SQ_MAX_WARPS * 32, 1) sweep_block_lane_kernel(
   st.hi_d = a.maxq - st.zero;
   st.e2 = 0.0;
   st.nonfinite = false;
-  if (!tc::mbar_wait(bar, 0, abort_flag)) {
+  if (!tc::mbar_wait(bar, 0, abort_flag, a.spin)) {
     // the record never arrived: let the copy land (bounded) and report
     for (uint32_t i = 0; i < tc::kSpinLimit; ++i)
       if (tc::mbar_try_wait(bar, 0)) break;
@@ -704,36 +705,31 @@ __global__ void loss_total_kernel(double* __restrict__ loss, int r) {
 }
 
 template <int SB>
-static void launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* Err,
-                         float* Err_lo, const float* U, const int32_t* perm, int r, int k, int s0,
-                         int bw, int B, int G, int ngroups, float maxq, int sym, float* scales,
-                         int32_t* zeros, uint8_t* codes, double* loss, int32_t* d_status) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(sweep_block_kernel<SB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)SW_SMEM);
-    attr = true;
-  }
+static gptq_status launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* Err,
+                                float* Err_lo, const float* U, const int32_t* perm, int r, int k,
+                                int s0, int bw, int B, int G, int ngroups, float maxq, int sym,
+                                float* scales, int32_t* zeros, uint8_t* codes, double* loss,
+                                int32_t* d_status) {
+  if (smem_optin((const void*)sweep_block_kernel<SB>, SW_SMEM) != cudaSuccess) return GPTQ_ERR_CUDA;
   sweep_block_kernel<SB><<<grid, SW_THREADS, SW_SMEM, s>>>(Wt, Err, Err_lo, U, perm, r, k, s0, bw,
                                                            B, G, ngroups, maxq, sym, scales,
                                                            zeros, codes, loss, d_status);
+  return GPTQ_OK;
 }
 
 // pdl: launch early behind the previous kernel (every block but the first,
 // whose record may still be in flight from the kernel right before it)
 template <int L, int MODE>
-static void launch_lane(unsigned grid, int threads, cudaStream_t s, const SqArgs& a, bool pdl) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(sweep_block_lane_kernel<L, MODE>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SqLayout<L>::SMEM);
-    attr = true;
-  }
+static gptq_status launch_lane(unsigned grid, int threads, cudaStream_t s, const SqArgs& a,
+                               bool pdl) {
+  if (smem_optin((const void*)sweep_block_lane_kernel<L, MODE>, SqLayout<L>::SMEM) != cudaSuccess)
+    return GPTQ_ERR_CUDA;
   if (pdl)
     launch_pdl(sweep_block_lane_kernel<L, MODE>, dim3(grid), dim3(threads), SqLayout<L>::SMEM, s,
                a);
   else
     sweep_block_lane_kernel<L, MODE><<<grid, threads, SqLayout<L>::SMEM, s>>>(a);
+  return GPTQ_OK;
 }
 
 template <typename T>
@@ -783,9 +779,7 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
   int q_warps = 1;
   unsigned q_grid = 0;
   if (lane_mode >= 0) {
-    int dev = 0, nsm = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int nsm = sm_count();
     if ((lane_mode == 1 && G % 8 != 0) || cdiv(r, 8) >= (int64_t)nsm * 8) lanes = 4;
     const int64_t warps = cdiv(r, 32 / lanes);
     q_warps = (int)std::min<int64_t>(SQ_MAX_WARPS, std::max<int64_t>(1, cdiv(warps, nsm)));
@@ -824,20 +818,24 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
       a.codes = codes;
       a.loss = lossp;
       a.d_status = d_status;
+      a.spin = wait_limit();
       // right behind a trailing update (not behind a group grid launch)
       const bool pdl = b > 0 && !(!stat && G > B && s0 % G == 0);
+      gptq_status st;
       if (lanes == 8) {
-        if (lane_mode == 0) launch_lane<8, 0>(q_grid, 32 * q_warps, s, a, pdl);
-        else if (lane_mode == 1) launch_lane<8, 1>(q_grid, 32 * q_warps, s, a, pdl);
-        else launch_lane<8, 2>(q_grid, 32 * q_warps, s, a, pdl);
+        if (lane_mode == 0) st = launch_lane<8, 0>(q_grid, 32 * q_warps, s, a, pdl);
+        else if (lane_mode == 1) st = launch_lane<8, 1>(q_grid, 32 * q_warps, s, a, pdl);
+        else st = launch_lane<8, 2>(q_grid, 32 * q_warps, s, a, pdl);
       } else {
-        if (lane_mode == 0) launch_lane<4, 0>(q_grid, 32 * q_warps, s, a, pdl);
-        else if (lane_mode == 1) launch_lane<4, 1>(q_grid, 32 * q_warps, s, a, pdl);
-        else launch_lane<4, 2>(q_grid, 32 * q_warps, s, a, pdl);
+        if (lane_mode == 0) st = launch_lane<4, 0>(q_grid, 32 * q_warps, s, a, pdl);
+        else if (lane_mode == 1) st = launch_lane<4, 1>(q_grid, 32 * q_warps, s, a, pdl);
+        else st = launch_lane<4, 2>(q_grid, 32 * q_warps, s, a, pdl);
       }
+      if (st != GPTQ_OK) return st;
     } else {
+      gptq_status st = GPTQ_OK;
 #define GPTQ_SWEEP_BLOCK(SBV)                                                                  \
-  launch_block<SBV>(grid, s, sc.Wt, sc.Err, err_lo, U, perm, r, k, s0, bw, B, G, ngroups, maxq, \
+  st = launch_block<SBV>(grid, s, sc.Wt, sc.Err, err_lo, U, perm, r, k, s0, bw, B, G, ngroups, maxq, \
                     cfg->sym, scales, zeros, codes, lossp, d_status)
       switch (SB) {
         case 16: GPTQ_SWEEP_BLOCK(16); break;
@@ -847,6 +845,7 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
         default: GPTQ_SWEEP_BLOCK(1); break;
       }
 #undef GPTQ_SWEEP_BLOCK
+      if (st != GPTQ_OK) return st;
     }
     GPTQ_CHECK_LAUNCH();
     int e0 = s0 + bw;

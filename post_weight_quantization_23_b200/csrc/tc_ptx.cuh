@@ -10,7 +10,10 @@ namespace gptq {
 namespace tc {
 
 // Bound on every spin-wait: after this many polls a wait gives up and the
-// caller takes its error path (a correct kernel never gets near it).
+// caller takes its error path (a correct kernel never gets near it).  The
+// pipeline waits take their limit from the launch (gptq_set_wait_limit can
+// lower it); the drain waits that let a CTA's own copies and MMAs land before
+// it exits always use this one.
 constexpr uint32_t kSpinLimit = 1u << 26;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -51,16 +54,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.  Returns
-// false if it gave up (or *abort became nonzero).
+// Bounded wait for the phase with the given parity to complete: at most
+// `limit` polls.  Returns false if it gave up (then *abort_flag is set) or
+// *abort_flag became nonzero.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+                                          volatile int* abort_flag, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 1023u) == 1023u && *abort_flag) return false;
   }
   *abort_flag = 1;
   return false;
+}
+
+// mbar_wait by every lane of a converged warp with one outcome for the whole
+// warp: if any lane gave up, every lane returns false, so the warp leaves its
+// loop together and its later .sync.aligned instructions (tcgen05.ld, wait)
+// stay converged.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort_flag, uint32_t limit) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, limit);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // 2-D TMA tile load into shared memory, completing on `bar` (bytes counted

@@ -63,6 +63,7 @@ struct TxArgs {
   int mode, split;
   int32_t* status;
   int32_t status_code;
+  uint32_t spin;  // polls before a pipeline wait gives up
 };
 
 __device__ __forceinline__ bool tile_skipped(const TxArgs& a, int m0, int n0) {
@@ -144,7 +145,7 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
         const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
         if (tile_skipped(a, m0, n0)) continue;
         for (int kc = 0; kc < nkc; ++kc) {
-          if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.spin)) { ok = false; break; }
           uint8_t* sb = smem + (size_t)stage * TX_STAGE_BYTES;
           tc::mbar_arrive_expect_tx(&full[stage], TX_STAGE_BYTES);
           const int k0 = kc * TX_KC;
@@ -175,11 +176,11 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
       for (int t = blockIdx.x; t < a.ntiles && ok; t += gridDim.x) {
         const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
         if (tile_skipped(a, m0, n0)) continue;
-        if (!tc::mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, a.spin)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t dcol = tmem + (uint32_t)(tb * TX_N);
         for (int kc = 0; kc < nkc; ++kc) {
-          if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          if (!tc::mbar_wait(&full[stage], phase, abort_flag, a.spin)) { ok = false; break; }
           tc::tc_fence_after();
           const uint32_t sb = tc::smem_u32(smem + (size_t)stage * TX_STAGE_BYTES);
           const uint32_t ah = sb, al = sb + TX_A_BYTES;
@@ -217,7 +218,7 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
     bool ok = true;
     for (int t = next_tile(a, -1); t < a.ntiles && ok; t = next_tile(a, t)) {
       const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
-      if (!tc::mbar_wait(&tfull[tb], tphase, abort_flag)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(&tfull[tb], tphase, abort_flag, a.spin)) { ok = false; break; }
       tc::tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(tb * TX_N);
       float v[32];
@@ -227,7 +228,8 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
         const int slot = g % TX_D_SLOTS;
         if (g >= TX_D_SLOTS) {
           // the slot's previous reduce must have read it
-          if (!tc::mbar_wait(&dfree[slot], (uint32_t)((g / TX_D_SLOTS) - 1) & 1u, abort_flag)) {
+          if (!tc::mbar_wait_warp(&dfree[slot], (uint32_t)((g / TX_D_SLOTS) - 1) & 1u, abort_flag,
+                                  a.spin)) {
             ok = false;
             break;
           }
@@ -247,17 +249,23 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
         tc::fence_proxy_async_smem();  // the reduce reads what this thread wrote
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&dwritten[slot]);
+        bool gave_up = false;
         if (dprod) {
-          if (!tc::mbar_wait(&dwritten[slot], (uint32_t)(g / TX_D_SLOTS) & 1u, abort_flag)) {
-            ok = false;
-            break;
+          if (tc::mbar_wait(&dwritten[slot], (uint32_t)(g / TX_D_SLOTS) & 1u, abort_flag, a.spin)) {
+            tc::tma_reduce_add_2d(&d_map, ring + slot * TX_D_BYTES, a.col0 + n0 + cc * TX_DC,
+                                  a.row0 + m0);
+            tc::bulk_commit_group();
+            // free the other slot for the chunk after next once its reduce has read it
+            tc::bulk_wait_read_1();
+            if (g >= 1) tc::mbar_arrive(&dfree[(g - 1) % TX_D_SLOTS]);
+          } else {
+            gave_up = true;
           }
-          tc::tma_reduce_add_2d(&d_map, ring + slot * TX_D_BYTES, a.col0 + n0 + cc * TX_DC,
-                                a.row0 + m0);
-          tc::bulk_commit_group();
-          // free the other slot for the chunk after next once its reduce has read it
-          tc::bulk_wait_read_1();
-          if (g >= 1) tc::mbar_arrive(&dfree[(g - 1) % TX_D_SLOTS]);
+        }
+        // the reduce thread's warp leaves the loop together with it
+        if (__shfl_sync(0xffffffffu, gave_up, 0)) {
+          ok = false;
+          break;
         }
       }
       if (++tb == 2) tb = 0, tphase ^= 1u;
@@ -271,28 +279,11 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
   if (warp == 1) tc::tmem_dealloc(tmem, TX_TMEM_COLS);
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)p;
-  }
-  return fn;
-}
 
 // fp32 2-D map (cols inner, rows outer), row stride ld floats, box {32, box_rows}.
 bool make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int64_t ld,
               uint32_t box_rows) {
-  EncodeTiledFn enc = encode_fn();
+  EncodeTiledFn enc = tensormap_encoder();
   if (enc == nullptr) return false;
   cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t gstride[1] = {(cuuint64_t)ld * 4};
@@ -305,16 +296,9 @@ bool make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int
 
 gptq_status launch(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMap& bh,
                    const CUtensorMap& bl, const CUtensorMap& dm, TxArgs& a, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(tf32x3_update_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TX_SMEM) != cudaSuccess)
-      return GPTQ_ERR_CUDA;
-    attr = true;
-  }
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (smem_optin((const void*)tf32x3_update_kernel, TX_SMEM) != cudaSuccess) return GPTQ_ERR_CUDA;
+  a.spin = wait_limit();
+  const int nsm = sm_count();
   const int grid = std::min(a.ntiles, nsm);
   if (grid <= 0) return GPTQ_OK;
   launch_pdl(tf32x3_update_kernel, dim3(grid), dim3(TX_THREADS), TX_SMEM, s, ah, al, bh, bl, dm,
@@ -362,7 +346,7 @@ __global__ void split_transpose_kernel(const float* __restrict__ src, int64_t ld
 
 }  // namespace
 
-bool tc_update_supported(int64_t k) { return k % 4 == 0 && encode_fn() != nullptr; }
+bool tc_update_supported(int64_t k) { return k % 4 == 0 && tensormap_encoder() != nullptr; }
 
 gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float sign,
                                int upper_only, float* hi, float* lo, int64_t ldo, cudaStream_t s) {

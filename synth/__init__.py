@@ -93,6 +93,10 @@ def stack_spec(sublayer, tokens=STACK_TOKENS):
     raise KeyError(sublayer)
 
 
+for _name, _r, _k, _stream in STACK_LAYER:
+    CONFIGS[f"stack_{_name}"] = stack_spec(_name)
+
+
 def tensor_seed(seed, layer, tensor_id):
     """Per-tensor seed: seed*1000 + layer*10 + tensor_id."""
     return int(seed) * 1000 + int(layer) * 10 + int(tensor_id)
@@ -172,3 +176,37 @@ def make_x(spec: LayerSpec, seed: int, layer: int = 0, t0: int = 0, t1: int | No
 
 def dtype_of(name: str) -> torch.dtype:
     return _DT[name]
+
+
+def make_x_device(spec: LayerSpec, seed: int, device, layer: int = 0) -> torch.Tensor:
+    """X (n, k) of the same distribution as ``make_x``, drawn on the device with
+    the device's generator (fast; the bytes differ from ``make_x``, so this is
+    for timing runs only, never for a comparison with the oracle)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(tensor_seed(seed, layer, 5))
+    dt = _DT[spec.x_dtype]
+    out = torch.empty(spec.n, spec.k, dtype=dt, device=device)
+    if spec.x_kind == "lognormal":
+        c = channel_scales(spec, seed, layer).to(device=device, dtype=torch.float32)
+    elif spec.x_kind == "mixed":
+        L = mixing_matrix(spec, seed, layer).to(device=device, dtype=torch.float32)
+    step = 16384
+    for a in range(0, spec.n, step):
+        rows = min(step, spec.n - a)
+        if spec.x_kind == "lognormal":
+            z = torch.randn(rows, spec.k, generator=g, device=device) * c
+        elif spec.x_kind == "silu":
+            z = torch.nn.functional.silu(torch.randn(rows, spec.k, generator=g, device=device))
+            z *= torch.randn(rows, spec.k, generator=g, device=device)
+        else:
+            z = torch.randn(rows, spec.k, generator=g, device=device) @ L
+        out[a:a + rows] = z.to(dt)
+    return out
+
+
+def make_w_device(spec: LayerSpec, seed: int, device, layer: int = 0) -> torch.Tensor:
+    """W (r, k) ~ N(0, w_std^2) drawn on the device (timing runs only)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(tensor_seed(seed, layer, 6))
+    w = torch.randn(spec.r, spec.k, generator=g, device=device) * spec.w_std
+    return w.to(_DT[spec.w_dtype])

@@ -46,6 +46,7 @@ def gpu_quantize(W, X, cfg, chunk_tokens=8192, deq_dtype=torch.float32):
 class Agreement:
     h_rel_fro: float
     u_rel_max: float
+    u_row_rel: float
     code_match: float
     n_forced: int
     replay_mismatch: int
@@ -80,9 +81,10 @@ def compare(gpu, W_np, X_np, cfg, rows=None, H=None):
     gperm = gpu["perm"].numpy().astype(np.int64)
     sym = bool(getattr(cfg, "sym", False))
     stat = bool(getattr(cfg, "static_groups", False))
-    own = O.gptq(Wc[:1], H, cfg.bits, cfg.group_size, cfg.block_size, cfg.percdamp, cfg.act_order,
-                 sym=sym, static_groups=stat)
-    perm_diff = int((own["perm"] != gperm).sum())
+    # the oracle's own act-order (before accepting the GPU's tie-equivalent one)
+    Hf = O.fix_dead_columns(H, Wc[:1])[0]
+    own_perm = O.act_order_perm(Hf) if cfg.act_order else np.arange(H.shape[0])
+    perm_diff = int((own_perm != gperm).sum())
     # the act-order permutation is decided from floating-point diag(H): the
     # oracle takes the GPU's order where (and only where) it is a valid order
     # within the Hessian tolerance; everything downstream is then compared
@@ -99,10 +101,13 @@ def compare(gpu, W_np, X_np, cfg, rows=None, H=None):
     perm_equal = bool(np.array_equal(gperm, ref["perm"]))
     U = gpu["U"].double().numpy()
     u_rel = float(np.abs(U - ref["U"]).max() / np.abs(ref["U"]).max())
+    # per row of U relative to that row (the sweep uses U[i, j] / U[i, i])
+    u_row = float(np.max(np.linalg.norm(U - ref["U"], axis=1) / np.linalg.norm(ref["U"], axis=1)))
     loss_g = gpu["loss_rows"].numpy()[sel].sum()
     return Agreement(
         h_rel_fro=h_rel,
         u_rel_max=u_rel,
+        u_row_rel=u_row,
         code_match=float((codes == ref["codes"]).mean()),
         n_forced=int(rep["n_forced"]),
         replay_mismatch=int((codes != rep["codes"]).sum()),

@@ -59,6 +59,9 @@ CASES = {
     # k not a multiple of 4: CUDA-core trailing and rank updates
     "k150_cuda_core": synth.CONFIGS["tiny"].scaled(r=40, k=150, n=2000, group_size=-1,
                                                    block_size=32),
+    # the same at a width of 9 row tiles (the triangular tile decode of the
+    # CUDA-core rank update), act-order, a ragged last group and block
+    "k1030_cuda_core": synth.CONFIGS["down_proj"].scaled(r=96, k=1030, n=8192),
 }
 
 

@@ -82,6 +82,37 @@ def test_noalloc_matches_workspace_entry_two_calls_in_a_row():
     assert list(np.flatnonzero(got2[3].numpy())) == [5, 400]
 
 
+def _gpu_hessian(spec, seed):
+    """H of a seeded layer from the library's own Hessian call (both entry
+    points under test then factor the same bytes)."""
+    from post_weight_quantization_23_b200 import _lib
+    X = synth.make_x(spec, seed).cuda()
+    H = torch.zeros(spec.k, spec.k, device="cuda")
+    ws = torch.zeros(_lib.workspace_size(_lib.OP_HESSIAN, 0, spec.k, spec.n, None),
+                     dtype=torch.uint8, device="cuda")
+    _lib.hessian_accumulate(X, H, 2.0 / spec.n, ws)
+    torch.cuda.synchronize()
+    return H
+
+
+@pytest.mark.parametrize("name,k", [("q_proj", 4096), ("opt175_width", 12288)])
+def test_noalloc_cuda_core_update_at_full_width(name, k):
+    """From k = 4064 the operand splits of the tensor-core rank update no
+    longer fit in the built-in scratch, so the call takes the fp32 CUDA-core
+    rank update (a triangular tile schedule over several row tiles): at the
+    q_proj width and at the OPT-175B width, twice in a row, against the
+    workspace entry point's tensor-core result."""
+    from post_weight_quantization_23_b200 import _lib
+    spec = synth.CONFIGS[name].scaled(r=64, k=k, n=16384)
+    H = _gpu_hessian(spec, 21)
+    for act_order in (False, True):
+        cfg = _lib.make_config(spec.bits, spec.group_size, spec.block_size, 0.01, act_order)
+        ref, got = _both(H, cfg)
+        rel = float((got[0].double() - ref[0].double()).abs().max() / ref[0].double().abs().max())
+        print(f"k={k} act_order={act_order}: max |dU| / max |U| = {rel:.3e}")
+        _assert_match(ref, got)
+
+
 def test_noalloc_rejects_k_beyond_its_scratch():
     from post_weight_quantization_23_b200 import _lib
     lib = _lib.load()
