@@ -199,14 +199,14 @@ GPTQ_API void gptq_set_wait_limit(uint32_t polls);
  * library holds until the process exits.
  *   k        1 .. 12288; a larger k returns GPTQ_ERR_WORKSPACE (the built-in
  *            scratch is too small) before anything is enqueued.
- *   Result.  Up to k = 4060 the tensor-core rank updates' operand splits
- *            (1 KiB per column) fit in the array and the call runs exactly the
- *            kernels of gptq_prepare_hinv: the outputs are bit for bit the
- *            same.  From k = 4064 to 12288 it runs the fp32 CUDA-core rank
- *            update instead: perm, invperm, dead and d_info are the same and
- *            U agrees with gptq_prepare_hinv's within fp32 rounding (1e-5
- *            relative to max |U|), not bit for bit, and the call is slower
- *            (at k = 4096 about 4x; the CUDA-core update is the cost).
+ *   Result.  perm, invperm, dead and d_info are those of
+ *            gptq_prepare_hinv; U agrees with its U within fp32 rounding
+ *            (1e-5 relative to max |U|), not bit for bit, because the array
+ *            holds less of the rank updates' operand splits than the
+ *            workspace does: up to k = 4060 the tensor-core updates run with
+ *            one level of 64-column blocks (gptq_prepare_hinv batches 8 of
+ *            them per update), and from k = 4064 to 12288 the fp32 CUDA-core
+ *            rank update runs instead, which is slower (at k = 4096 about 4x).
  *   Setup.   Host code cannot hand the array's name to a kernel; its device
  *            address comes from cudaGetSymbolAddress, looked up with the
  *            device current on every call made outside stream capture (so a

@@ -16,7 +16,7 @@ size_t hinv_workspace_bytes(int64_t k);
 gptq_status prepare_hinv_impl(const float* H, int64_t k, const gptq_config* cfg, float* U,
                               int32_t* perm, int32_t* invperm, uint8_t* dead, int32_t* d_info,
                               void* ws, size_t ws_bytes, cudaStream_t s);
-size_t sweep_workspace_bytes(int64_t r, int64_t k, int B);
+size_t sweep_workspace_bytes(int64_t r, int64_t k, int B, int G, bool static_groups);
 gptq_status quantize_layer_impl(const void* W, gptq_dtype dt, int64_t r, int64_t k, int64_t ldw,
                                 const float* U, const int32_t* perm, const uint8_t* dead,
                                 const float* H0, const gptq_config* cfg, uint8_t* codes,
@@ -97,7 +97,7 @@ size_t gptq_workspace_size(int op, int64_t r, int64_t k, int64_t n, const gptq_c
       return hinv_workspace_bytes(k);
     case GPTQ_OP_QUANTIZE:
       if (cfg == nullptr) return 0;
-      return sweep_workspace_bytes(r, k, cfg->block_size);
+      return sweep_workspace_bytes(r, k, cfg->block_size, cfg->group_size, cfg->static_groups != 0);
   }
   return 0;
 }
@@ -150,7 +150,8 @@ gptq_status gptq_quantize_layer(const void* W, gptq_dtype dt, int64_t r, int64_t
       scales == nullptr || zeros == nullptr || g_idx == nullptr)
     return GPTQ_ERR_INVALID_ARG;
   if (!aligned(W, dtype_bytes(dt))) return GPTQ_ERR_INVALID_ARG;
-  size_t need = sweep_workspace_bytes(r, k, cfg->block_size);
+  size_t need = sweep_workspace_bytes(r, k, cfg->block_size, cfg->group_size,
+                                      cfg->static_groups != 0);
   if (ws == nullptr || ws_bytes < need || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
   return quantize_layer_impl(W, dt, r, k, ldw, U, perm, dead, H0, cfg, codes, scales, zeros, g_idx,
                              loss, d_status, ws, (cudaStream_t)stream);

@@ -29,26 +29,38 @@
 //      The tensor-core form updates the whole square [0, j0)^2 (tiles that
 //      lie entirely above its diagonal excepted), so the strip
 //      A[0:j0, j0:j1] is cleared by K2 before Y's block-J columns start.
-// so every step's large work is a short-K product with a big output.
+// On the tensor-core path the update has two levels: outer blocks O =
+// [o0, o1) of HV_O = 512 indices (8 blocks).  Block J's update goes at once
+// only to the band of rows [o0, j0) -- everything the later blocks of O read
+// (their diagonal blocks, panels and Y rows) -- and the rows [0, o0) above O
+// get the contributions of all of O's blocks in one K = 512 product at O's
+// end.  Its operand holds the 8 row blocks side by side; the Schur part of a
+// block inside O (columns [o0, j0)) is zeroed once its band update has used
+// it, so that only Y contributions reach those columns of the rows above.
+// Adds are reordered, nothing else: the result is that of the one-level
+// scheme up to fp32 rounding, and the k x k matrix (larger than L2 for the
+// widest layers) is streamed 8 times less often.
 // A final pass zeroes the strict lower triangle.
 #include "common.cuh"
 
 namespace gptq {
 
-constexpr int HV_B = 64;  // block width
+constexpr int HV_B = 64;   // block width
+constexpr int HV_O = 512;  // outer block width of the two-level tensor-core path
 
 bool tc_update_supported(int64_t k);
-gptq_status tc_rank_update(float* A, int k, int j0, int b, const float* s_hi, const float* s_lo,
-                           const float* r_hi, const float* r_lo, int32_t* d_info, cudaStream_t s);
+gptq_status tc_rank_update(float* A, int k, int row0, int row1, int split, int K, int ld_s,
+                           const float* s_hi, const float* s_lo, const float* r_hi,
+                           const float* r_lo, int32_t* d_info, cudaStream_t s);
 
 struct HinvScratch {
   double* sum_diag;  // [1]
   float* lambda;     // [1]
   float* diag;       // [k] diag(H) after the dead-column fix
   float* ujj;        // [HV_B * HV_B] U_JJ of the current step
-  float* s_hi;       // [k * HV_B] signed split of the current row block, transposed (tensor-core path)
-  float* s_lo;
-  float* r_hi;       // [k * HV_B] unsigned split (columns < j0 only)
+  float* s_hi;       // [k * HV_O] signed splits of the outer block's row blocks, transposed
+  float* s_lo;       //   (tensor-core path; row block J at column j0 - o0)
+  float* r_hi;       // [k * HV_O] unsigned splits (columns < j0 only)
   float* r_lo;
 };
 
@@ -62,14 +74,18 @@ size_t hinv_workspace_min_bytes(int64_t k) {
   return b;
 }
 
-// Scratch of the tensor-core path (the size gptq_workspace_size reports).
-size_t hinv_workspace_bytes(int64_t k) {
-  size_t b = hinv_workspace_min_bytes(k);
-  if (tc_update_supported(k)) b += 4 * align256(sizeof(float) * HV_B * (size_t)k);
-  return b;
+// Scratch of the tensor-core path with outer blocks of `outer` columns.
+static size_t hinv_workspace_tc_bytes(int64_t k, int outer) {
+  return hinv_workspace_min_bytes(k) + 4 * align256(sizeof(float) * (size_t)outer * (size_t)k);
 }
 
-static HinvScratch carve(void* ws, int64_t k, bool tc) {
+// Scratch the call asks for (gptq_workspace_size): the two-level tensor-core
+// path where it applies.
+size_t hinv_workspace_bytes(int64_t k) {
+  return tc_update_supported(k) ? hinv_workspace_tc_bytes(k, HV_O) : hinv_workspace_min_bytes(k);
+}
+
+static HinvScratch carve(void* ws, int64_t k, int outer) {
   char* p = (char*)ws;
   HinvScratch s;
   s.sum_diag = (double*)p; p += align256(sizeof(double));
@@ -77,9 +93,9 @@ static HinvScratch carve(void* ws, int64_t k, bool tc) {
   s.diag = (float*)p; p += align256(sizeof(float) * (size_t)k);
   s.ujj = (float*)p; p += align256(sizeof(float) * HV_B * HV_B);
   float* t[4] = {nullptr, nullptr, nullptr, nullptr};
-  for (int i = 0; i < 4 && tc; ++i) {
+  for (int i = 0; i < 4 && outer > 0; ++i) {
     t[i] = (float*)p;
-    p += align256(sizeof(float) * HV_B * (size_t)k);
+    p += align256(sizeof(float) * (size_t)outer * (size_t)k);
   }
   s.s_hi = t[0], s.s_lo = t[1], s.r_hi = t[2], s.r_lo = t[3];
   return s;
@@ -174,68 +190,89 @@ __device__ __forceinline__ void set_info(int32_t* d_info, int idx) { atomicCAS(d
 // With B = P A_JJ P (P reverses the indices), A_JJ = L^T L (L lower, the
 // factorisation that starts from the last index) becomes the ordinary lower
 // Cholesky B = M M^T with M = P L^T P, and U_JJ = (L^T)^-1 = P M^-1 P.  The
-// kernel factors B and inverts M in 16 x 16 blocks (rows and columns past b
-// padded with the identity):
-//   factor, block column kb = 0..3:
-//     M_kk = chol(B_kk)                 one warp, the block in registers
-//     M_ik = B_ik M_kk^-T   (i > kb)    one thread per row, forward substitution
-//     B_ij -= M_ik M_jk^T   (kb < j <= i) the whole CTA
-//   inverse N = M^-1:
-//     N_kk = M_kk^-1                    four warps, one block each, one lane per column
-//     N_ik = -N_ii sum_{m=k}^{i-1} M_im N_mk, by block distance i - k = 1, 2, 3
+// kernel factors B and inverts M together, in 16 x 16 blocks (rows and
+// columns past b padded with the identity), block column kb = 0..3:
+//   (A) one warp: M_kk = chol(B_kk) and N_kk = M_kk^-1, lane i holding row i
+//       in registers, the pivots' columns passed along by shuffles;
+//   (B) the CTA: M_ik = B_ik N_kk^T for the rows below (a product, no
+//       substitution chain), and X_m = sum_{l=m}^{kb-1} M_kl N_lm for m < kb;
+//   (C) the CTA: B_ij -= M_ik M_jk^T below, and the inverse's block row
+//       N_km = -N_kk X_m (m < kb), so N = M^-1 is complete when the loop ends.
 // U_JJ goes to the scratch, to the upper part of A[J, J] and, transposed and
-// split into tf32 hi / lo, to the rank update's operand.
-// Lower Cholesky of a 16 x 16 block whose lower triangle is held whole in
-// registers, a[i (i + 1) / 2 + j] = B_ij (j <= i); every lane of the warp
-// runs it (no communication).  Column C: pivot, scale, then the rank-1
-// update of the trailing triangle -- all independent instructions.  rd[C]
-// receives 1 / M_CC; first_bad = the first pivot that is not positive and
-// finite, else unchanged.  Unrolled by template recursion so that a stays
-// in registers inside the caller's block loop.
-__device__ __forceinline__ constexpr int tri(int i, int j) { return i * (i + 1) / 2 + j; }
-
-template <int C>
-struct Chol16 {
-  __device__ __forceinline__ static void run(float (&a)[136], float (&rd)[16], int& first_bad) {
-    const float p = a[tri(C, C)];
-    if ((!(p > 0.f) || !isfinite(p)) && first_bad < 0) first_bad = C;
-    const float r = rsqrtf(p);  // 1 / sqrt(p), within 2 ulp
-    rd[C] = r;
-    a[tri(C, C)] = p * r;
-#pragma unroll
-    for (int i = C + 1; i < 16; ++i) a[tri(i, C)] *= r;
-#pragma unroll
-    for (int i = C + 1; i < 16; ++i)
-#pragma unroll
-      for (int j = C + 1; j <= i; ++j) a[tri(i, j)] = fmaf(-a[tri(i, C)], a[tri(j, C)], a[tri(i, j)]);
-    Chol16<C + 1>::run(a, rd, first_bad);
-  }
-};
-template <>
-struct Chol16<16> {
-  __device__ __forceinline__ static void run(float (&)[136], float (&)[16], int&) {}
-};
-
+// split into tf32 hi / lo, to the rank update's operand (row stride ld_s,
+// column offset s_off).
 constexpr int K1_BS = 16;                 // block size
 constexpr int K1_NB = HV_B / K1_BS;       // blocks per side
 constexpr int K1_LD = HV_B + 1;
 
+// Lower Cholesky and inverse of the 16 x 16 block at (c0, c0) of S, by one
+// warp: lane i (and its mirror i + 16) holds row i.  M goes back to S, N =
+// M^-1 to T (lower parts).  Returns the index of the first pivot that is not
+// positive and finite, or -1 (the same on every lane).
+__device__ __forceinline__ int chol_inv16_warp(float (*S)[K1_LD], float (*T)[K1_LD], int c0,
+                                               int lane) {
+  const int i = lane & 15;
+  float a[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) a[j] = (j <= i) ? S[c0 + i][c0 + j] : 0.f;
+  int bad = -1;
+  float myr = 0.f;
+#pragma unroll
+  for (int C = 0; C < 16; ++C) {
+    const float p = __shfl_sync(0xffffffffu, a[C], C);
+    if ((!(p > 0.f) || !isfinite(p)) && bad < 0) bad = C;
+    const float r = rsqrtf(p);  // 1 / sqrt(p), within 2 ulp
+    if (i == C) myr = r;
+    if (i >= C) a[C] *= r;      // column C of M (the pivot row gets sqrt(p))
+#pragma unroll
+    for (int j = C + 1; j < 16; ++j) {
+      const float lj = __shfl_sync(0xffffffffu, a[C], j);
+      if (i >= j) a[j] = fmaf(-a[C], lj, a[j]);
+    }
+  }
+  // N = M^-1 row by row: N_mm = 1 / M_mm, N_mj = -(sum_{q=j}^{m-1} M_mq N_qj) / M_mm
+  float n[16], acc[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) n[j] = 0.f, acc[j] = 0.f;
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    if (i == m) {
+#pragma unroll
+      for (int j = 0; j < m; ++j) n[j] = -acc[j] * myr;
+      n[m] = myr;
+    }
+#pragma unroll
+    for (int j = 0; j <= m; ++j) {
+      const float v = __shfl_sync(0xffffffffu, n[j], m);
+      if (i > m) acc[j] = fmaf(a[m], v, acc[j]);
+    }
+  }
+  if (lane < 16) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j <= i) S[c0 + i][c0 + j] = a[j], T[c0 + i][c0 + j] = n[j];
+  }
+  return bad;
+}
+
 __global__ void __launch_bounds__(256)
 chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
                      float* __restrict__ ujj, float* __restrict__ st_hi,
-                     float* __restrict__ st_lo, int32_t* __restrict__ d_info) {
+                     float* __restrict__ st_lo, int ld_s, int s_off, int s_prev,
+                     int32_t* __restrict__ d_info) {
   pdl_wait();
   pdl_trigger();
   if (*d_info != 0) return;
-  __shared__ float S[HV_B][K1_LD];                 // B, then M (lower part)
-  __shared__ float T[HV_B][K1_LD];                 // N = M^-1 (lower part)
-  __shared__ float X[K1_NB - 1][K1_BS][K1_BS + 1];  // sums of one inverse round
-  __shared__ float rdg[HV_B];                        // 1 / M_ii
+  __shared__ float S[HV_B][K1_LD];                  // B, then M (lower part)
+  __shared__ float T[HV_B][K1_LD];                  // N = M^-1 (lower part)
+  __shared__ float Mt[HV_B - K1_BS][K1_BS + 1];     // M_ik of the current block column
+  __shared__ float Xs[K1_NB - 1][K1_BS][K1_BS + 1];  // X_m of the current block row
   __shared__ int fail;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   for (int e = t; e < HV_B * HV_B; e += 256) {
     const int i = e / HV_B, j = e % HV_B;
     S[i][j] = (i == j && i >= b) ? 1.f : 0.f;
+    T[i][j] = 0.f;
   }
   if (t == 0) fail = -1;
   __syncthreads();
@@ -257,102 +294,60 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
   __syncthreads();
 
   for (int kb = 0; kb < K1_NB; ++kb) {
-    const int c0 = kb * K1_BS;
+    const int c0 = kb * K1_BS, r0 = c0 + K1_BS, nr = HV_B - r0;
+    // (A) the diagonal block
     if (warp == 0) {
-      // every lane factors the whole block in registers; lane 0 writes it back
-      float a[136], rd[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-#pragma unroll
-        for (int j = 0; j <= i; ++j) a[tri(i, j)] = S[c0 + i][c0 + j];
-      int first_bad = -1;
-      Chol16<0>::run(a, rd, first_bad);
-      if (lane == 0) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-#pragma unroll
-          for (int j = 0; j <= i; ++j) S[c0 + i][c0 + j] = a[tri(i, j)];
-          rdg[c0 + i] = rd[i];
-        }
-        if (first_bad >= 0) fail = c0 + first_bad;
-      }
+      const int bad = chol_inv16_warp(S, T, c0, lane);
+      if (lane == 0 && bad >= 0) fail = c0 + bad;
     }
     __syncthreads();
     if (fail >= 0) break;
-    const int r0 = c0 + K1_BS, nr = HV_B - r0;
-    if (t < nr) {
-      // x M_kk^T = b_i by columns: fix x_m, then take it out of the later ones
-      const int i = r0 + t;
-      float x[K1_BS];
+    // (B) M_ik = B_ik N_kk^T (rows below), X_m for the inverse's block row kb
+    for (int e = t; e < nr * K1_BS + kb * K1_BS * K1_BS; e += 256) {
+      if (e < nr * K1_BS) {
+        const int ii = e / K1_BS, j = e % K1_BS;
+        float acc = 0.f;
 #pragma unroll
-      for (int m = 0; m < K1_BS; ++m) x[m] = S[i][c0 + m];
-#pragma unroll
-      for (int m = 0; m < K1_BS; ++m) {
-        x[m] *= rdg[c0 + m];
-#pragma unroll
-        for (int q = m + 1; q < K1_BS; ++q) x[q] = fmaf(-x[m], S[c0 + q][c0 + m], x[q]);
+        for (int m = 0; m < K1_BS; ++m)
+          if (m <= j) acc = fmaf(S[r0 + ii][c0 + m], T[c0 + j][c0 + m], acc);
+        Mt[ii][j] = acc;
+      } else {
+        const int f = e - nr * K1_BS, mb = f / (K1_BS * K1_BS);
+        const int q = (f / K1_BS) % K1_BS, c = f % K1_BS;
+        float acc = 0.f;
+        for (int col = mb * K1_BS; col < c0; ++col)
+          acc = fmaf(S[c0 + q][col], T[col][mb * K1_BS + c], acc);
+        Xs[mb][q][c] = acc;
       }
-#pragma unroll
-      for (int m = 0; m < K1_BS; ++m) S[i][c0 + m] = x[m];
     }
     __syncthreads();
+    // (C) M_ik back into B, the trailing update, the inverse's block row kb
+    for (int e = t; e < nr * K1_BS; e += 256) {
+      const int ii = e / K1_BS, j = e % K1_BS;
+      S[r0 + ii][c0 + j] = Mt[ii][j];
+    }
     for (int e = t; e < nr * nr; e += 256) {
       const int ii = e / nr, jj = e % nr;
       if (jj <= ii) {
         float acc = S[r0 + ii][r0 + jj];
 #pragma unroll
-        for (int m = 0; m < K1_BS; ++m) acc = fmaf(-S[r0 + ii][c0 + m], S[r0 + jj][c0 + m], acc);
+        for (int m = 0; m < K1_BS; ++m) acc = fmaf(-Mt[ii][m], Mt[jj][m], acc);
         S[r0 + ii][r0 + jj] = acc;
       }
+    }
+    for (int e = t; e < kb * K1_BS * K1_BS; e += 256) {
+      const int mb = e / (K1_BS * K1_BS), r = (e / K1_BS) % K1_BS, c = e % K1_BS;
+      float acc = 0.f;
+#pragma unroll
+      for (int q = 0; q < K1_BS; ++q)
+        if (q <= r) acc = fmaf(T[c0 + r][c0 + q], Xs[mb][q][c], acc);
+      T[c0 + r][mb * K1_BS + c] = -acc;
     }
     __syncthreads();
   }
   if (fail >= 0) {
     if (t == 0) set_info(d_info, j0 + (b - 1 - fail));
     return;
-  }
-
-  // inverse of M: diagonal blocks
-  if (warp < K1_NB && lane < K1_BS) {
-    const int c0 = warp * K1_BS, j = lane;
-    // column j of M_kk^-1: fix x_i, then take it out of the later rows
-    float x[K1_BS];
-#pragma unroll
-    for (int i = 0; i < K1_BS; ++i) x[i] = (i == j) ? 1.f : 0.f;
-#pragma unroll
-    for (int i = 0; i < K1_BS; ++i) {
-      x[i] = (i < j) ? 0.f : x[i] * rdg[c0 + i];
-#pragma unroll
-      for (int q = i + 1; q < K1_BS; ++q) x[q] = fmaf(-S[c0 + q][c0 + i], x[i], x[q]);
-    }
-#pragma unroll
-    for (int i = 0; i < K1_BS; ++i) T[c0 + i][c0 + j] = x[i];
-  }
-  __syncthreads();
-  // off-diagonal blocks by distance d
-  for (int d = 1; d < K1_NB; ++d) {
-    const int nblk = K1_NB - d;
-    for (int e = t; e < nblk * K1_BS * K1_BS; e += 256) {
-      const int q = e / (K1_BS * K1_BS), r = (e / K1_BS) % K1_BS, c = e % K1_BS;
-      const int ib = q + d;
-      float acc = 0.f;
-      for (int mb = q; mb < ib; ++mb)
-#pragma unroll
-        for (int m = 0; m < K1_BS; ++m)
-          acc = fmaf(S[ib * K1_BS + r][mb * K1_BS + m], T[mb * K1_BS + m][q * K1_BS + c], acc);
-      X[q][r][c] = acc;
-    }
-    __syncthreads();
-    for (int e = t; e < nblk * K1_BS * K1_BS; e += 256) {
-      const int q = e / (K1_BS * K1_BS), r = (e / K1_BS) % K1_BS, c = e % K1_BS;
-      const int ib = q + d;
-      float acc = 0.f;
-#pragma unroll
-      for (int m = 0; m < K1_BS; ++m)
-        if (m <= r) acc = fmaf(T[ib * K1_BS + r][ib * K1_BS + m], X[q][m][c], acc);
-      T[ib * K1_BS + r][q * K1_BS + c] = -acc;
-    }
-    __syncthreads();
   }
   // U_JJ[iu][cu] = N[b-1-iu][b-1-cu] (iu <= cu < b)
   for (int e = t; e < HV_B * HV_B; e += 256) {
@@ -363,14 +358,20 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
     if (in) A[(int64_t)(j0 + iu) * k + j0 + cu] = u;
   }
   if (st_hi != nullptr) {
-    // rank-update operand s[j0 + cu][iu] = U_JJ[iu][cu]  (columns of block J, sign +)
+    // rank-update operand s[j0 + cu][s_off + iu] = U_JJ[iu][cu]  (columns of block J, sign +)
     for (int e = t; e < b * HV_B; e += 256) {
       const int cu = e / HV_B, iu = e % HV_B;
       const float u = (iu <= cu) ? T[b - 1 - iu][b - 1 - cu] : 0.f;
       float h, l;
       hv_split_tf32(u, h, l);
-      st_hi[(int64_t)(j0 + cu) * HV_B + iu] = h;
-      st_lo[(int64_t)(j0 + cu) * HV_B + iu] = l;
+      st_hi[(int64_t)(j0 + cu) * ld_s + s_off + iu] = h;
+      st_lo[(int64_t)(j0 + cu) * ld_s + s_off + iu] = l;
+      if (s_prev >= 0) {
+        // the block below in the same outer block: its Schur part at these
+        // columns was used by its band update and must not reach the outer one
+        st_hi[(int64_t)(j0 + cu) * ld_s + s_prev + iu] = 0.f;
+        st_lo[(int64_t)(j0 + cu) * ld_s + s_prev + iu] = 0.f;
+      }
     }
   }
 }
@@ -387,15 +388,19 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
 //     writes the whole square [0, j0)^2 and leaves values above its diagonal).
 // Thread (r = t / 4, cq = t % 4) computes row r, columns 4 cq .. 4 cq + 3.  When
 // st_hi is given, the new row-block tile also goes out transposed and split
-// into tf32 hi / lo in the rank update's operand layout: st[c][m] = -R[m][c]
-// for c < j0 and +R[m][c] above, rt[c][m] = R[m][c] for c < j0.
+// into tf32 hi / lo in the rank update's operand layout (row stride ld_s,
+// this block's slice at column s_off): st[c][m] = -R[m][c] for c < j0 and
+// +R[m][c] above, rt[c][m] = R[m][c] for c < j0.  With two-level blocking the
+// panel CTAs also zero the slice s_prev of the block below (same outer block
+// [o0, ...)) at columns [o0, j0): that block's Schur part inside the outer
+// block has been applied by its band update and must not reach the outer one.
 constexpr int K2_W = 16;  // columns per CTA
 
 __global__ void __launch_bounds__(256)
 panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* __restrict__ ujj,
                       int n_pan, float* __restrict__ st_hi, float* __restrict__ st_lo,
-                      float* __restrict__ rt_hi, float* __restrict__ rt_lo,
-                      const int32_t* __restrict__ d_info) {
+                      float* __restrict__ rt_hi, float* __restrict__ rt_lo, int ld_s, int s_off,
+                      int o0, int s_prev, const int32_t* __restrict__ d_info) {
   pdl_wait();
   pdl_trigger();
   if (*d_info != 0) return;
@@ -471,11 +476,16 @@ panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* 
       const float x = m < b ? Os[m][cc] : 0.f;  // the new row block R
       float h, l;
       hv_split_tf32(pan ? -x : x, h, l);  // st = -R for c < j0, +R for c >= j1
-      st_hi[(int64_t)(c0 + cc) * HV_B + m] = h;
-      st_lo[(int64_t)(c0 + cc) * HV_B + m] = l;
+      const int64_t o = (int64_t)(c0 + cc) * ld_s + s_off + m;
+      st_hi[o] = h;
+      st_lo[o] = l;
       if (pan) {
-        rt_hi[(int64_t)(c0 + cc) * HV_B + m] = -h;
-        rt_lo[(int64_t)(c0 + cc) * HV_B + m] = -l;
+        rt_hi[o] = -h;
+        rt_lo[o] = -l;
+        if (s_prev >= 0 && c0 + cc >= o0) {
+          st_hi[o - s_off + s_prev] = 0.f;
+          st_lo[o - s_off + s_prev] = 0.f;
+        }
       }
     }
   }
@@ -608,9 +618,16 @@ gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cf
                               int32_t* perm, int32_t* invperm, uint8_t* dead, int32_t* d_info,
                               void* ws, size_t ws_bytes, cudaStream_t s) {
   const int k = (int)k64;
-  // tensor-core rank updates when the workspace holds their operand splits
-  const bool tc = tc_update_supported(k) && ws_bytes >= hinv_workspace_bytes(k);
-  HinvScratch sc = carve(ws, k, tc);
+  // tensor-core rank updates when the workspace holds their operand splits:
+  // two-level (outer blocks of HV_O) when it holds HV_O columns of them per
+  // row, one level (outer = HV_B) when it holds HV_B; else CUDA-core updates
+  int outer = 0;
+  if (tc_update_supported(k)) {
+    if (ws_bytes >= hinv_workspace_tc_bytes(k, HV_O)) outer = HV_O;
+    else if (ws_bytes >= hinv_workspace_tc_bytes(k, HV_B)) outer = HV_B;
+  }
+  const bool tc = outer > 0;
+  HinvScratch sc = carve(ws, k, outer);
   hinv_prep_kernel<<<1, 1024, 0, s>>>(H, k, cfg->percdamp, dead, sc.diag, sc.sum_diag, sc.lambda,
                                       d_info);
   GPTQ_CHECK_LAUNCH();
@@ -622,39 +639,60 @@ gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cf
     hinv_gather_lower_kernel<<<grid, 256, 0, s>>>(H, k, perm, sc.diag, sc.lambda, U);
     GPTQ_CHECK_LAUNCH();
   }
-  // blocks from the bottom; the short block (if any) is the top one
-  for (int j1 = k; j1 > 0; j1 -= HV_B) {
-    const int j0 = j1 > HV_B ? j1 - HV_B : 0;
-    const int b = j1 - j0;
-    // the tensor-core update takes row block J transposed and split into
-    // tf32 hi / lo, written by K1 (diagonal columns) and K2 (the rest); its
-    // Schur part leaves values above the diagonal of [0, j0)^2, so K2 also
-    // clears the strip where block J's Y columns start accumulating
-    const bool tcs = tc && j0 > 0;
-    launch_pdl(chol_inv_diag_kernel, dim3(1), dim3(256), 0, s, U, k, j0, b, sc.ujj,
-               tcs ? sc.s_hi : nullptr, tcs ? sc.s_lo : nullptr, d_info);
-    GPTQ_CHECK_LAUNCH();
-    const int n_pan = (int)cdiv(j0, K2_W);
-    const int n_row = (int)cdiv(k - j1, K2_W);
-    if (n_pan + n_row > 0) {
-      launch_pdl(panel_rowblock_kernel, dim3((unsigned)(n_pan + n_row)), dim3(256), 0, s, U, k, j0,
-                 b, (const float*)sc.ujj, n_pan, tcs ? sc.s_hi : nullptr,
-                 tcs ? sc.s_lo : nullptr, tcs ? sc.r_hi : nullptr, tcs ? sc.r_lo : nullptr,
-                 (const int32_t*)d_info);
+  // blocks from the bottom; the short block (if any) is the top one.  Outer
+  // blocks [o0, o1) of `outer` columns (whole blocks; the top one may be
+  // shorter).  Per block J = [j0, j1) of an outer block: K1, K2, then the
+  // band update of rows [o0, j0) (everything the outer block's later blocks
+  // read); after the outer block's top block, the outer update of rows
+  // [0, o0) with K = o1 - o0.  One level (outer = HV_B) has no band updates.
+  const int ob = tc ? outer : HV_B;
+  for (int o1 = k; o1 > 0; o1 -= ob) {
+    const int o0 = o1 > ob ? o1 - ob : 0;
+    for (int j1 = o1; j1 > o0; j1 -= HV_B) {
+      const int j0 = j1 - HV_B > o0 ? j1 - HV_B : o0;
+      const int b = j1 - j0;
+      // the tensor-core updates take row block J transposed and split into
+      // tf32 hi / lo, written by K1 (diagonal columns) and K2 (the rest) at
+      // column j0 - o0 of the outer block's slices; their Schur part leaves
+      // values above the diagonal of the square they update, so K2 also
+      // clears the strip where block J's Y columns start accumulating
+      const bool tcs = tc && j0 > 0;
+      const int s_off = j0 - o0;
+      const int s_prev = (tcs && j1 < o1) ? j1 - o0 : -1;  // the block below, same outer block
+      launch_pdl(chol_inv_diag_kernel, dim3(1), dim3(256), 0, s, U, k, j0, b, sc.ujj,
+                 tcs ? sc.s_hi : nullptr, tcs ? sc.s_lo : nullptr, outer, s_off, s_prev, d_info);
       GPTQ_CHECK_LAUNCH();
-    }
-    if (j0 > 0) {
-      if (tc) {
-        gptq_status st = tc_rank_update(U, k, j0, b, sc.s_hi, sc.s_lo, sc.r_hi, sc.r_lo, d_info, s);
-        if (st != GPTQ_OK) return st;
-      } else {
+      const int n_pan = (int)cdiv(j0, K2_W);
+      const int n_row = (int)cdiv(k - j1, K2_W);
+      if (n_pan + n_row > 0) {
+        launch_pdl(panel_rowblock_kernel, dim3((unsigned)(n_pan + n_row)), dim3(256), 0, s, U, k,
+                   j0, b, (const float*)sc.ujj, n_pan, tcs ? sc.s_hi : nullptr,
+                   tcs ? sc.s_lo : nullptr, tcs ? sc.r_hi : nullptr, tcs ? sc.r_lo : nullptr,
+                   outer, s_off, o0, s_prev, (const int32_t*)d_info);
+        GPTQ_CHECK_LAUNCH();
+      }
+      if (j0 == 0) continue;
+      if (!tc) {
         const int nt = (int)cdiv(j0, 128);
         const int n_low = nt * (nt + 1) / 2;
         const int n_right = nt * (int)cdiv(k - j0, 128);
         rank_update_kernel<<<(unsigned)(n_low + n_right), 256, 0, s>>>(U, k, j0, b, n_low,
                                                                        d_info);
         GPTQ_CHECK_LAUNCH();
+      } else if (j0 > o0) {
+        // band: rows [o0, j0) += (block J's panel)^T (its signed row block)
+        gptq_status st = tc_rank_update(U, k, o0, j0, j0, b, outer, sc.s_hi + s_off,
+                                        sc.s_lo + s_off, sc.r_hi + s_off, sc.r_lo + s_off,
+                                        d_info, s);
+        if (st != GPTQ_OK) return st;
       }
+    }
+    if (tc && o0 > 0) {
+      // outer: rows [0, o0) += (the outer block's panels)^T (its row blocks,
+      // without their Schur parts inside the outer block)
+      gptq_status st = tc_rank_update(U, k, 0, o0, o0, o1 - o0, outer, sc.s_hi, sc.s_lo,
+                                      sc.r_hi, sc.r_lo, d_info, s);
+      if (st != GPTQ_OK) return st;
     }
   }
   {

@@ -13,9 +13,10 @@
 // The array is `kScratchBytes` (4 MiB) on every device that loads the
 // library and is held until the process exits; it covers k up to
 // kNoAllocMaxK = 12288.  Up to k = 4060 the tensor-core rank updates' operand
-// splits fit beside the rest and the kernels are those of gptq_prepare_hinv
-// (bit-identical results); above, the fp32 CUDA-core rank update runs instead
-// (same result within fp32 rounding, slower).  All calls share it and it keeps the previous call's
+// splits for one 64-column block fit beside the rest (one-level updates, where
+// gptq_prepare_hinv batches 8 blocks); above, the fp32 CUDA-core rank update
+// runs instead (slower).  Either way U equals gptq_prepare_hinv's within fp32
+// rounding.  All calls share it and it keeps the previous call's
 // contents; the Cholesky stages write every scratch word before reading it,
 // so nothing needs clearing.  Calls whose work overlaps on the GPU (two
 // streams, or two host threads) race on the array: serialise them.

@@ -14,6 +14,15 @@
 //   (trailing)      W[:, e:] -= Err * U[s:e, e:]: on the tensor cores in
 //                   fp32-accurate 3xTF32 (tf32x3.cu) when k % 4 == 0, else an
 //                   fp32 CUDA-core GEMM.
+// On the tensor-core path the lazy batching has two levels: blocks of B
+// columns inside outer blocks of WO = 512 columns.  A block's errors update
+// only the rest of its outer block at once (W[:, e:o1] -= Err_b U[s:e, e:o1]);
+// the outer block's errors (r x WO) update everything beyond it in one
+// K = WO product at its end (W[:, o1:] -= Err_O U[o0:o1, o1:]).  Every column
+// still receives every earlier column's compensation before its own turn, so
+// the result is that of the one-level sweep (and of the column-by-column
+// sweep) up to fp32 summation order, while the trailing matrix, which is
+// larger than L2 for the big layers, is streamed WO / B = 4 times less often.
 // The layer loss is accumulated inside the block kernel through the Optimal
 // Brain Surgeon accounting: fixing column i and compensating the later ones
 // raises (w - q) Hd (w - q)^T by err_i^2, so per row
@@ -63,33 +72,47 @@ static size_t sweep_records_bytes(int64_t k, int B) { return (size_t)cdiv(k, B) 
 bool tc_update_supported(int64_t k);
 gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols, float sign,
                                int upper_only, float* hi, float* lo, int64_t ldo, cudaStream_t s);
-gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* nut_hi,
-                              const float* nut_lo, float* Wt, int r, int k, int s0, int e,
-                              int32_t* d_status, cudaStream_t s);
+gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int ldE, int K,
+                              const float* nut_hi, const float* nut_lo, float* Wt, int r, int k,
+                              int s0, int c0, int c1, int32_t* d_status, cudaStream_t s);
+
+constexpr int SW_OUTER = 512;  // outer lazy block of the tensor-core path
+
+// Outer block width: SW_OUTER when every dynamic grid wider than a block
+// still sees all of its group's columns up to date at the group's start
+// (groups inside a block, static grids, one grid per row, or groups that
+// nest with the outer blocks), else B (one level).
+static int sweep_outer_width(int64_t k, int B, int G, bool static_groups, bool tc) {
+  if (!tc || B >= SW_OUTER || SW_OUTER % B != 0) return B;
+  if (static_groups || G <= B || G >= k || SW_OUTER % G == 0 || G % SW_OUTER == 0) return SW_OUTER;
+  return B;
+}
 
 struct SweepScratch {
   float* Wt;      // [r * k] working weights, processing order
-  float* Err;     // [r * B] errors of the current block (tf32 high part on the tensor-core path)
-  float* Err_lo;  // [r * B] tf32 low part (tensor-core path)
+  float* Err;     // [r * WO] errors of the current outer block (tf32 high part on the tensor-core path)
+  float* Err_lo;  // [r * WO] tf32 low part (tensor-core path)
   float* U_hi;    // [k * k] tf32 split of -U^T (tensor-core path)
   float* U_lo;    // [k * k]
   float* lambda;  // [1] damping added to the Hessian diagonal (for the loss)
   uint8_t* rec;   // per-block records of the 4-lanes-per-row kernel
 };
 
-size_t sweep_workspace_bytes(int64_t r, int64_t k, int B) {
-  size_t b = align256(sizeof(float) * (size_t)r * k) + 2 * align256(sizeof(float) * (size_t)r * B) +
+size_t sweep_workspace_bytes(int64_t r, int64_t k, int B, int G, bool static_groups) {
+  const bool tc = tc_update_supported(k);
+  const int WO = sweep_outer_width(k, B, G == -1 ? (int)k : G, static_groups, tc);
+  size_t b = align256(sizeof(float) * (size_t)r * k) + 2 * align256(sizeof(float) * (size_t)r * WO) +
              align256(sizeof(float)) + align256(sweep_records_bytes(k, B));
-  if (tc_update_supported(k)) b += 2 * align256(sizeof(float) * (size_t)k * k);
+  if (tc) b += 2 * align256(sizeof(float) * (size_t)k * k);
   return b;
 }
 
-static SweepScratch carve_sweep(void* ws, int64_t r, int64_t k, int B, bool tc) {
+static SweepScratch carve_sweep(void* ws, int64_t r, int64_t k, int B, int WO, bool tc) {
   char* p = (char*)ws;
   SweepScratch s;
   s.Wt = (float*)p; p += align256(sizeof(float) * (size_t)r * k);
-  s.Err = (float*)p; p += align256(sizeof(float) * (size_t)r * B);
-  s.Err_lo = (float*)p; p += align256(sizeof(float) * (size_t)r * B);
+  s.Err = (float*)p; p += align256(sizeof(float) * (size_t)r * WO);
+  s.Err_lo = (float*)p; p += align256(sizeof(float) * (size_t)r * WO);
   s.lambda = (float*)p; p += align256(sizeof(float));
   s.rec = (uint8_t*)p; p += align256(sweep_records_bytes(k, B));
   s.U_hi = tc ? (float*)p : nullptr;
@@ -217,8 +240,8 @@ template <int SB>
 __global__ void __launch_bounds__(SW_THREADS)
 sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
                    float* __restrict__ Err_lo, const float* __restrict__ U,
-                   const int32_t* __restrict__ perm, int r, int k, int s, int bw, int B, int G,
-                   int ngroups, float maxq, int sym, float* __restrict__ scales,
+                   const int32_t* __restrict__ perm, int r, int k, int s, int bw, int B, int ldE,
+                   int G, int ngroups, float maxq, int sym, float* __restrict__ scales,
                    int32_t* __restrict__ zeros, uint8_t* __restrict__ codes,
                    double* __restrict__ loss, int32_t* __restrict__ d_status) {
   extern __shared__ float sm_sweep[];
@@ -323,10 +346,10 @@ sweep_block_kernel(const float* __restrict__ Wt, float* __restrict__ Err,
           if (Err_lo != nullptr) {
             float h, l;
             split_tf32(errs[ii], h, l);
-            Err[(int64_t)row * B + c0 + ii] = h;
-            Err_lo[(int64_t)row * B + c0 + ii] = l;
+            Err[(int64_t)row * ldE + c0 + ii] = h;
+            Err_lo[(int64_t)row * ldE + c0 + ii] = l;
           } else {
-            Err[(int64_t)row * B + c0 + ii] = errs[ii];
+            Err[(int64_t)row * ldE + c0 + ii] = errs[ii];
           }
         }
     }
@@ -404,6 +427,7 @@ struct SqArgs {
   float* Err_lo;
   const uint8_t* rec;  // this block's record
   int r, k, s, bw, B, G, ngroups;
+  int ldE;  // row stride of Err / Err_lo (Err points at this block's first column)
   float maxq;
   int sym;  // symmetric grid
   float* scales;
@@ -563,10 +587,10 @@ __device__ __forceinline__ void sq_sub_block(SqState<L>& st, int m, const SqArgs
     if (a.Err_lo != nullptr) {
       float h, lo;
       split_tf32(e_own, h, lo);
-      a.Err[(int64_t)row * a.B + c] = h;
-      a.Err_lo[(int64_t)row * a.B + c] = lo;
+      a.Err[(int64_t)row * a.ldE + c] = h;
+      a.Err_lo[(int64_t)row * a.ldE + c] = lo;
     } else {
-      a.Err[(int64_t)row * a.B + c] = e_own;
+      a.Err[(int64_t)row * a.ldE + c] = e_own;
     }
     st.nonfinite |= !isfinite(e_own);
     st.e2 += (double)e_own * (double)e_own;
@@ -707,12 +731,12 @@ __global__ void loss_total_kernel(double* __restrict__ loss, int r) {
 template <int SB>
 static gptq_status launch_block(unsigned grid, cudaStream_t s, const float* Wt, float* Err,
                                 float* Err_lo, const float* U, const int32_t* perm, int r, int k,
-                                int s0, int bw, int B, int G, int ngroups, float maxq, int sym,
-                                float* scales, int32_t* zeros, uint8_t* codes, double* loss,
-                                int32_t* d_status) {
+                                int s0, int bw, int B, int ldE, int G, int ngroups, float maxq,
+                                int sym, float* scales, int32_t* zeros, uint8_t* codes,
+                                double* loss, int32_t* d_status) {
   if (smem_optin((const void*)sweep_block_kernel<SB>, SW_SMEM) != cudaSuccess) return GPTQ_ERR_CUDA;
   sweep_block_kernel<SB><<<grid, SW_THREADS, SW_SMEM, s>>>(Wt, Err, Err_lo, U, perm, r, k, s0, bw,
-                                                           B, G, ngroups, maxq, sym, scales,
+                                                           B, ldE, G, ngroups, maxq, sym, scales,
                                                            zeros, codes, loss, d_status);
   return GPTQ_OK;
 }
@@ -743,7 +767,9 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
   const int ngroups = (int)cdiv(k, G);
   const float maxq = (float)((1 << cfg->bits) - 1);
   const bool tc = tc_update_supported(k);
-  SweepScratch sc = carve_sweep(ws, r, k, B, tc);
+  const bool stat = cfg->static_groups != 0;
+  const int WO = sweep_outer_width(k, B, G, stat, tc);
+  SweepScratch sc = carve_sweep(ws, r, k, B, WO, tc);
   const bool want_loss = (H0 != nullptr && loss != nullptr);
   double* lossp = want_loss ? loss : nullptr;
   {
@@ -752,7 +778,6 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
                                               sc.Wt, g_idx, lossp, d_status);
     GPTQ_CHECK_LAUNCH();
   }
-  const bool stat = cfg->static_groups != 0;
   if (stat) {
     static_grid_kernel<T><<<(unsigned)cdiv((int64_t)r * ngroups * kWarp, 256), 256, 0, s>>>(
         W, ldw, r, k, dead, G, ngroups, maxq, cfg->sym, scales, zeros);
@@ -795,9 +820,11 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     while (SB < 16 && G % (SB * 2) == 0) SB *= 2;
   }
   const unsigned grid = (unsigned)cdiv(r, SW_ROWS);
-  float* err_lo = tc ? sc.Err_lo : nullptr;
   for (int s0 = 0, b = 0; s0 < k; s0 += B, ++b) {
-    int bw = min(B, k - s0);
+    const int bw = min(B, k - s0);
+    const int o0 = (s0 / WO) * WO, o1 = min(o0 + WO, k);  // the outer block of this block
+    float* err_b = sc.Err + (s0 - o0);                     // this block's columns of Err
+    float* err_lo_b = tc ? sc.Err_lo + (s0 - o0) : nullptr;
     if (!stat && G > B && s0 % G == 0) {
       int gw = min(G, k - s0);
       group_grid_kernel<<<(unsigned)cdiv((int64_t)r * kWarp, 256), 256, 0, s>>>(
@@ -807,8 +834,9 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     if (lane_mode >= 0) {
       SqArgs a;
       a.Wt = sc.Wt;
-      a.Err = sc.Err;
-      a.Err_lo = err_lo;
+      a.Err = err_b;
+      a.Err_lo = err_lo_b;
+      a.ldE = WO;
       a.rec = sc.rec + (size_t)b * SQ_REC_MAX;
       a.r = r, a.k = k, a.s = s0, a.bw = bw, a.B = B, a.G = G, a.ngroups = ngroups;
       a.maxq = maxq;
@@ -834,9 +862,9 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
       if (st != GPTQ_OK) return st;
     } else {
       gptq_status st = GPTQ_OK;
-#define GPTQ_SWEEP_BLOCK(SBV)                                                                  \
-  st = launch_block<SBV>(grid, s, sc.Wt, sc.Err, err_lo, U, perm, r, k, s0, bw, B, G, ngroups, maxq, \
-                    cfg->sym, scales, zeros, codes, lossp, d_status)
+#define GPTQ_SWEEP_BLOCK(SBV)                                                                   \
+  st = launch_block<SBV>(grid, s, sc.Wt, err_b, err_lo_b, U, perm, r, k, s0, bw, B, WO, G, ngroups, \
+                         maxq, cfg->sym, scales, zeros, codes, lossp, d_status)
       switch (SB) {
         case 16: GPTQ_SWEEP_BLOCK(16); break;
         case 8: GPTQ_SWEEP_BLOCK(8); break;
@@ -848,18 +876,25 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
       if (st != GPTQ_OK) return st;
     }
     GPTQ_CHECK_LAUNCH();
-    int e0 = s0 + bw;
-    if (e0 < k) {
-      if (tc) {
-        gptq_status st = tc_sweep_trailing(sc.Err, sc.Err_lo, B, sc.U_hi, sc.U_lo, sc.Wt, r, k,
-                                           s0, e0, d_status, s);
-        if (st != GPTQ_OK) return st;
+    const int e0 = s0 + bw;
+    if (e0 >= k) continue;
+    if (tc) {
+      gptq_status st = GPTQ_OK;
+      if (e0 < o1) {
+        // the rest of the outer block: W[:, e0:o1] -= Err_b U[s0:e0, e0:o1]
+        st = tc_sweep_trailing(err_b, err_lo_b, WO, bw, sc.U_hi, sc.U_lo, sc.Wt, r, k, s0, e0, o1,
+                               d_status, s);
       } else {
-        sgemm<false, false, false, false, false>(r, k - e0, bw, -1.0f, sc.Err, B,
-                                                 U + (int64_t)s0 * k + e0, k, 1.0f, sc.Wt + e0, k,
-                                                 nullptr, s);
-        GPTQ_CHECK_LAUNCH();
+        // everything beyond the outer block: W[:, o1:] -= Err_O U[o0:o1, o1:]
+        st = tc_sweep_trailing(sc.Err, sc.Err_lo, WO, o1 - o0, sc.U_hi, sc.U_lo, sc.Wt, r, k, o0,
+                               o1, k, d_status, s);
       }
+      if (st != GPTQ_OK) return st;
+    } else {  // one level (WO == B)
+      sgemm<false, false, false, false, false>(r, k - e0, bw, -1.0f, sc.Err, WO,
+                                               U + (int64_t)s0 * k + e0, k, 1.0f, sc.Wt + e0, k,
+                                               nullptr, s);
+      GPTQ_CHECK_LAUNCH();
     }
   }
   if (want_loss) {

@@ -68,8 +68,8 @@ struct TxArgs {
 
 __device__ __forceinline__ bool tile_skipped(const TxArgs& a, int m0, int n0) {
   // mode 1: a tile whose columns all lie in [0, split) and strictly right of
-  // the diagonal of its rows has nothing the factorisation reads
-  return a.mode == 1 && n0 + TX_N <= a.split && n0 >= m0 + TX_M;
+  // the diagonal of its rows (row0 + m0 ...) has nothing the factorisation reads
+  return a.mode == 1 && n0 + TX_N <= a.split && n0 >= a.row0 + m0 + TX_M;
 }
 
 // Next tile of this CTA after t (t = -1: the first) that has work, or ntiles.
@@ -358,31 +358,34 @@ gptq_status tc_split_transpose(const float* src, int64_t lds, int rows, int cols
   return GPTQ_OK;
 }
 
-// Wt[0:r, e:k] -= Err[0:r, 0:B] * U[s:s+B, e:k]   (Err_hi/lo: r x B, ld B;
-// nut_hi/lo: the split of -U^T, k x k).  A timeout sets
-// *d_status = GPTQ_ERR_TIMEOUT.
-gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, const float* nut_hi,
-                              const float* nut_lo, float* Wt, int r, int k, int s0, int e,
-                              int32_t* d_status, cudaStream_t s) {
+// Wt[0:r, c0:c1] -= Err[0:r, 0:K] * U[s0:s0+K, c0:c1]   (Err_hi/lo: r x K at
+// row stride ldE, 16-byte aligned; nut_hi/lo: the split of -U^T, k x k).  The
+// output map ends at column c1 and Err's at column K (a K that is not a
+// multiple of the 32-wide stage reads zeros past it), so nothing outside
+// [c0, c1) is touched.  A timeout sets *d_status = GPTQ_ERR_TIMEOUT.
+gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int ldE, int K,
+                              const float* nut_hi, const float* nut_lo, float* Wt, int r, int k,
+                              int s0, int c0, int c1, int32_t* d_status, cudaStream_t s) {
+  if (c1 <= c0 || K <= 0) return GPTQ_OK;
   CUtensorMap ah, al, bh, bl, dm;
-  if (!make_map(&ah, err_hi, B, r, B, TX_M) || !make_map(&al, err_lo, B, r, B, TX_M) ||
+  if (!make_map(&ah, err_hi, K, r, ldE, TX_M) || !make_map(&al, err_lo, K, r, ldE, TX_M) ||
       !make_map(&bh, nut_hi, k, k, k, TX_N) || !make_map(&bl, nut_lo, k, k, k, TX_N) ||
-      !make_map(&dm, Wt, k, r, k, TX_M))
+      !make_map(&dm, Wt, c1, r, k, TX_M))
     return GPTQ_ERR_INVALID_ARG;
   TxArgs a;
   a.D = Wt;
   a.ldd = k;
   a.M = r;
-  a.N = k - e;
+  a.N = c1 - c0;
   a.row0 = 0;
-  a.col0 = e;
-  a.K = B;
+  a.col0 = c0;
+  a.K = K;
   a.a_k0 = 0;
   a.a_r0 = 0;
   a.b_k0 = s0;
-  a.b_r0 = e;
+  a.b_r0 = c0;
   a.ntm = (int)cdiv(r, TX_M);
-  a.ntiles = a.ntm * (int)cdiv(k - e, TX_N);
+  a.ntiles = a.ntm * (int)cdiv(c1 - c0, TX_N);
   a.mode = 0;
   a.split = 0;
   a.status = d_status;
@@ -390,36 +393,38 @@ gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int B, c
   return launch(ah, al, bh, bl, dm, a, s);
 }
 
-// Rows [0, j0) of the k x k work matrix A += R^T S (see the file comment):
-// r_hi / r_lo = row block J transposed and split (k x 64, r[c][m] =
-// A[j0 + m][c]), read for c < j0 (the rows of the update); s_hi / s_lo = the
-// same with columns c < j0 negated (the columns of the update).  Both written
-// by the caller.  A timeout sets *d_info = k + 1.
-gptq_status tc_rank_update(float* A, int k, int j0, int b, const float* s_hi, const float* s_lo,
-                           const float* r_hi, const float* r_lo, int32_t* d_info, cudaStream_t s) {
-  if (j0 <= 0) return GPTQ_OK;
+// Rows [row0, row1) of the k x k work matrix A += R^T S (see the file
+// comment): r_hi / r_lo = row blocks transposed and split, r[c][m] =
+// A[j0 + m][c] for the K = K rows m of the update, read for the output rows c;
+// s_hi / s_lo = the same with the Schur columns (c < split) negated, read for
+// every column c.  Both have row stride ld_s and start at the update's first
+// K column (16-byte aligned); written by the caller.  The output map ends at
+// row row1 and the operands' at column K.  A timeout sets *d_info = k + 1.
+gptq_status tc_rank_update(float* A, int k, int row0, int row1, int split, int K, int ld_s,
+                           const float* s_hi, const float* s_lo, const float* r_hi,
+                           const float* r_lo, int32_t* d_info, cudaStream_t s) {
+  if (row1 <= row0 || K <= 0) return GPTQ_OK;
   CUtensorMap ah, al, bh, bl, dm;
-  // D's map ends at row j0: rows at and below the current row block are never touched
-  if (!make_map(&ah, r_hi, 64, j0, 64, TX_M) || !make_map(&al, r_lo, 64, j0, 64, TX_M) ||
-      !make_map(&bh, s_hi, 64, k, 64, TX_N) || !make_map(&bl, s_lo, 64, k, 64, TX_N) ||
-      !make_map(&dm, A, k, j0, k, TX_M))
+  if (!make_map(&ah, r_hi, K, row1, ld_s, TX_M) || !make_map(&al, r_lo, K, row1, ld_s, TX_M) ||
+      !make_map(&bh, s_hi, K, k, ld_s, TX_N) || !make_map(&bl, s_lo, K, k, ld_s, TX_N) ||
+      !make_map(&dm, A, k, row1, k, TX_M))
     return GPTQ_ERR_INVALID_ARG;
   TxArgs a;
   a.D = A;
   a.ldd = k;
-  a.M = j0;
+  a.M = row1 - row0;
   a.N = k;
-  a.row0 = 0;
+  a.row0 = row0;
   a.col0 = 0;
-  a.K = b;
+  a.K = K;
   a.a_k0 = 0;
-  a.a_r0 = 0;
+  a.a_r0 = row0;
   a.b_k0 = 0;
   a.b_r0 = 0;
-  a.ntm = (int)cdiv(j0, TX_M);
+  a.ntm = (int)cdiv(row1 - row0, TX_M);
   a.ntiles = a.ntm * (int)cdiv(k, TX_N);
   a.mode = 1;
-  a.split = j0;
+  a.split = split;
   a.status = d_info;
   a.status_code = k + 1;
   return launch(ah, al, bh, bl, dm, a, s);

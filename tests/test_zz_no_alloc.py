@@ -111,6 +111,31 @@ def test_noalloc_cuda_core_update_at_full_width(name, k):
         rel = float((got[0].double() - ref[0].double()).abs().max() / ref[0].double().abs().max())
         print(f"k={k} act_order={act_order}: max |dU| / max |U| = {rel:.3e}")
         _assert_match(ref, got)
+    print(f"k={k}: device ms workspace / no-alloc = {_time_both(H, cfg)}")
+
+
+def _time_both(H, cfg):
+    """Device time of one call of each entry point (for the record)."""
+    from post_weight_quantization_23_b200 import _lib
+    k = H.shape[0]
+    U = torch.empty(k, k, device="cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    perm, invperm, d_info = torch.empty(k, **i32), torch.empty(k, **i32), torch.empty(1, **i32)
+    dead = torch.empty(k, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(_lib.workspace_size(_lib.OP_PREPARE_HINV, 0, k, 0, cfg), dtype=torch.uint8,
+                     device="cuda")
+    out = []
+    for noalloc in (False, True):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        if noalloc:
+            _lib.prepare_hinv_noalloc(H, cfg, U, perm, invperm, dead, d_info)
+        else:
+            _lib.prepare_hinv(H, cfg, U, perm, invperm, dead, d_info, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        out.append(round(e0.elapsed_time(e1), 2))
+    return out
 
 
 def test_noalloc_rejects_k_beyond_its_scratch():
