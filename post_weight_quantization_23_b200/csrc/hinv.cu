@@ -205,20 +205,16 @@ constexpr int K1_BS = 16;                 // block size
 constexpr int K1_NB = HV_B / K1_BS;       // blocks per side
 constexpr int K1_LD = HV_B + 1;
 
-// Lower Cholesky and inverse of the 16 x 16 block at (c0, c0) of S, by one
-// warp: lane i (and its mirror i + 16) holds row i.  M goes back to S, N =
-// M^-1 to T (lower parts).  Returns the index of the first pivot that is not
-// positive and finite, or -1 (the same on every lane).
-__device__ __forceinline__ int chol_inv16_warp(float (*S)[K1_LD], float (*T)[K1_LD], int c0,
-                                               int lane) {
-  const int i = lane & 15;
-  float a[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) a[j] = (j <= i) ? S[c0 + i][c0 + j] : 0.f;
-  int bad = -1;
-  float myr = 0.f;
-#pragma unroll
-  for (int C = 0; C < 16; ++C) {
+// Lower Cholesky of the 16 x 16 block at (c0, c0) of S, by one warp: lane i
+// (and its mirror i + 16) holds row i in registers and the pivots' columns are
+// passed along by shuffles.  M goes back to S (lower part), 1 / M_ii to
+// rd[c0 + i].  Returns the index of the first pivot that is not positive and
+// finite, or -1 (the same on every lane).
+// Pivot C of chol16_rows and the ones after it, unrolled at compile time by
+// template recursion (so that a[] stays in registers).
+template <int C>
+struct Chol16Rows {
+  __device__ __forceinline__ static void run(float (&a)[16], int i, float& myr, int& bad) {
     const float p = __shfl_sync(0xffffffffu, a[C], C);
     if ((!(p > 0.f) || !isfinite(p)) && bad < 0) bad = C;
     const float r = rsqrtf(p);  // 1 / sqrt(p), within 2 ulp
@@ -229,30 +225,50 @@ __device__ __forceinline__ int chol_inv16_warp(float (*S)[K1_LD], float (*T)[K1_
       const float lj = __shfl_sync(0xffffffffu, a[C], j);
       if (i >= j) a[j] = fmaf(-a[C], lj, a[j]);
     }
+    Chol16Rows<C + 1>::run(a, i, myr, bad);
   }
-  // N = M^-1 row by row: N_mm = 1 / M_mm, N_mj = -(sum_{q=j}^{m-1} M_mq N_qj) / M_mm
-  float n[16], acc[16];
+};
+template <>
+struct Chol16Rows<16> {
+  __device__ __forceinline__ static void run(float (&)[16], int, float&, int&) {}
+};
+
+__device__ __forceinline__ int chol16_rows(float (*S)[K1_LD], float* rd, int c0, int lane) {
+  const int i = lane & 15;
+  float a[16];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) n[j] = 0.f, acc[j] = 0.f;
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    if (i == m) {
-#pragma unroll
-      for (int j = 0; j < m; ++j) n[j] = -acc[j] * myr;
-      n[m] = myr;
-    }
-#pragma unroll
-    for (int j = 0; j <= m; ++j) {
-      const float v = __shfl_sync(0xffffffffu, n[j], m);
-      if (i > m) acc[j] = fmaf(a[m], v, acc[j]);
-    }
-  }
+  for (int j = 0; j < 16; ++j) a[j] = (j <= i) ? S[c0 + i][c0 + j] : 0.f;
+  int bad = -1;
+  float myr = 0.f;
+  Chol16Rows<0>::run(a, i, myr, bad);
   if (lane < 16) {
 #pragma unroll
     for (int j = 0; j < 16; ++j)
-      if (j <= i) S[c0 + i][c0 + j] = a[j], T[c0 + i][c0 + j] = n[j];
+      if (j <= i) S[c0 + i][c0 + j] = a[j];
+    rd[c0 + i] = myr;
   }
   return bad;
+}
+
+// N = M^-1 of the 16 x 16 lower block at (c0, c0) of S, into T: lane j < 16
+// solves for column j (x_j = 1 / M_jj, x_i = -(sum_{m=j}^{i-1} M_im x_m) / M_ii),
+// every lane reading the same row of M at a time (broadcast).
+__device__ __forceinline__ void inv16_cols(const float (*S)[K1_LD], float (*T)[K1_LD],
+                                           const float* rd, int c0, int lane) {
+  if (lane >= 16) return;
+  const int j = lane;
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float acc = 0.f;
+#pragma unroll
+    for (int m = 0; m < i; ++m) acc = fmaf(S[c0 + i][c0 + m], x[m], acc);
+    const float r = rd[c0 + i];
+    x[i] = (i < j) ? 0.f : (i == j ? r : -acc * r);
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (i >= j) T[c0 + i][c0 + j] = x[i];
 }
 
 __global__ void __launch_bounds__(256)
@@ -267,6 +283,7 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
   __shared__ float T[HV_B][K1_LD];                  // N = M^-1 (lower part)
   __shared__ float Mt[HV_B - K1_BS][K1_BS + 1];     // M_ik of the current block column
   __shared__ float Xs[K1_NB - 1][K1_BS][K1_BS + 1];  // X_m of the current block row
+  __shared__ float rdg[HV_B];                        // 1 / M_ii
   __shared__ int fail;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   for (int e = t; e < HV_B * HV_B; e += 256) {
@@ -297,8 +314,10 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
     const int c0 = kb * K1_BS, r0 = c0 + K1_BS, nr = HV_B - r0;
     // (A) the diagonal block
     if (warp == 0) {
-      const int bad = chol_inv16_warp(S, T, c0, lane);
+      const int bad = chol16_rows(S, rdg, c0, lane);
       if (lane == 0 && bad >= 0) fail = c0 + bad;
+      __syncwarp();
+      inv16_cols(S, T, rdg, c0, lane);
     }
     __syncthreads();
     if (fail >= 0) break;
@@ -315,8 +334,11 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
         const int f = e - nr * K1_BS, mb = f / (K1_BS * K1_BS);
         const int q = (f / K1_BS) % K1_BS, c = f % K1_BS;
         float acc = 0.f;
-        for (int col = mb * K1_BS; col < c0; ++col)
-          acc = fmaf(S[c0 + q][col], T[col][mb * K1_BS + c], acc);
+        for (int l = mb; l < kb; ++l) {
+#pragma unroll
+          for (int p = 0; p < K1_BS; ++p)
+            acc = fmaf(S[c0 + q][l * K1_BS + p], T[l * K1_BS + p][mb * K1_BS + c], acc);
+        }
         Xs[mb][q][c] = acc;
       }
     }
