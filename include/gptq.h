@@ -203,9 +203,9 @@ GPTQ_API void gptq_set_wait_limit(uint32_t polls);
  *            gptq_prepare_hinv; U agrees with its U within fp32 rounding
  *            (1e-5 relative to max |U|), not bit for bit, because the array
  *            holds less of the rank updates' operand splits than the
- *            workspace does: up to k = 4060 the tensor-core updates run with
+ *            workspace does: up to k = 4076 the tensor-core updates run with
  *            one level of 64-column blocks (gptq_prepare_hinv batches 8 of
- *            them per update), and from k = 4064 to 12288 the fp32 CUDA-core
+ *            them per update), and from k = 4080 to 12288 the fp32 CUDA-core
  *            rank update runs instead, which is slower (at k = 4096 about 4x).
  *   Setup.   Host code cannot hand the array's name to a kernel; its device
  *            address comes from cudaGetSymbolAddress, looked up with the

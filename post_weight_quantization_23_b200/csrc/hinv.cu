@@ -14,8 +14,8 @@
 // (rows above the processed part) and turns into U row block by row block.
 // Blocks of HV_B = 64 indices, from the last one up; step J = [j0, j1), e = j1:
 //   K1 diag    L_JJ from the Schur-updated diagonal block (lower part) and
-//              U_JJ = (L_JJ^T)^-1, written to A[J, J] (upper) and the scratch
-//              (blocked in 16 x 16 pieces inside one CTA).
+//              U_JJ = (L_JJ^T)^-1, written to A[J, J] (upper part; blocked in
+//              16 x 16 pieces inside one CTA).
 //   K2 panel   P = L[J, 0:j0] = U_JJ * Hp[J, 0:j0]   (in place, lower part),
 //      and     U[J, e:] = -U_JJ * Y[J, e:]          (in place, upper part):
 //              V = [[V_JJ, V_J*], [0, V_**]] gives U_J* = -V_JJ^-1 V_J* U_**.
@@ -57,7 +57,6 @@ struct HinvScratch {
   double* sum_diag;  // [1]
   float* lambda;     // [1]
   float* diag;       // [k] diag(H) after the dead-column fix
-  float* ujj;        // [HV_B * HV_B] U_JJ of the current step
   float* s_hi;       // [k * HV_O] signed splits of the outer block's row blocks, transposed
   float* s_lo;       //   (tensor-core path; row block J at column j0 - o0)
   float* r_hi;       // [k * HV_O] unsigned splits (columns < j0 only)
@@ -70,7 +69,6 @@ size_t hinv_workspace_min_bytes(int64_t k) {
   b += align256(sizeof(double));
   b += align256(sizeof(float));
   b += align256(sizeof(float) * (size_t)k);
-  b += align256(sizeof(float) * HV_B * HV_B);
   return b;
 }
 
@@ -91,7 +89,6 @@ static HinvScratch carve(void* ws, int64_t k, int outer) {
   s.sum_diag = (double*)p; p += align256(sizeof(double));
   s.lambda = (float*)p; p += align256(sizeof(float));
   s.diag = (float*)p; p += align256(sizeof(float) * (size_t)k);
-  s.ujj = (float*)p; p += align256(sizeof(float) * HV_B * HV_B);
   float* t[4] = {nullptr, nullptr, nullptr, nullptr};
   for (int i = 0; i < 4 && outer > 0; ++i) {
     t[i] = (float*)p;
@@ -191,25 +188,33 @@ __device__ __forceinline__ void set_info(int32_t* d_info, int idx) { atomicCAS(d
 // factorisation that starts from the last index) becomes the ordinary lower
 // Cholesky B = M M^T with M = P L^T P, and U_JJ = (L^T)^-1 = P M^-1 P.  The
 // kernel factors B and inverts M together, in 16 x 16 blocks (rows and
-// columns past b padded with the identity), block column kb = 0..3:
-//   (A) one warp: M_kk = chol(B_kk) and N_kk = M_kk^-1, lane i holding row i
-//       in registers, the pivots' columns passed along by shuffles;
-//   (B) the CTA: M_ik = B_ik N_kk^T for the rows below (a product, no
-//       substitution chain), and X_m = sum_{l=m}^{kb-1} M_kl N_lm for m < kb;
-//   (C) the CTA: B_ij -= M_ik M_jk^T below, and the inverse's block row
-//       N_km = -N_kk X_m (m < kb), so N = M^-1 is complete when the loop ends.
-// U_JJ goes to the scratch, to the upper part of A[J, J] and, transposed and
-// split into tf32 hi / lo, to the rank update's operand (row stride ld_s,
-// column offset s_off).
+// columns past b padded with the identity), block column kb = 0..3, with two
+// roles so that the serial chain of diagonal blocks runs at the speed of one
+// warp:
+//   warp 0 (diagonal): M_kk = chol(B_kk) and N_kk = M_kk^-1, lane i holding
+//     row i in registers, the pivots' columns passed along by shuffles; then
+//     it hands N_kk over and waits for the next diagonal block;
+//   warps 1-7 (bulk): M_ik = B_ik N_kk^T for block row kb+1 first, the rank-16
+//     update of diagonal block kb+1 (handed to warp 0 at once), then the
+//     rest: M_ik for the rows further down, their rank-16 update, and the
+//     inverse's block row N_km = -N_kk sum_{l=m}^{kb-1} M_kl N_lm (m < kb), so
+//     that N = M^-1 is complete when the loop ends.
+// The hand-overs are named barriers (arrive by the producer, sync by the
+// consumer); every thread takes the same sequence of barriers whatever the
+// data (a failed pivot only marks the result).  U_JJ goes to the upper part of
+// A[J, J]; the panel kernel reads it from there.
 constexpr int K1_BS = 16;                 // block size
 constexpr int K1_NB = HV_B / K1_BS;       // blocks per side
 constexpr int K1_LD = HV_B + 1;
+constexpr int K1_BULK = 224;              // threads of warps 1-7
 
-// Lower Cholesky of the 16 x 16 block at (c0, c0) of S, by one warp: lane i
-// (and its mirror i + 16) holds row i in registers and the pivots' columns are
-// passed along by shuffles.  M goes back to S (lower part), 1 / M_ii to
-// rd[c0 + i].  Returns the index of the first pivot that is not positive and
-// finite, or -1 (the same on every lane).
+__device__ __forceinline__ void k1_bar_sync(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void k1_bar_arrive(uint32_t id, uint32_t n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // Pivot C of chol16_rows and the ones after it, unrolled at compile time by
 // template recursion (so that a[] stays in registers).
 template <int C>
@@ -272,10 +277,7 @@ __device__ __forceinline__ void inv16_cols(const float (*S)[K1_LD], float (*T)[K
 }
 
 __global__ void __launch_bounds__(256)
-chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
-                     float* __restrict__ ujj, float* __restrict__ st_hi,
-                     float* __restrict__ st_lo, int ld_s, int s_off, int s_prev,
-                     int32_t* __restrict__ d_info) {
+chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b, int32_t* __restrict__ d_info) {
   pdl_wait();
   pdl_trigger();
   if (*d_info != 0) return;
@@ -310,100 +312,118 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
   }
   __syncthreads();
 
-  for (int kb = 0; kb < K1_NB; ++kb) {
-    const int c0 = kb * K1_BS, r0 = c0 + K1_BS, nr = HV_B - r0;
-    // (A) the diagonal block
-    if (warp == 0) {
+  if (warp == 0) {
+    for (int kb = 0; kb < K1_NB; ++kb) {
+      const int c0 = kb * K1_BS;
+      if (kb > 0) k1_bar_sync(2, 256);  // diagonal block kb updated by the bulk warps
       const int bad = chol16_rows(S, rdg, c0, lane);
-      if (lane == 0 && bad >= 0) fail = c0 + bad;
+      if (lane == 0 && bad >= 0 && fail < 0) fail = c0 + bad;
       __syncwarp();
       inv16_cols(S, T, rdg, c0, lane);
+      __syncwarp();
+      k1_bar_arrive(1, 256);            // M_kk, N_kk ready
     }
-    __syncthreads();
-    if (fail >= 0) break;
-    // (B) M_ik = B_ik N_kk^T (rows below), X_m for the inverse's block row kb
-    for (int e = t; e < nr * K1_BS + kb * K1_BS * K1_BS; e += 256) {
-      if (e < nr * K1_BS) {
-        const int ii = e / K1_BS, j = e % K1_BS;
-        float acc = 0.f;
+  } else {
+    const int u = t - 32;  // 0 .. K1_BULK - 1
+    for (int kb = 0; kb < K1_NB; ++kb) {
+      const int c0 = kb * K1_BS, r0 = c0 + K1_BS, nr = HV_B - r0;
+      k1_bar_sync(1, 256);
+      if (kb + 1 < K1_NB) {
+        // block row kb + 1 first: M_{kb+1,kb} = B_{kb+1,kb} N_kk^T ...
+        for (int e = u; e < K1_BS * K1_BS; e += K1_BULK) {
+          const int ii = e / K1_BS, j = e % K1_BS;
+          float acc = 0.f;
 #pragma unroll
-        for (int m = 0; m < K1_BS; ++m)
-          if (m <= j) acc = fmaf(S[r0 + ii][c0 + m], T[c0 + j][c0 + m], acc);
-        Mt[ii][j] = acc;
-      } else {
-        const int f = e - nr * K1_BS, mb = f / (K1_BS * K1_BS);
-        const int q = (f / K1_BS) % K1_BS, c = f % K1_BS;
-        float acc = 0.f;
-        for (int l = mb; l < kb; ++l) {
-#pragma unroll
-          for (int p = 0; p < K1_BS; ++p)
-            acc = fmaf(S[c0 + q][l * K1_BS + p], T[l * K1_BS + p][mb * K1_BS + c], acc);
+          for (int m = 0; m < K1_BS; ++m)
+            if (m <= j) acc = fmaf(S[r0 + ii][c0 + m], T[c0 + j][c0 + m], acc);
+          Mt[ii][j] = acc;
         }
-        Xs[mb][q][c] = acc;
-      }
-    }
-    __syncthreads();
-    // (C) M_ik back into B, the trailing update, the inverse's block row kb
-    for (int e = t; e < nr * K1_BS; e += 256) {
-      const int ii = e / K1_BS, j = e % K1_BS;
-      S[r0 + ii][c0 + j] = Mt[ii][j];
-    }
-    for (int e = t; e < nr * nr; e += 256) {
-      const int ii = e / nr, jj = e % nr;
-      if (jj <= ii) {
-        float acc = S[r0 + ii][r0 + jj];
+        k1_bar_sync(3, K1_BULK);
+        // ... and the rank-16 update of diagonal block kb + 1
+        for (int e = u; e < K1_BS * K1_BS; e += K1_BULK) {
+          const int ii = e / K1_BS, jj = e % K1_BS;
+          if (jj <= ii) {
+            float acc = S[r0 + ii][r0 + jj];
 #pragma unroll
-        for (int m = 0; m < K1_BS; ++m) acc = fmaf(-Mt[ii][m], Mt[jj][m], acc);
-        S[r0 + ii][r0 + jj] = acc;
+            for (int m = 0; m < K1_BS; ++m) acc = fmaf(-Mt[ii][m], Mt[jj][m], acc);
+            S[r0 + ii][r0 + jj] = acc;
+          }
+          S[r0 + ii][c0 + jj] = Mt[ii][jj];
+        }
+        k1_bar_arrive(2, 256);  // diagonal block kb + 1 ready
       }
-    }
-    for (int e = t; e < kb * K1_BS * K1_BS; e += 256) {
-      const int mb = e / (K1_BS * K1_BS), r = (e / K1_BS) % K1_BS, c = e % K1_BS;
-      float acc = 0.f;
+      // the rows below block row kb + 1, and X_m for the inverse's block row kb
+      const int nr2 = nr > K1_BS ? nr - K1_BS : 0;
+      for (int e = u; e < nr2 * K1_BS + kb * K1_BS * K1_BS; e += K1_BULK) {
+        if (e < nr2 * K1_BS) {
+          const int ii = K1_BS + e / K1_BS, j = e % K1_BS;
+          float acc = 0.f;
 #pragma unroll
-      for (int q = 0; q < K1_BS; ++q)
-        if (q <= r) acc = fmaf(T[c0 + r][c0 + q], Xs[mb][q][c], acc);
-      T[c0 + r][mb * K1_BS + c] = -acc;
+          for (int m = 0; m < K1_BS; ++m)
+            if (m <= j) acc = fmaf(S[r0 + ii][c0 + m], T[c0 + j][c0 + m], acc);
+          Mt[ii][j] = acc;
+        } else {
+          const int f = e - nr2 * K1_BS, mb = f / (K1_BS * K1_BS);
+          const int q = (f / K1_BS) % K1_BS, c = f % K1_BS;
+          float acc = 0.f;
+          for (int l = mb; l < kb; ++l) {
+#pragma unroll
+            for (int p = 0; p < K1_BS; ++p)
+              acc = fmaf(S[c0 + q][l * K1_BS + p], T[l * K1_BS + p][mb * K1_BS + c], acc);
+          }
+          Xs[mb][q][c] = acc;
+        }
+      }
+      k1_bar_sync(3, K1_BULK);
+      // M_ik back into B, the rank-16 update below block row kb + 1 (rows and
+      // columns from r0 + 16 down, and block column kb + 1 of those rows),
+      // the inverse's block row kb
+      for (int e = u; e < nr2 * K1_BS; e += K1_BULK) {
+        const int ii = K1_BS + e / K1_BS, j = e % K1_BS;
+        S[r0 + ii][c0 + j] = Mt[ii][j];
+      }
+      for (int e = u; e < nr2 * nr; e += K1_BULK) {
+        const int ii = K1_BS + e / nr, jj = e % nr;
+        if (jj <= ii) {
+          float acc = S[r0 + ii][r0 + jj];
+#pragma unroll
+          for (int m = 0; m < K1_BS; ++m) acc = fmaf(-Mt[ii][m], Mt[jj][m], acc);
+          S[r0 + ii][r0 + jj] = acc;
+        }
+      }
+      for (int e = u; e < kb * K1_BS * K1_BS; e += K1_BULK) {
+        const int mb = e / (K1_BS * K1_BS), r = (e / K1_BS) % K1_BS, c = e % K1_BS;
+        float acc = 0.f;
+#pragma unroll
+        for (int q = 0; q < K1_BS; ++q)
+          if (q <= r) acc = fmaf(T[c0 + r][c0 + q], Xs[mb][q][c], acc);
+        T[c0 + r][mb * K1_BS + c] = -acc;
+      }
+      k1_bar_sync(3, K1_BULK);
     }
-    __syncthreads();
   }
+  __syncthreads();
   if (fail >= 0) {
     if (t == 0) set_info(d_info, j0 + (b - 1 - fail));
     return;
   }
-  // U_JJ[iu][cu] = N[b-1-iu][b-1-cu] (iu <= cu < b)
+  // U_JJ[iu][cu] = N[b-1-iu][b-1-cu] (iu <= cu < b) into the upper part of A[J, J]
   for (int e = t; e < HV_B * HV_B; e += 256) {
     const int iu = e / HV_B, cu = e % HV_B;
-    const bool in = (iu <= cu && cu < b);
-    const float u = in ? T[b - 1 - iu][b - 1 - cu] : 0.f;
-    ujj[e] = u;
-    if (in) A[(int64_t)(j0 + iu) * k + j0 + cu] = u;
-  }
-  if (st_hi != nullptr) {
-    // rank-update operand s[j0 + cu][s_off + iu] = U_JJ[iu][cu]  (columns of block J, sign +)
-    for (int e = t; e < b * HV_B; e += 256) {
-      const int cu = e / HV_B, iu = e % HV_B;
-      const float u = (iu <= cu) ? T[b - 1 - iu][b - 1 - cu] : 0.f;
-      float h, l;
-      hv_split_tf32(u, h, l);
-      st_hi[(int64_t)(j0 + cu) * ld_s + s_off + iu] = h;
-      st_lo[(int64_t)(j0 + cu) * ld_s + s_off + iu] = l;
-      if (s_prev >= 0) {
-        // the block below in the same outer block: its Schur part at these
-        // columns was used by its band update and must not reach the outer one
-        st_hi[(int64_t)(j0 + cu) * ld_s + s_prev + iu] = 0.f;
-        st_lo[(int64_t)(j0 + cu) * ld_s + s_prev + iu] = 0.f;
-      }
-    }
+    if (iu <= cu && cu < b) A[(int64_t)(j0 + iu) * k + j0 + cu] = T[b - 1 - iu][b - 1 - cu];
   }
 }
 
-// K2, one launch, two independent roles (16-column tiles, so that the launch
-// fills the GPU; each CTA reads its whole 64 x 16 tile before writing it):
+// K2, one launch, three independent roles (16-column tiles, so that the launch
+// fills the GPU; each CTA reads U_JJ from the upper part of A[J, J] and its
+// whole 64 x 16 tile before writing it):
 //   CTAs [0, n_pan): columns c0 .. c0+15 of [0, j0): P[:, c] = U_JJ * A[J, c]
 //     (lower part of row block J, in place).
-//   CTAs [n_pan, ...): columns c0 .. c0+15 of [e, k): U[J, c] = -U_JJ * Y[J, c]
-//     (upper part of row block J, in place).
+//   CTAs [n_pan, n_pan + n_row): columns c0 .. c0+15 of [e, k): U[J, c] =
+//     -U_JJ * Y[J, c] (upper part of row block J, in place).
+//   With st_hi given, cdiv(b, 16) more CTAs: block J's own columns of the
+//     operand, st[j0 + c][s_off + m] = U_JJ[m][c] (0 below the diagonal), and
+//     the s_prev slice cleared there.
 //   With the tensor-core update (st_hi given) each panel CTA also zeroes rows
 //     [c0, c0 + 16) of the strip A[0:j0, j0:j1], where Y's columns of block J
 //     start accumulating in this step's update (the tensor-core Schur update
@@ -419,8 +439,8 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b,
 constexpr int K2_W = 16;  // columns per CTA
 
 __global__ void __launch_bounds__(256)
-panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* __restrict__ ujj,
-                      int n_pan, float* __restrict__ st_hi, float* __restrict__ st_lo,
+panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, int n_pan, int n_row,
+                      float* __restrict__ st_hi, float* __restrict__ st_lo,
                       float* __restrict__ rt_hi, float* __restrict__ rt_lo, int ld_s, int s_off,
                       int o0, int s_prev, const int32_t* __restrict__ d_info) {
   pdl_wait();
@@ -430,16 +450,50 @@ panel_rowblock_kernel(float* __restrict__ A, int k, int j0, int b, const float* 
   __shared__ __align__(16) float Hs[HV_B][K2_W + 4];  // row stride 20: aligned float4 rows
   __shared__ float Os[HV_B][K2_W + 1];                // results; stride 17: conflict-free columns
   const int t = threadIdx.x;
+  const bool vec = (k % 4 == 0);
+  if ((int)blockIdx.x >= n_pan + n_row) {
+    // block J's own columns of the operand: U_JJ (upper triangle) transposed and split
+    const int d0 = ((int)blockIdx.x - n_pan - n_row) * K2_W;
+#pragma unroll
+    for (int q = 0; q < K2_W * HV_B / 256; ++q) {
+      const int e = t + 256 * q, cc = d0 + e / HV_B, m = e % HV_B;
+      if (cc < b) {
+        const float u = (m <= cc) ? A[(int64_t)(j0 + m) * k + j0 + cc] : 0.f;
+        float h, l;
+        hv_split_tf32(u, h, l);
+        const int64_t o = (int64_t)(j0 + cc) * ld_s + s_off + m;
+        st_hi[o] = h;
+        st_lo[o] = l;
+        if (s_prev >= 0) {
+          st_hi[o - s_off + s_prev] = 0.f;
+          st_lo[o - s_off + s_prev] = 0.f;
+        }
+      }
+    }
+    return;
+  }
   const bool pan = (int)blockIdx.x < n_pan;
   const int c0 = pan ? blockIdx.x * K2_W : j0 + b + (blockIdx.x - n_pan) * K2_W;
   const int cend = pan ? j0 : k;
   const float sign = pan ? 1.0f : -1.0f;
-  const bool vec = (k % 4 == 0);
   const int r = t >> 2, j = (t & 3) * 4;  // this thread's row and first column in the tile
   {
+    // U_JJ from the upper part of A[J, J]; only entries (row, col >= row) are
+    // used below, so the lower part's contents do not matter
     float4 uv[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) uv[q] = reinterpret_cast<const float4*>(ujj)[t + 256 * q];
+    for (int q = 0; q < 4; ++q) {
+      const int e4 = t + 256 * q, ur = e4 >> 4, uc = (e4 & 15) * 4;
+      const float* us = A + (int64_t)(j0 + ur) * k + j0 + uc;
+      if (ur < b && vec && uc + 3 < b) {
+        uv[q] = *reinterpret_cast<const float4*>(us);
+      } else {
+        uv[q].x = (ur < b && uc < b) ? us[0] : 0.f;
+        uv[q].y = (ur < b && uc + 1 < b) ? us[1] : 0.f;
+        uv[q].z = (ur < b && uc + 2 < b) ? us[2] : 0.f;
+        uv[q].w = (ur < b && uc + 3 < b) ? us[3] : 0.f;
+      }
+    }
     float4 hv;
     const float* src = A + (int64_t)(j0 + r) * k + c0 + j;
     if (r < b && vec && c0 + j + 3 < cend) {
@@ -681,14 +735,14 @@ gptq_status prepare_hinv_impl(const float* H, int64_t k64, const gptq_config* cf
       const bool tcs = tc && j0 > 0;
       const int s_off = j0 - o0;
       const int s_prev = (tcs && j1 < o1) ? j1 - o0 : -1;  // the block below, same outer block
-      launch_pdl(chol_inv_diag_kernel, dim3(1), dim3(256), 0, s, U, k, j0, b, sc.ujj,
-                 tcs ? sc.s_hi : nullptr, tcs ? sc.s_lo : nullptr, outer, s_off, s_prev, d_info);
+      launch_pdl(chol_inv_diag_kernel, dim3(1), dim3(256), 0, s, U, k, j0, b, d_info);
       GPTQ_CHECK_LAUNCH();
       const int n_pan = (int)cdiv(j0, K2_W);
       const int n_row = (int)cdiv(k - j1, K2_W);
-      if (n_pan + n_row > 0) {
-        launch_pdl(panel_rowblock_kernel, dim3((unsigned)(n_pan + n_row)), dim3(256), 0, s, U, k,
-                   j0, b, (const float*)sc.ujj, n_pan, tcs ? sc.s_hi : nullptr,
+      const int n_diag = tcs ? (int)cdiv(b, K2_W) : 0;
+      if (n_pan + n_row + n_diag > 0) {
+        launch_pdl(panel_rowblock_kernel, dim3((unsigned)(n_pan + n_row + n_diag)), dim3(256), 0,
+                   s, U, k, j0, b, n_pan, n_row, tcs ? sc.s_hi : nullptr,
                    tcs ? sc.s_lo : nullptr, tcs ? sc.r_hi : nullptr, tcs ? sc.r_lo : nullptr,
                    outer, s_off, o0, s_prev, (const int32_t*)d_info);
         GPTQ_CHECK_LAUNCH();

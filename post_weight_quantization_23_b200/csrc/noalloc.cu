@@ -12,7 +12,7 @@
 //
 // The array is `kScratchBytes` (4 MiB) on every device that loads the
 // library and is held until the process exits; it covers k up to
-// kNoAllocMaxK = 12288.  Up to k = 4060 the tensor-core rank updates' operand
+// kNoAllocMaxK = 12288.  Up to k = 4076 the tensor-core rank updates' operand
 // splits for one 64-column block fit beside the rest (one-level updates, where
 // gptq_prepare_hinv batches 8 blocks); above, the fp32 CUDA-core rank update
 // runs instead (slower).  Either way U equals gptq_prepare_hinv's within fp32

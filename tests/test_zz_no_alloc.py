@@ -97,7 +97,7 @@ def _gpu_hessian(spec, seed):
 
 @pytest.mark.parametrize("name,k", [("q_proj", 4096), ("opt175_width", 12288)])
 def test_noalloc_cuda_core_update_at_full_width(name, k):
-    """From k = 4064 the operand splits of the tensor-core rank update no
+    """From k = 4080 the operand splits of the tensor-core rank update no
     longer fit in the built-in scratch, so the call takes the fp32 CUDA-core
     rank update (a triangular tile schedule over several row tiles): at the
     q_proj width and at the OPT-175B width, twice in a row, against the
