@@ -60,8 +60,12 @@ struct QvShape {
   static constexpr uint32_t MASK = (1u << BITS) - 1u;
 };
 
-inline int qv_kc(int k, int slab) {
-  const int kc = k < QV_KC ? k : QV_KC;
+// Columns of X staged per pass for M tokens (the staging buffer stays under
+// 150 KB of shared memory).
+constexpr int qv_kc_max(int M) { return M <= 4 ? QV_KC : QV_KC / 2; }
+
+inline int qv_kc(int k, int slab, int M) {
+  const int kc = k < qv_kc_max(M) ? k : qv_kc_max(M);
   return (int)(cdiv(kc, slab) * slab);
 }
 
@@ -144,7 +148,13 @@ __device__ __forceinline__ void qv_compute(const QvSlab<BITS>& S, const float* x
     for (int t = 0; t < M; ++t) y[i][t] = fmaf(S.sc[i], acc[i][t].x + acc[i][t].y, y[i][t]);
 }
 
-// Decode kernel: CTA = 16 rows x M tokens, 8 warps sharing the column slabs.
+// Decode kernel: CTA = 16 rows x M tokens (M = 1, 2, 4 or 8), 8 warps sharing
+// the column slabs.  The CTAs of one row block are consecutive (the block index
+// runs over the token groups first), so a second token group finds the row
+// block's packed words in L2.  Launched with programmatic dependent launch:
+// the first slab of packed words is requested before waiting for the previous
+// kernel (only X depends on it; the weights must not be written by a kernel
+// that lets this one start early).
 // Lane (q = lane / 8, p = lane % 8) loads, for i = 0..3, the 16-byte piece p
 // of row 4 i + q in its warp's slab, so each load instruction reads four whole
 // 128-byte row segments.  The first slab's words are requested before the
@@ -164,8 +174,9 @@ qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
   float* red = xs + M * XS;       // [QV_WARPS][M][QV_ROWS] per-warp row sums
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int q = lane >> 3, p = lane & 7;
-  const int r0 = blockIdx.x * QV_ROWS;
-  const int t0 = blockIdx.y * M;
+  const int ntg = (m + M - 1) / M;
+  const int r0 = (int)(blockIdx.x / ntg) * QV_ROWS;
+  const int t0 = (int)(blockIdx.x % ntg) * M;
   const int64_t wpr = (int64_t)k / Sh::CPW;  // words per row
 
   float y[QV_RPL][M];
@@ -182,6 +193,11 @@ qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
     {
       const int cl = sl + p * Sh::CH;
       qv_load<BITS>(cur, qw, scales, zeros, wpr, r0, q, n, kc0 + cl, cl < kcw, G, ngroups);
+    }
+    if (kc0 == 0) {
+      // X comes from the previous kernel
+      pdl_wait();
+      pdl_trigger();
     }
     __syncthreads();  // the previous pass is done with xs
     if (xvec) {
@@ -305,17 +321,20 @@ gptq_status launch_qgemv(const T* X, int64_t ldx, int m, int k, const int32_t* q
                          const float* scales, const int32_t* zeros, int n, int G, int ngroups,
                          T* Y, int64_t ldy, cudaStream_t s) {
   using Sh = QvShape<BITS>;
-  const int KC = qv_kc(k, Sh::SLAB);
+  const int KC = qv_kc(k, Sh::SLAB, M);
   const size_t smem = qv_smem_bytes<BITS>(M, KC);
   // opt in once per device to the most this instantiation can ask for
   if (smem > 48 * 1024 &&
-      smem_optin((const void*)qgemv_kernel<BITS, M, T>, qv_smem_bytes<BITS>(M, QV_KC)) != cudaSuccess)
+      smem_optin((const void*)qgemv_kernel<BITS, M, T>,
+                 qv_smem_bytes<BITS>(M, (int)(cdiv(qv_kc_max(M), Sh::SLAB) * Sh::SLAB))) !=
+          cudaSuccess)
     return GPTQ_ERR_CUDA;
-  const dim3 grid((unsigned)cdiv(n, QV_ROWS), (unsigned)cdiv(m, M));
+  const int64_t nblk = cdiv(n, QV_ROWS) * cdiv(m, M);
+  if (nblk > (int64_t)INT32_MAX) return GPTQ_ERR_INVALID_ARG;
   // 16-byte activation loads when every row of X starts on a 16-byte boundary
   const int xvec = ((uintptr_t)X % 16) == 0 && ldx % 8 == 0;
-  qgemv_kernel<BITS, M, T><<<grid, QV_WARPS * 32, smem, s>>>(X, ldx, m, k, qw, scales, zeros, n,
-                                                             G, ngroups, KC, xvec, Y, ldy);
+  launch_pdl(qgemv_kernel<BITS, M, T>, dim3((unsigned)nblk), dim3(QV_WARPS * 32), smem, s, X, ldx,
+             m, k, qw, scales, zeros, n, G, ngroups, KC, xvec, Y, ldy);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
 }
@@ -324,10 +343,12 @@ template <int BITS, typename T>
 gptq_status qgemv_bits(const T* X, int64_t ldx, int m, int k, const int32_t* qw,
                        const float* scales, const int32_t* zeros, int n, int G, int ngroups, T* Y,
                        int64_t ldy, cudaStream_t s) {
-  // one token, or pairs of tokens on the grid's y axis (later pairs re-read
-  // the packed weights, mostly from L2)
+  // up to 8 tokens per CTA; more tokens take several CTAs per row block,
+  // which find its packed words in L2
   if (m == 1) return launch_qgemv<BITS, 1, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
-  return launch_qgemv<BITS, 2, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
+  if (m == 2) return launch_qgemv<BITS, 2, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
+  if (m <= 4) return launch_qgemv<BITS, 4, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
+  return launch_qgemv<BITS, 8, T>(X, ldx, m, k, qw, scales, zeros, n, G, ngroups, Y, ldy, s);
 }
 
 template <typename T>

@@ -21,7 +21,8 @@
 //     tiles that lie entirely right of the diagonal inside [0, j0)^2 are
 //     skipped, the others are updated whole.
 //
-// Tiles of 128 x 256 (rows x columns) on a persistent grid; warp 0 issues the
+// Tiles of 128 x 256 (128 x 128 for updates with fewer tiles than SMs) on a
+// persistent grid; warp 0 issues the
 // operand TMA loads, warp 1 the MMAs (one thread), warps 2..5 are the
 // epilogue.  TMEM holds two accumulators, so a tile's epilogue overlaps the
 // next tile's MMAs.  D is never read by the kernel: the epilogue writes the
@@ -38,18 +39,25 @@ namespace gptq {
 
 namespace {
 
-constexpr int TX_M = 128, TX_N = 256, TX_KC = 32;   // tile rows, cols, K per stage
+constexpr int TX_M = 128, TX_KC = 32;                // tile rows, K per stage
 constexpr int TX_STAGES = 2;
 constexpr int TX_A_BYTES = TX_M * TX_KC * 4;         // 16 KB
-constexpr int TX_B_BYTES = TX_N * TX_KC * 4;         // 32 KB
-constexpr int TX_STAGE_BYTES = 2 * TX_A_BYTES + 2 * TX_B_BYTES;  // hi + lo of both: 96 KB
 constexpr int TX_THREADS = 192;                      // TMA, MMA, 4 epilogue warps
-constexpr int TX_TMEM_COLS = 512;
 constexpr int TX_DC = 32;                             // D chunk columns (one 128-byte row)
 constexpr int TX_D_BYTES = TX_M * TX_DC * 4;          // 16 KB per D chunk
 constexpr int TX_D_SLOTS = 2;
-constexpr size_t TX_SMEM =
-    (size_t)TX_STAGES * TX_STAGE_BYTES + (size_t)TX_D_SLOTS * TX_D_BYTES + 1024 + 256;
+
+// Tile width TN = 256 (large updates: more reuse of each operand byte) or 128
+// (updates with fewer tiles than SMs: twice the CTAs, half the chain of MMAs
+// and epilogue chunks per CTA).
+template <int TN>
+struct TxTile {
+  static constexpr int B_BYTES = TN * TX_KC * 4;                        // 32 / 16 KB
+  static constexpr int STAGE_BYTES = 2 * TX_A_BYTES + 2 * B_BYTES;      // hi + lo of both
+  static constexpr int TMEM_COLS = 2 * TN;                              // two accumulators
+  static constexpr size_t SMEM =
+      (size_t)TX_STAGES * STAGE_BYTES + (size_t)TX_D_SLOTS * TX_D_BYTES + 1024 + 256;
+};
 
 struct TxArgs {
   float* D;
@@ -66,28 +74,31 @@ struct TxArgs {
   uint32_t spin;  // polls before a pipeline wait gives up
 };
 
+template <int TN>
 __device__ __forceinline__ bool tile_skipped(const TxArgs& a, int m0, int n0) {
   // mode 1: a tile whose columns all lie in [0, split) and strictly right of
   // the diagonal of its rows (row0 + m0 ...) has nothing the factorisation reads
-  return a.mode == 1 && n0 + TX_N <= a.split && n0 >= a.row0 + m0 + TX_M;
+  return a.mode == 1 && n0 + TN <= a.split && n0 >= a.row0 + m0 + TX_M;
 }
 
 // Next tile of this CTA after t (t = -1: the first) that has work, or ntiles.
+template <int TN>
 __device__ __forceinline__ int next_tile(const TxArgs& a, int t) {
   for (t = (t < 0) ? (int)blockIdx.x : t + (int)gridDim.x; t < a.ntiles; t += gridDim.x) {
-    const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
-    if (!tile_skipped(a, m0, n0)) return t;
+    const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TN;
+    if (!tile_skipped<TN>(a, m0, n0)) return t;
   }
   return a.ntiles;
 }
 
+template <int TN>
 __global__ void __launch_bounds__(TX_THREADS, 1)
 tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
                      const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo,
                      const __grid_constant__ CUtensorMap d_map, TxArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* ring = smem + TX_STAGES * TX_STAGE_BYTES;  // D chunks, 1024-byte aligned
+  uint8_t* ring = smem + TX_STAGES * TxTile<TN>::STAGE_BYTES;  // D chunks, 1024-byte aligned
   uint64_t* bars = (uint64_t*)(ring + TX_D_SLOTS * TX_D_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + TX_STAGES;
@@ -122,7 +133,7 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
     tc::prefetch_tensormap(&b_lo);
     tc::prefetch_tensormap(&d_map);
   }
-  if (warp == 1) tc::tmem_alloc(tmem_slot, TX_TMEM_COLS);
+  if (warp == 1) tc::tmem_alloc(tmem_slot, TxTile<TN>::TMEM_COLS);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -131,7 +142,7 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
   pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const int nkc = (a.K + TX_KC - 1) / TX_KC;
-  const uint32_t idesc = tc::instr_desc(2, TX_M, TX_N, 0, 0);  // both operands K-major
+  const uint32_t idesc = tc::instr_desc(2, TX_M, TN, 0, 0);  // both operands K-major
 
   if (warp == 0) {
     if (lane == 0) {
@@ -142,18 +153,18 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
       for (int s = 0; s < TX_STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < a.ntiles && ok; t += gridDim.x) {
-        const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
-        if (tile_skipped(a, m0, n0)) continue;
+        const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TN;
+        if (tile_skipped<TN>(a, m0, n0)) continue;
         for (int kc = 0; kc < nkc; ++kc) {
           if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.spin)) { ok = false; break; }
-          uint8_t* sb = smem + (size_t)stage * TX_STAGE_BYTES;
-          tc::mbar_arrive_expect_tx(&full[stage], TX_STAGE_BYTES);
+          uint8_t* sb = smem + (size_t)stage * TxTile<TN>::STAGE_BYTES;
+          tc::mbar_arrive_expect_tx(&full[stage], TxTile<TN>::STAGE_BYTES);
           const int k0 = kc * TX_KC;
           tc::tma_load_2d(sb, &a_hi, &full[stage], a.a_k0 + k0, a.a_r0 + m0);
           tc::tma_load_2d(sb + TX_A_BYTES, &a_lo, &full[stage], a.a_k0 + k0, a.a_r0 + m0);
           uint8_t* bb = sb + 2 * TX_A_BYTES;
           tc::tma_load_2d(bb, &b_hi, &full[stage], a.b_k0 + k0, a.b_r0 + n0);
-          tc::tma_load_2d(bb + TX_B_BYTES, &b_lo, &full[stage], a.b_k0 + k0, a.b_r0 + n0);
+          tc::tma_load_2d(bb + TxTile<TN>::B_BYTES, &b_lo, &full[stage], a.b_k0 + k0, a.b_r0 + n0);
           issued[stage] = true;
           issued_parity[stage] = phase;
           if (++stage == TX_STAGES) stage = 0, phase ^= 1u;
@@ -174,17 +185,17 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
       uint32_t tphase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < a.ntiles && ok; t += gridDim.x) {
-        const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
-        if (tile_skipped(a, m0, n0)) continue;
+        const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TN;
+        if (tile_skipped<TN>(a, m0, n0)) continue;
         if (!tc::mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, a.spin)) { ok = false; break; }
         tc::tc_fence_after();
-        const uint32_t dcol = tmem + (uint32_t)(tb * TX_N);
+        const uint32_t dcol = tmem + (uint32_t)(tb * TN);
         for (int kc = 0; kc < nkc; ++kc) {
           if (!tc::mbar_wait(&full[stage], phase, abort_flag, a.spin)) { ok = false; break; }
           tc::tc_fence_after();
-          const uint32_t sb = tc::smem_u32(smem + (size_t)stage * TX_STAGE_BYTES);
+          const uint32_t sb = tc::smem_u32(smem + (size_t)stage * TxTile<TN>::STAGE_BYTES);
           const uint32_t ah = sb, al = sb + TX_A_BYTES;
-          const uint32_t bh = sb + 2 * TX_A_BYTES, bl = bh + TX_B_BYTES;
+          const uint32_t bh = sb + 2 * TX_A_BYTES, bl = bh + TxTile<TN>::B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < TX_KC / 8; ++kk) {
             // K-major, 128-byte swizzle: 8-row groups 1024 B apart, K step 32 B
@@ -216,14 +227,14 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
     int tb = 0, g = 0;
     uint32_t tphase = 0;
     bool ok = true;
-    for (int t = next_tile(a, -1); t < a.ntiles && ok; t = next_tile(a, t)) {
-      const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TX_N;
+    for (int t = next_tile<TN>(a, -1); t < a.ntiles && ok; t = next_tile<TN>(a, t)) {
+      const int m0 = (t % a.ntm) * TX_M, n0 = (t / a.ntm) * TN;
       if (!tc::mbar_wait_warp(&tfull[tb], tphase, abort_flag, a.spin)) { ok = false; break; }
       tc::tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(tb * TX_N);
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(tb * TN);
       float v[32];
       tc::tmem_ld_32x32b_x32(tbase, v);
-      for (int cc = 0; cc < TX_N / TX_DC; ++cc, ++g) {
+      for (int cc = 0; cc < TN / TX_DC; ++cc, ++g) {
         tc::tmem_ld_wait();
         const int slot = g % TX_D_SLOTS;
         if (g >= TX_D_SLOTS) {
@@ -239,7 +250,7 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
         for (int u = 0; u < 8; ++u)
           *(float4*)(rowp + ((u ^ (trow & 7)) << 4)) =
               make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-        if (cc + 1 < TX_N / TX_DC) {
+        if (cc + 1 < TN / TX_DC) {
           tc::tmem_ld_32x32b_x32(tbase + (uint32_t)((cc + 1) * TX_DC), v);
         } else {  // accumulator fully read: hand it back to the MMA warp
           tc::tc_fence_before();
@@ -276,7 +287,7 @@ tf32x3_update_kernel(const __grid_constant__ CUtensorMap a_hi, const __grid_cons
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0 && a.status != nullptr) atomicCAS(a.status, 0, a.status_code);
   tc::tc_fence_after();
-  if (warp == 1) tc::tmem_dealloc(tmem, TX_TMEM_COLS);
+  if (warp == 1) tc::tmem_dealloc(tmem, TxTile<TN>::TMEM_COLS);
 }
 
 
@@ -294,17 +305,25 @@ bool make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int TN>
 gptq_status launch(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMap& bh,
                    const CUtensorMap& bl, const CUtensorMap& dm, TxArgs& a, cudaStream_t s) {
-  if (smem_optin((const void*)tf32x3_update_kernel, TX_SMEM) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if (smem_optin((const void*)tf32x3_update_kernel<TN>, TxTile<TN>::SMEM) != cudaSuccess)
+    return GPTQ_ERR_CUDA;
   a.spin = wait_limit();
   const int nsm = sm_count();
   const int grid = std::min(a.ntiles, nsm);
   if (grid <= 0) return GPTQ_OK;
-  launch_pdl(tf32x3_update_kernel, dim3(grid), dim3(TX_THREADS), TX_SMEM, s, ah, al, bh, bl, dm,
-             a);
+  launch_pdl(tf32x3_update_kernel<TN>, dim3(grid), dim3(TX_THREADS), TxTile<TN>::SMEM, s, ah, al,
+             bh, bl, dm, a);
   GPTQ_CHECK_LAUNCH();
   return GPTQ_OK;
+}
+
+// The tile width for an update of M x N outputs: 128 when 256-wide tiles
+// would leave SMs idle.
+int pick_tn(int M, int N) {
+  return cdiv(M, TX_M) * cdiv(N, 256) < (int64_t)sm_count() ? 128 : 256;
 }
 
 
@@ -367,9 +386,10 @@ gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int ldE,
                               const float* nut_hi, const float* nut_lo, float* Wt, int r, int k,
                               int s0, int c0, int c1, int32_t* d_status, cudaStream_t s) {
   if (c1 <= c0 || K <= 0) return GPTQ_OK;
+  const int tn = pick_tn(r, c1 - c0);
   CUtensorMap ah, al, bh, bl, dm;
   if (!make_map(&ah, err_hi, K, r, ldE, TX_M) || !make_map(&al, err_lo, K, r, ldE, TX_M) ||
-      !make_map(&bh, nut_hi, k, k, k, TX_N) || !make_map(&bl, nut_lo, k, k, k, TX_N) ||
+      !make_map(&bh, nut_hi, k, k, k, tn) || !make_map(&bl, nut_lo, k, k, k, tn) ||
       !make_map(&dm, Wt, c1, r, k, TX_M))
     return GPTQ_ERR_INVALID_ARG;
   TxArgs a;
@@ -385,12 +405,12 @@ gptq_status tc_sweep_trailing(const float* err_hi, const float* err_lo, int ldE,
   a.b_k0 = s0;
   a.b_r0 = c0;
   a.ntm = (int)cdiv(r, TX_M);
-  a.ntiles = a.ntm * (int)cdiv(c1 - c0, TX_N);
+  a.ntiles = a.ntm * (int)cdiv(c1 - c0, tn);
   a.mode = 0;
   a.split = 0;
   a.status = d_status;
   a.status_code = GPTQ_ERR_TIMEOUT;
-  return launch(ah, al, bh, bl, dm, a, s);
+  return tn == 128 ? launch<128>(ah, al, bh, bl, dm, a, s) : launch<256>(ah, al, bh, bl, dm, a, s);
 }
 
 // Rows [row0, row1) of the k x k work matrix A += R^T S (see the file
@@ -404,9 +424,10 @@ gptq_status tc_rank_update(float* A, int k, int row0, int row1, int split, int K
                            const float* s_hi, const float* s_lo, const float* r_hi,
                            const float* r_lo, int32_t* d_info, cudaStream_t s) {
   if (row1 <= row0 || K <= 0) return GPTQ_OK;
+  const int tn = pick_tn(row1 - row0, k);
   CUtensorMap ah, al, bh, bl, dm;
   if (!make_map(&ah, r_hi, K, row1, ld_s, TX_M) || !make_map(&al, r_lo, K, row1, ld_s, TX_M) ||
-      !make_map(&bh, s_hi, K, k, ld_s, TX_N) || !make_map(&bl, s_lo, K, k, ld_s, TX_N) ||
+      !make_map(&bh, s_hi, K, k, ld_s, tn) || !make_map(&bl, s_lo, K, k, ld_s, tn) ||
       !make_map(&dm, A, k, row1, k, TX_M))
     return GPTQ_ERR_INVALID_ARG;
   TxArgs a;
@@ -422,12 +443,12 @@ gptq_status tc_rank_update(float* A, int k, int row0, int row1, int split, int K
   a.b_k0 = 0;
   a.b_r0 = 0;
   a.ntm = (int)cdiv(row1 - row0, TX_M);
-  a.ntiles = a.ntm * (int)cdiv(k, TX_N);
+  a.ntiles = a.ntm * (int)cdiv(k, tn);
   a.mode = 1;
   a.split = split;
   a.status = d_info;
   a.status_code = k + 1;
-  return launch(ah, al, bh, bl, dm, a, s);
+  return tn == 128 ? launch<128>(ah, al, bh, bl, dm, a, s) : launch<256>(ah, al, bh, bl, dm, a, s);
 }
 
 }  // namespace gptq

@@ -74,6 +74,9 @@ CASES = [
     (256, 1024, 4, 128, 2, torch.float16, False, False),   # decode kernel, a token pair
     (100, 4352, 4, 128, 3, torch.bfloat16, False, False),  # ragged rows, 2 passes over X, odd m
     (64, 8192, 4, 32, 5, torch.float16, False, False),     # smallest 4-bit group, 2 passes
+    (50, 4352, 4, 128, 8, torch.float16, False, False),    # 8 tokens per CTA, 2 passes over X
+    (100, 2048, 2, 64, 12, torch.bfloat16, False, False),  # 2-bit, two 8-token groups
+    (70, 1024, 8, 32, 20, torch.float16, False, False),    # 8-bit past 16 tokens: decode kernel
     (96, 1536, 2, 64, 1, torch.float16, False, False),     # 2-bit decode
     (96, 1536, 8, 16, 2, torch.bfloat16, False, False),    # 8-bit decode, 16-column groups
     (33, 2048, 4, 2048, 1, torch.float16, False, False),   # one group per row
