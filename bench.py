@@ -328,13 +328,26 @@ def timed_replays(graph, steps, dev, stream):
     return t0.elapsed_time(t1) / steps
 
 
-def phase_figures(spec, phase, peaks):
+def measured_rates():
+    """fp32-FMA and kind::tf32 peak rates of this device (gptq_measure_peaks),
+    the denominators of the inverse factor's and the updates' fractions."""
+    from post_weight_quantization_23_b200 import _lib
+    try:
+        r = _lib.measure_peaks()
+    except Exception as e:  # report, do not fail the bench over a calibration
+        return {"error": repr(e)}
+    r["how"] = ("gptq_measure_peaks: packed fp32x2 FMA chains on every SM; kind::tf32 "
+                "128x256x8 MMAs back to back, one issuing thread per SM; one timed launch each")
+    return r
+
+
+def phase_figures(spec, phase, peaks, rates=None):
     """Absolute and roofline figures of one layer's per-phase times (ms)."""
     flops = float(spec.n) * spec.k * (spec.k + 1)  # symmetric triangle, algorithmic
     t_h = phase[0] / 1e3
     sweep_bytes = sweep_model_bytes(spec)
     hess = flops / t_h / 1e12
-    return {
+    out = {
         "hessian_ms": phase[0], "prepare_ms": phase[1], "quantize_ms": phase[2],
         "pack_ms": phase[3], "dequant_ms": phase[4],
         "hessian_tflops": hess,
@@ -347,9 +360,14 @@ def phase_figures(spec, phase, peaks):
         "sweep_model_gbs": sweep_bytes / (phase[2] / 1e3) / 1e9,
         "sweep_frac_hbm": sweep_bytes / (phase[2] / 1e3) / 1e9 / peaks["hbm"],
     }
+    if rates and "tf32_tflops" in rates:
+        # the factor's rank updates issue 3 kind::tf32 MMAs per useful product
+        out["prepare_frac_tf32_issued"] = (3.0 * out["prepare_tflops_algorithmic"]
+                                           / rates["tf32_tflops"])
+    return out
 
 
-def other_configs(dev, stream, peaks, seed, steps, names):
+def other_configs(dev, stream, peaks, seed, steps, names, rates=None):
     """The other layer shapes of the pages (down_proj, the OPT-175B-width
     layer, one decoder layer of the 7B stack), each measured alone with inputs
     drawn on the device (same distributions as the CPU generator; timing
@@ -371,7 +389,7 @@ def other_configs(dev, stream, peaks, seed, steps, names):
         for run in runs:
             ph = run.phase_ms(3)
             entry[run.spec.name] = {"workload": workload_config(run.spec)["workload"],
-                                    **phase_figures(run.spec, ph, peaks)}
+                                    **phase_figures(run.spec, ph, peaks, rates)}
         graph = runs[0].plan.capture(lambda: [r.step() for r in runs])
         ms = timed_replays(graph, steps, dev, stream)
         for run in runs:
@@ -447,7 +465,8 @@ def native_arm(args, spec, world, rank, local):
                "d2h_bytes_per_step": pipe.d2h_bytes()}
 
     peaks = _peaks()
-    phases = phase_figures(spec, phase, peaks)
+    rates = measured_rates()
+    phases = phase_figures(spec, phase, peaks, rates)
     flops = float(spec.n) * spec.k * (spec.k + 1)
     traffic, tsrc = None, None
     if args.traffic is not None:
@@ -471,12 +490,13 @@ def native_arm(args, spec, world, rank, local):
                        launch="one CUDA graph per step (library calls captured once)"),
         "roofline": roofline, "phases": phases,
         "gpu_launches": launches * args.steps if launches is not None else None,
-        "gpu_launches_per_step": launches, "clocks": clk, "e2e": e2e,
+        "gpu_launches_per_step": launches, "clocks": clk, "e2e": e2e, "measured_rates": rates,
     }
     del graph
     if not args.no_other_configs and world == 1:
         names = [n for n in ("down_proj", "opt175_width", "stack_layer") if n != spec.name]
-        line["other_configs"] = other_configs(dev, stream, peaks, seed, args.other_steps, names)
+        line["other_configs"] = other_configs(dev, stream, peaks, seed, args.other_steps, names,
+                                              rates)
     if not args.no_qgemm:
         line["inference_matmul"] = qgemm_measure(dev, stream, peaks, args.seed + rank)
     if not args.no_rotation:
@@ -744,7 +764,7 @@ def main():
                     help="skip the inference-product measurement")
     ap.add_argument("--no-rotation", action="store_true",
                     help="skip the rotation-preprocessing measurement")
-    ap.add_argument("--only", choices=["inference", "rotation"], default=None,
+    ap.add_argument("--only", choices=["inference", "rotation", "peaks"], default=None,
                     help="run one side measurement alone (a short command for profiling)")
     ap.add_argument("--act-order", action="store_true", help="variant: act-order")
     ap.add_argument("--sym", action="store_true", help="variant: symmetric grid")
@@ -774,6 +794,8 @@ def main():
         stream = torch.cuda.current_stream(dev)
         if args.only == "inference":
             out = qgemm_measure(dev, stream, _peaks(), args.seed, reps=args.steps)
+        elif args.only == "peaks":
+            out = measured_rates()
         else:
             X = synth.make_x(spec, args.seed).to(dev)
             out = rotation_measure(X, dev, stream, _peaks(), args.seed)

@@ -337,6 +337,18 @@ GPTQ_API gptq_status gptq_rotate(const void* in, gptq_dtype dt, int64_t rows, in
                         int64_t ld_in, const int8_t* signs, int block, int inverse, void* out,
                         int64_t ld_out, gptq_stream_t stream);
 
+/* Measured peak rates of the current device, for roofline fractions (a
+ * calibration utility, not part of the method): fp32 FMA on the CUDA cores
+ * (packed fp32x2 FMA chains on every SM) and kind::tf32 MMAs on the tensor
+ * cores (M = 128, N = 256, K = 8 back to back, one issuing thread per SM), in
+ * TFLOP/s (2 flops per multiply-add), each from one launch timed with events
+ * after a warm-up launch.  Runs on the legacy default stream and waits for it.
+ * Allocates nothing (two file-scope device words).
+ *   fp32_tflops, tf32_tflops  host pointers, written on GPTQ_OK.
+ * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_CUDA, GPTQ_ERR_TIMEOUT (an
+ * MMA wait gave up). */
+GPTQ_API gptq_status gptq_measure_peaks(double* fp32_tflops, double* tf32_tflops);
+
 #ifdef __cplusplus
 }
 #endif

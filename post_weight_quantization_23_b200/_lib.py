@@ -41,6 +41,7 @@ EXPORTED = (
     "gptq_gemm",
     "gptq_rotate",
     "gptq_set_wait_limit",
+    "gptq_measure_peaks",
 )
 
 WAIT_LIMIT_DEFAULT = 0xFFFFFFFF
@@ -115,6 +116,9 @@ def load(path: str = LIB_PATH):
     lib.gptq_rotate.argtypes = [vp, i32, i64, i64, i64, vp, i32, i32, vp, i64, vp]
     lib.gptq_set_wait_limit.restype = None
     lib.gptq_set_wait_limit.argtypes = [ctypes.c_uint32]
+    lib.gptq_measure_peaks.restype = i32
+    lib.gptq_measure_peaks.argtypes = [ctypes.POINTER(ctypes.c_double),
+                                       ctypes.POINTER(ctypes.c_double)]
     _lib = lib
     return lib
 
@@ -178,6 +182,14 @@ def set_wait_limit(polls: int):
     """Test hook (gptq_set_wait_limit): polls before a pipeline wait of the
     tensor-core kernels gives up; WAIT_LIMIT_DEFAULT restores the default."""
     load().gptq_set_wait_limit(int(polls) & 0xFFFFFFFF)
+
+
+def measure_peaks() -> dict:
+    """Measured fp32-FMA and kind::tf32 peak rates (TFLOP/s) of the current
+    device (gptq_measure_peaks)."""
+    a, b = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    _check(load().gptq_measure_peaks(ctypes.byref(a), ctypes.byref(b)), "gptq_measure_peaks")
+    return {"fp32_tflops": a.value, "tf32_tflops": b.value}
 
 
 def prepare_hinv_noalloc(H, cfg, U, perm, invperm, dead, d_info, stream=None):

@@ -21,7 +21,8 @@
 //
 // Work units are (tile, token chunk) pairs taken token-major, strided over a
 // persistent grid of one CTA per SM, so all CTAs stream through the same
-// token rows of X at the same time and X is read from HBM about once.
+// token rows of X at the same time; tiles are numbered in blocks (see
+// decode_tile) so that the CTAs of one wave share their feature panels.
 //
 // Every mbarrier wait is bounded.  If one gives up, the CTA stops, waits for
 // its own copies and MMAs in flight, frees TMEM and raises a flag in the
@@ -62,16 +63,40 @@ struct HtArgs {
   uint32_t spin;  // polls before a pipeline wait gives up
 };
 
+// Tiles (I, J) reaching the upper triangle: J >= I / 2 (rows of 128, columns
+// of 256).  They are numbered block by block, blocks of HT_BI x HT_BJ tiles in
+// row-major block order, so that the CTAs running at the same time work on one
+// block: together they read HT_BI * 128 + HT_BJ * 256 = 4096 features of each
+// token row, which L2 keeps while the token range is streamed (numbering the
+// tiles row by row made each wave read whole rows, and wide layers read X from
+// DRAM once per wave).
+constexpr int HT_BI = 16, HT_BJ = 8;
+
+__device__ __forceinline__ int tiles_in_row(int I, int J0, int J1, int nJ) {
+  const int lo = max(J0, I / 2), hi = min(J1, nJ);
+  return hi > lo ? hi - lo : 0;
+}
+
 __device__ __forceinline__ void decode_tile(int t, int nI, int nJ, int& I, int& J) {
-  // rows I = 0..nI-1, each with columns J = I/2 .. nJ-1 (tiles reaching j >= i)
-  int i = 0;
-  for (; i < nI; ++i) {
-    int cnt = nJ - i / 2;
-    if (t < cnt) break;
-    t -= cnt;
+  const int nbI = (nI + HT_BI - 1) / HT_BI, nbJ = (nJ + HT_BJ - 1) / HT_BJ;
+  for (int bi = 0; bi < nbI; ++bi) {
+    const int I0 = bi * HT_BI, I1 = min(nI, I0 + HT_BI);
+    for (int bj = 0; bj < nbJ; ++bj) {
+      const int J0 = bj * HT_BJ, J1 = J0 + HT_BJ;
+      if (J1 <= I0 / 2) continue;  // block entirely below the triangle
+      for (int i = I0; i < I1; ++i) {
+        const int cnt = tiles_in_row(i, J0, J1, nJ);
+        if (t < cnt) {
+          I = i;
+          J = max(J0, i / 2) + t;
+          return;
+        }
+        t -= cnt;
+      }
+    }
   }
-  I = i;
-  J = i / 2 + t;
+  I = nI;  // past the last tile (never reached for t < ntiles)
+  J = nJ;
 }
 
 __global__ void __launch_bounds__(HT_THREADS, 1)
