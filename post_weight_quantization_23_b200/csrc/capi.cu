@@ -10,7 +10,8 @@ gptq_status hessian_simt(const void* X, gptq_dtype dt, int64_t n, int64_t k, int
                          float alpha, float* H, cudaStream_t s);
 gptq_status hessian_tc(const void* X, gptq_dtype dt, int64_t n, int64_t k, int64_t ldx,
                        float alpha, float* H, void* ws, cudaStream_t s);
-bool hessian_tc_supported(gptq_dtype dt, int64_t n, int64_t k, int64_t ldx, const void* X);
+bool hessian_tc_supported(gptq_dtype dt, int64_t n, int64_t k, int64_t ldx, const void* X,
+                          const float* H);
 size_t hessian_tc_workspace_bytes(int64_t k, int64_t n);
 size_t hinv_workspace_bytes(int64_t k);
 gptq_status prepare_hinv_impl(const float* H, int64_t k, const gptq_config* cfg, float* U,
@@ -111,7 +112,7 @@ gptq_status gptq_hessian_accumulate(const void* X, gptq_dtype dt, int64_t n, int
   if (X == nullptr || H == nullptr) return GPTQ_ERR_INVALID_ARG;
   if (!aligned(X, dtype_bytes(dt)) || !aligned(H, 4)) return GPTQ_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
-  if (hessian_tc_supported(dt, n, k, ldx, X)) {
+  if (hessian_tc_supported(dt, n, k, ldx, X, H)) {
     size_t need = hessian_tc_workspace_bytes(k, n);
     if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned(ws, 256)))
       return GPTQ_ERR_WORKSPACE;

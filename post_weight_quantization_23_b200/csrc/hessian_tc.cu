@@ -15,7 +15,8 @@
 // Accuracy: the tensor core accumulates at most 256 tokens (16 MMAs) in TMEM;
 // the epilogue then adds that partial into fp32 registers (TMEM is double
 // buffered, so the next 256 tokens accumulate meanwhile) and flushes the
-// register sum into H with fp32 atomics once per unit of up to 65536 tokens.
+// register sum into H once per unit of up to 65536 tokens, by TMA reduce-adds
+// of 32 x 32 chunks staged through one shared-memory slot per epilogue warp.
 // A plain fp32 running sum over all n tokens would miss the 1e-5 relative
 // Frobenius target at n = 262144.
 //
@@ -49,7 +50,10 @@ constexpr int HT_STAGE_BYTES = HT_B_BYTES + HT_A_BYTES; // 48 KB
 constexpr int HT_THREADS = 320;                         // TMA warp, MMA warp, 8 epilogue warps
 constexpr int HT_TMEM_COLS = 512;                       // 2 accumulators x 256 columns
 constexpr int HT_MAX_CHUNK = 65536;
-constexpr size_t HT_SMEM = (size_t)HT_STAGES * HT_STAGE_BYTES + 1024 + 256;
+constexpr int HT_SLOT_BYTES = 32 * 32 * 4;              // one warp's 32 x 32 flush chunk
+constexpr int HT_EPI_WARPS = 8;
+constexpr size_t HT_SMEM = (size_t)HT_STAGES * HT_STAGE_BYTES +
+                           (size_t)HT_EPI_WARPS * HT_SLOT_BYTES + 1024 + 256;
 
 struct HtArgs {
   int k;
@@ -100,11 +104,13 @@ __device__ __forceinline__ void decode_tile(int t, int nI, int nJ, int& I, int& 
 }
 
 __global__ void __launch_bounds__(HT_THREADS, 1)
-hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HtArgs a, int fmt_bf16) {
+hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap hmap,
+                  HtArgs a, int fmt_bf16) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* stages = smem;
-  uint64_t* bars = (uint64_t*)(smem + HT_STAGES * HT_STAGE_BYTES);
+  uint8_t* slots = smem + HT_STAGES * HT_STAGE_BYTES;  // [8] flush chunks, 1024-byte aligned
+  uint64_t* bars = (uint64_t*)(slots + HT_EPI_WARPS * HT_SLOT_BYTES);
   uint64_t* full = bars;                      // [HT_STAGES]
   uint64_t* empty = bars + HT_STAGES;         // [HT_STAGES]
   uint64_t* tfull = bars + 2 * HT_STAGES;     // [2]
@@ -127,6 +133,7 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HtArgs a, int fmt_bf
     *abort_flag = 0;
     tc::fence_barrier_init();
     tc::prefetch_tensormap(&xmap);
+    tc::prefetch_tensormap(&hmap);
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, HT_TMEM_COLS);
   tc::tc_fence_before();
@@ -272,17 +279,30 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HtArgs a, int fmt_bf
         if (++tb == 2) tb = 0, tphase ^= 1u;
       }
       if (!ok) break;
-      const int gi = i0 + row;
-      if (gi < a.k) {
-        float* hrow = a.H + (int64_t)gi * a.k;
-        const int jb = j0 + half * 128;
+      // flush: alpha * the unit's sums into H, 32 x 32 chunks reduce-added by
+      // TMA (L2 adds them; rows and columns past k are clipped).  Entries
+      // below the diagonal are added as well: the mirror pass overwrites them.
+      uint8_t* slot = slots + ew * HT_SLOT_BYTES;
+      const int jb = j0 + half * 128;
 #pragma unroll
-        for (int q = 0; q < 128; ++q) {
-          const int gj = jb + q;
-          if (gj >= gi && gj < a.k) atomicAdd(hrow + gj, a.alpha * acc[q]);
+      for (int c = 0; c < 4; ++c) {
+        if (lane == 0) tc::bulk_wait_read_all();  // the slot's previous reduce has read it
+        __syncwarp();
+        uint8_t* rowp = slot + lane * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *(float4*)(rowp + ((u ^ (lane & 7)) << 4)) =
+              make_float4(a.alpha * acc[c * 32 + 4 * u], a.alpha * acc[c * 32 + 4 * u + 1],
+                          a.alpha * acc[c * 32 + 4 * u + 2], a.alpha * acc[c * 32 + 4 * u + 3]);
+        tc::fence_proxy_async_smem();  // the reduce reads what this thread wrote
+        __syncwarp();
+        if (lane == 0) {
+          tc::tma_reduce_add_2d(&hmap, slot, jb + c * 32, i0 + quarter * 32);
+          tc::bulk_commit_group();
         }
       }
     }
+    if (lane == 0) tc::bulk_wait_all();  // every reduce of this warp has completed
   }
 
   __syncthreads();
@@ -293,9 +313,11 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HtArgs a, int fmt_bf
 
 }  // namespace
 
-bool hessian_tc_supported(gptq_dtype dt, int64_t n, int64_t k, int64_t ldx, const void* X) {
+bool hessian_tc_supported(gptq_dtype dt, int64_t n, int64_t k, int64_t ldx, const void* X,
+                          const float* H) {
   if (dt != GPTQ_F16 && dt != GPTQ_BF16) return false;
   if (k < 64 || k % 8 != 0 || ldx % 8 != 0 || ((uintptr_t)X % 16) != 0) return false;
+  if (((uintptr_t)H % 16) != 0) return false;  // H is reduce-added by TMA
   if (n <= 0 || n > ((int64_t)1 << 31) - HT_MAX_CHUNK) return false;
   return tensormap_encoder() != nullptr;
 }
@@ -317,6 +339,16 @@ gptq_status hessian_tc(const void* X, gptq_dtype dt, int64_t n, int64_t k, int64
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return GPTQ_ERR_INVALID_ARG;
+  CUtensorMap hmap;
+  {
+    cuuint64_t hdim[2] = {(cuuint64_t)k, (cuuint64_t)k};
+    cuuint64_t hstride[1] = {(cuuint64_t)k * 4};
+    cuuint32_t hbox[2] = {32, 32};
+    if (enc(&hmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, H, hdim, hstride, hbox, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GPTQ_ERR_INVALID_ARG;
+  }
 
   const int nsm = sm_count();
   if (smem_optin((const void*)hessian_tc_kernel, HT_SMEM) != cudaSuccess) return GPTQ_ERR_CUDA;
@@ -340,7 +372,7 @@ gptq_status hessian_tc(const void* X, gptq_dtype dt, int64_t n, int64_t k, int64
   // word 0: this call's give-up flag; word 1 (the caller's status) is only ever set
   if (cudaMemsetAsync(ws, 0, sizeof(int32_t), s) != cudaSuccess) return GPTQ_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(a.nunits, nsm);
-  hessian_tc_kernel<<<grid, HT_THREADS, HT_SMEM, s>>>(map, a, dt == GPTQ_BF16 ? 1 : 0);
+  hessian_tc_kernel<<<grid, HT_THREADS, HT_SMEM, s>>>(map, hmap, a, dt == GPTQ_BF16 ? 1 : 0);
   GPTQ_CHECK_LAUNCH();
   int nb = (int)cdiv(k, 32);
   mirror_upper_kernel<<<dim3(nb, nb), dim3(32, 8), 0, s>>>(H, (int)k, (int32_t*)ws);
