@@ -278,9 +278,6 @@ __device__ __forceinline__ void inv16_cols(const float (*S)[K1_LD], float (*T)[K
 
 __global__ void __launch_bounds__(256)
 chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b, int32_t* __restrict__ d_info) {
-  pdl_wait();
-  pdl_trigger();
-  if (*d_info != 0) return;
   __shared__ float S[HV_B][K1_LD];                  // B, then M (lower part)
   __shared__ float T[HV_B][K1_LD];                  // N = M^-1 (lower part)
   __shared__ float Mt[HV_B - K1_BS][K1_BS + 1];     // M_ik of the current block column
@@ -288,15 +285,18 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b, int32_t* __res
   __shared__ float rdg[HV_B];                        // 1 / M_ii
   __shared__ int fail;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // the padding and the zeros go in while the previous kernel finishes
   for (int e = t; e < HV_B * HV_B; e += 256) {
     const int i = e / HV_B, j = e % HV_B;
     S[i][j] = (i == j && i >= b) ? 1.f : 0.f;
     T[i][j] = 0.f;
   }
   if (t == 0) fail = -1;
-  __syncthreads();
-  // B[b-1-ca][b-1-ra] = A[ra][ca] for ca <= ra < b (coalesced along ca; all
-  // loads issued before the stores)
+  pdl_wait();
+  pdl_trigger();
+  if (*d_info != 0) return;  // the same word for every thread: the whole CTA leaves
+  // B[b-1-ca][b-1-ra] = A[ra][ca] for ca <= ra < b (coalesced along ca; the
+  // loads are in flight across the barrier that orders them after the zeros)
   {
     float v[HV_B * HV_B / 256];
 #pragma unroll
@@ -304,6 +304,7 @@ chol_inv_diag_kernel(float* __restrict__ A, int k, int j0, int b, int32_t* __res
       const int e = t + 256 * q, ra = e / HV_B, ca = e % HV_B;
       v[q] = (ra < b && ca <= ra) ? A[(int64_t)(j0 + ra) * k + j0 + ca] : 0.f;
     }
+    __syncthreads();
 #pragma unroll
     for (int q = 0; q < HV_B * HV_B / 256; ++q) {
       const int e = t + 256 * q, ra = e / HV_B, ca = e % HV_B;
