@@ -52,9 +52,17 @@ UNIT = "Mweights/s"
 # smaller token count, scaled by tokens to a full launch: an estimate).  Only
 # the widths a capture exists for; the line reports null elsewhere.
 HESS_TRAFFIC = {
-    4096: ((645.9e6 + 65.9e6) / 32768,
+    # per token: ncu dram__bytes_read.sum + dram__bytes_write.sum of one hessian_tc_kernel
+    # launch on 32768 tokens of the config's width, divided by 32768
+    4096: ((602.87e6 + 72.25e6) / 32768,
            "estimate: ncu dram bytes of hessian_tc_kernel on a 32768 x 4096 capture, scaled by "
-           "tokens (profiles/hessian_tc_kernel_q_proj_32k_tokens.md)"),
+           "tokens (profiles/hessian_tc_kernel_dram_by_width.md)"),
+    11008: ((6971.02e6 + 249.56e6) / 32768,
+            "estimate: ncu dram bytes of hessian_tc_kernel on a 32768 x 11008 capture, scaled by "
+            "tokens (profiles/hessian_tc_kernel_dram_by_width.md)"),
+    12288: ((8592.74e6 + 311.70e6) / 32768,
+            "estimate: ncu dram bytes of hessian_tc_kernel on a 32768 x 12288 capture, scaled by "
+            "tokens (profiles/hessian_tc_kernel_dram_by_width.md)"),
 }
 
 
@@ -360,6 +368,11 @@ def phase_figures(spec, phase, peaks, rates=None):
         "sweep_model_gbs": sweep_bytes / (phase[2] / 1e3) / 1e9,
         "sweep_frac_hbm": sweep_bytes / (phase[2] / 1e3) / 1e9 / peaks["hbm"],
     }
+    if spec.k in HESS_TRAFFIC:
+        per_tok, src = HESS_TRAFFIC[spec.k]
+        out["hessian_traffic_bytes"] = per_tok * spec.n
+        out["hessian_traffic_source"] = src
+        out["hessian_traffic_over_x"] = per_tok * spec.n / (spec.n * spec.k * 2.0)
     if rates and "tf32_tflops" in rates:
         # the factor's rank updates issue 3 kind::tf32 MMAs per useful product
         out["prepare_frac_tf32_issued"] = (3.0 * out["prepare_tflops_algorithmic"]

@@ -152,17 +152,17 @@ __device__ __forceinline__ void qv_compute(const QvSlab<BITS>& S, const float* x
 // the column slabs.  The CTAs of one row block are consecutive (the block index
 // runs over the token groups first), so a second token group finds the row
 // block's packed words in L2.  Launched with programmatic dependent launch:
-// the first slab of packed words is requested before waiting for the previous
-// kernel (only X depends on it; the weights must not be written by a kernel
-// that lets this one start early).
+// the first slabs of packed words are requested before waiting for the
+// previous kernel (only X depends on it; the weights must not be written by a
+// kernel that lets this one start early).
 // Lane (q = lane / 8, p = lane % 8) loads, for i = 0..3, the 16-byte piece p
 // of row 4 i + q in its warp's slab, so each load instruction reads four whole
-// 128-byte row segments.  The first slab's words are requested before the
-// activations are staged, and each next slab's before the current one is
-// computed.  Needs k % CH == 0 and a group size that is a multiple of CH (or
+// 128-byte row segments.  The first AHEAD slabs' words (two for M = 1, one
+// otherwise) are requested before the activations are staged, and each later
+// slab's AHEAD slabs before it is computed.  Needs k % CH == 0 and a group size that is a multiple of CH (or
 // one group per row), so a piece lies in one group.
 template <int BITS, int M, typename T>
-__global__ void __launch_bounds__(QV_WARPS * 32)
+__global__ void __launch_bounds__(QV_WARPS * 32, M <= 2 ? 2 : 1)  // decode: 2 CTAs per SM
 qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
              const int32_t* __restrict__ qw, const float* __restrict__ scales,
              const int32_t* __restrict__ zeros, int n, int G, int ngroups, int KC,
@@ -178,6 +178,11 @@ qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
   const int r0 = (int)(blockIdx.x / ntg) * QV_ROWS;
   const int t0 = (int)(blockIdx.x % ntg) * M;
   const int64_t wpr = (int64_t)k / Sh::CPW;  // words per row
+  constexpr int STEP = QV_WARPS * Sh::SLAB;  // columns per round of the 8 warps
+  // slabs in flight beyond the one being computed: two for one token (whose
+  // few slabs per warp are then all requested early; measured 290 -> 273 us
+  // for the 28-layer decode pass, while two tokens ran 316 -> 325 us)
+  constexpr int AHEAD = M == 1 ? 2 : 1;
 
   float y[QV_RPL][M];
 #pragma unroll
@@ -187,12 +192,16 @@ qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
 
   for (int kc0 = 0; kc0 < k; kc0 += KC) {
     const int kcw = min(KC, k - kc0);
-    // this warp's first slab of the chunk, requested before the staging
+    // this warp's first AHEAD slabs of the chunk, requested before the staging
     int sl = warp * Sh::SLAB;
-    QvSlab<BITS> cur;
+    QvSlab<BITS> cur, nxt;
     {
       const int cl = sl + p * Sh::CH;
       qv_load<BITS>(cur, qw, scales, zeros, wpr, r0, q, n, kc0 + cl, cl < kcw, G, ngroups);
+      if (AHEAD == 2) {
+        const int cn = sl + STEP + p * Sh::CH;
+        qv_load<BITS>(nxt, qw, scales, zeros, wpr, r0, q, n, kc0 + cn, cn < kcw, G, ngroups);
+      }
     }
     if (kc0 == 0) {
       // X comes from the previous kernel
@@ -224,20 +233,25 @@ qgemv_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
       }
     }
     __syncthreads();
-    for (; sl < kcw; sl += QV_WARPS * Sh::SLAB) {
+    for (; sl < kcw; sl += STEP) {
       const int cl = sl + p * Sh::CH;  // this lane's piece, local column
       const bool have = cl < kcw;
-      QvSlab<BITS> nxt;
-      const int sn = sl + QV_WARPS * Sh::SLAB;
-      if (sn < kcw) {
-        const int cn = sn + p * Sh::CH;
-        qv_load<BITS>(nxt, qw, scales, zeros, wpr, r0, q, n, kc0 + cn, cn < kcw, G, ngroups);
+      QvSlab<BITS> nn;
+      const int sa = sl + AHEAD * STEP;  // the slab requested now
+      if (sa < kcw) {
+        const int ca = sa + p * Sh::CH;
+        qv_load<BITS>(nn, qw, scales, zeros, wpr, r0, q, n, kc0 + ca, ca < kcw, G, ngroups);
       }
       // lanes past the chunk's end have zero words and scale 0; they read
       // (and discard) the chunk's first columns instead of past the buffer
       const int clx = have ? cl : 0;
       qv_compute<BITS, M>(cur, xs + clx + Sh::PAD * (clx / Sh::CH), XS, y);
-      if (sn < kcw) cur = nxt;
+      if (AHEAD == 2) {
+        cur = nxt;
+        if (sa < kcw) nxt = nn;
+      } else if (sa < kcw) {
+        cur = nn;
+      }
     }
   }
   // sum the 8 pieces of each row, then the warps
