@@ -280,7 +280,7 @@ def _cfg_of(spec):
 class LayerRun:
     """One layer's plan and its device-resident inputs; ``step`` issues the
     whole hot path (H reset, Hessian over all tokens, factor, sweep with the
-    loss, pack, dequant), optionally with events between the phases."""
+    loss, pack, dequant)."""
 
     PHASES = ("hessian", "prepare", "quantize", "pack", "dequant")
 
@@ -289,7 +289,6 @@ class LayerRun:
         self.spec, self.Xd, self.Wd, self.dev = spec, Xd, Wd, dev
         self.plan = GptqPlan(spec.r, spec.k, _cfg_of(spec), dev, want_loss=True,
                              deq_dtype=torch.float16, hessian_tokens_hint=spec.n)
-        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
 
     def lib_calls(self):
         p = self.plan
@@ -299,28 +298,37 @@ class LayerRun:
         p.pack()
         p.dequant()
 
-    def step(self, record=False, stream=None):
-        p, ev = self.plan, self.ev
-        stream = stream or torch.cuda.current_stream(self.dev)
-        if record:
-            ev[0].record(stream)
+    def step(self):
+        p = self.plan
         p.hessian_reset()
         p.hessian_add(self.Xd, self.spec.n)
-        for i, fn in enumerate((p.prepare, lambda: p.quantize(self.Wd), p.pack, p.dequant)):
-            if record:
-                ev[i + 1].record(stream)
-            fn()
-        if record:
-            ev[5].record(stream)
+        p.prepare()
+        p.quantize(self.Wd)
+        p.pack()
+        p.dequant()
 
     def phase_ms(self, reps):
-        """Per-phase device times (CUDA events between phases), mean of reps."""
-        acc = np.zeros(5)
-        for _ in range(reps):
-            self.step(record=True)
-            torch.cuda.synchronize(self.dev)
-            acc += [self.ev[i].elapsed_time(self.ev[i + 1]) for i in range(5)]
-        return acc / reps
+        """Per-phase device times: each phase's library calls captured into a
+        CUDA graph of its own and replayed reps times back to back (events
+        around the replays), in pipeline order so that every phase reads what
+        the previous one wrote.  Host launch cost is out of the figures, as in
+        the graph-replayed step (the eager form is host-bound for the factor's
+        ~3 launches per 64 columns at the wide layers)."""
+        p = self.plan
+        stream = torch.cuda.current_stream(self.dev)
+
+        def hess():
+            p.hessian_reset()
+            p.hessian_add(self.Xd, self.spec.n)
+
+        fns = (hess, p.prepare, lambda: p.quantize(self.Wd), p.pack, p.dequant)
+        out = []
+        for fn in fns:
+            g = p.capture(fn)
+            g.replay()
+            out.append(timed_replays(g, reps, self.dev, stream))
+            del g
+        return np.array(out)
 
 
 def timed_replays(graph, steps, dev, stream):
