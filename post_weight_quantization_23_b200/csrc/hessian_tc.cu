@@ -243,7 +243,6 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constan
     const int ew = warp - 2;
     const int quarter = warp & 3;        // TMEM lane quarter this warp may access
     const int half = ew >> 2;            // column half of the 256-wide tile
-    const int row = quarter * 32 + lane; // tile row = TMEM lane
     int tb = 0;
     uint32_t tphase = 0;
     bool ok = true;
