@@ -308,28 +308,32 @@ class LayerRun:
         p.dequant()
 
     def phase_ms(self, reps):
-        """Per-phase device times: each phase's library calls captured into a
-        CUDA graph of its own and replayed reps times back to back (events
-        around the replays), in pipeline order so that every phase reads what
-        the previous one wrote.  Host launch cost is out of the figures, as in
-        the graph-replayed step (the eager form is host-bound for the factor's
-        ~3 launches per 64 columns at the wide layers)."""
+        """Per-phase device times inside the step: the whole step captured as
+        one CUDA graph with timing events between the phases (external event
+        nodes), replayed reps times; mean of the replays.  Host launch cost
+        stays out (the eager form is host-bound for the factor's ~3 launches
+        per 64 columns at the wide layers), and every phase runs in the step's
+        own order and clocks."""
         p = self.plan
-        stream = torch.cuda.current_stream(self.dev)
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
 
-        def hess():
+        def body():
+            ev[0].record()
             p.hessian_reset()
             p.hessian_add(self.Xd, self.spec.n)
+            for i, fn in enumerate((p.prepare, lambda: p.quantize(self.Wd), p.pack, p.dequant)):
+                ev[i + 1].record()
+                fn()
+            ev[5].record()
 
-        fns = (hess, p.prepare, lambda: p.quantize(self.Wd), p.pack, p.dequant)
-        out = []
-        for fn in fns:
-            g = p.capture(fn)
+        g = p.capture(body)
+        acc = np.zeros(5)
+        for _ in range(reps):
             g.replay()
-            out.append(timed_replays(g, reps, self.dev, stream))
-            del g
-        return np.array(out)
-
+            torch.cuda.synchronize(self.dev)
+            acc += [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
+        del g
+        return acc / reps
 
 def timed_replays(graph, steps, dev, stream):
     """Device ms per replay of ``graph`` over ``steps`` back-to-back replays."""
