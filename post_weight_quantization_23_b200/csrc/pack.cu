@@ -45,12 +45,46 @@ template <> __device__ __forceinline__ __nv_bfloat16 cvt_out<__nv_bfloat16>(floa
   return __float2bfloat16_rn(v);
 }
 
+// Store 32 consecutive outputs of one run: with `vec` as 16-byte vectors (the
+// run's outputs are contiguous and, for an aligned `out` and k % 32 == 0,
+// 16-byte aligned), else one by one.
+template <typename OutT>
+__device__ __forceinline__ void store_run(OutT* dst, const float (&v)[32], bool vec) {
+  if (vec) {
+    if constexpr (sizeof(OutT) == 4) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<float4*>(dst)[q] =
+            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const OutT lo = cvt_out<OutT>(v[8 * q + 2 * h]), hi = cvt_out<OutT>(v[8 * q + 2 * h + 1]);
+          w[h] = (uint32_t)(*reinterpret_cast<const uint16_t*>(&lo)) |
+                 ((uint32_t)(*reinterpret_cast<const uint16_t*>(&hi)) << 16);
+        }
+        reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) dst[j] = cvt_out<OutT>(v[j]);
+  }
+}
+
+// One thread per run of 32 codes (`bits` words): the run's g_idx entries come
+// in as 16-byte vectors, each code becomes scale[g] * (code - zero[g]) in fp32
+// and the 32 outputs leave as 16-byte vectors (vec: out and g_idx 16-byte
+// aligned).
 template <int BITS, typename OutT>
 __global__ void dequant_kernel(const int32_t* __restrict__ qweight,
                                const float* __restrict__ scales,
                                const int32_t* __restrict__ zeros,
                                const int32_t* __restrict__ g_idx, int64_t r, int64_t k,
-                               int64_t ngroups, OutT* __restrict__ out) {
+                               int64_t ngroups, int vec, OutT* __restrict__ out) {
   const int64_t runs_per_row = k / 32;
   const int64_t nruns = r * runs_per_row;
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < nruns;
@@ -60,19 +94,31 @@ __global__ void dequant_kernel(const int32_t* __restrict__ qweight,
     uint32_t in[BITS];
 #pragma unroll
     for (int w = 0; w < BITS; ++w) in[w] = (uint32_t)src[w];
+    int gi[32];
+    if (vec) {
+      const int4* gsrc = reinterpret_cast<const int4*>(g_idx + run * 32);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int4 g4 = gsrc[q];
+        gi[4 * q] = g4.x, gi[4 * q + 1] = g4.y, gi[4 * q + 2] = g4.z, gi[4 * q + 3] = g4.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) gi[j] = g_idx[run * 32 + j];
+    }
     const float* srow = scales + row * ngroups;
     const int32_t* zrow = zeros + row * ngroups;
-    OutT* orow = out + row * k + run * 32;
+    float v[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int bit = j * BITS;
       uint32_t c = in[bit / 32] >> (bit % 32);
       if ((bit % 32) + BITS > 32) c |= in[bit / 32 + 1] << (32 - bit % 32);
       c &= (1u << BITS) - 1u;
-      const int g = g_idx[run * 32 + j];
-      const float v = srow[g] * (float)((int32_t)c - zrow[g]);
-      orow[j] = cvt_out<OutT>(v);
+      const int g = gi[j];
+      v[j] = srow[g] * (float)((int32_t)c - zrow[g]);
     }
+    store_run<OutT>(out + row * k + run * 32, v, vec != 0);
   }
 }
 
@@ -105,11 +151,12 @@ static gptq_status dequant_typed(const int32_t* qweight, const float* scales, co
   const int64_t work = r * (k / 32);
   if (work == 0) return GPTQ_OK;
   const unsigned g = grid_for(work);
+  const int vec = ((uintptr_t)out % 16 == 0 && (uintptr_t)g_idx % 16 == 0) ? 1 : 0;
   switch (bits) {
-    case 2: dequant_kernel<2, OutT><<<g, 256, 0, s>>>(qweight, scales, zeros, g_idx, r, k, ngroups, out); break;
-    case 3: dequant_kernel<3, OutT><<<g, 256, 0, s>>>(qweight, scales, zeros, g_idx, r, k, ngroups, out); break;
-    case 4: dequant_kernel<4, OutT><<<g, 256, 0, s>>>(qweight, scales, zeros, g_idx, r, k, ngroups, out); break;
-    case 8: dequant_kernel<8, OutT><<<g, 256, 0, s>>>(qweight, scales, zeros, g_idx, r, k, ngroups, out); break;
+    case 2: dequant_kernel<2, OutT><<<g, 256, 0, s>>>(qweight, scales, zeros, g_idx, r, k, ngroups, vec, out); break;
+    case 3: dequant_kernel<3, OutT><<<g, 256, 0, s>>>(qweight, scales, zeros, g_idx, r, k, ngroups, vec, out); break;
+    case 4: dequant_kernel<4, OutT><<<g, 256, 0, s>>>(qweight, scales, zeros, g_idx, r, k, ngroups, vec, out); break;
+    case 8: dequant_kernel<8, OutT><<<g, 256, 0, s>>>(qweight, scales, zeros, g_idx, r, k, ngroups, vec, out); break;
     default: return GPTQ_ERR_UNSUPPORTED;
   }
   GPTQ_CHECK_LAUNCH();

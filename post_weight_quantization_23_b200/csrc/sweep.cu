@@ -129,20 +129,39 @@ __device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
   lo = x - hi;
 }
 
+// vec: four positions per thread (perm read and Wt written as 16-byte vectors;
+// k % 4 == 0 and perm 16-byte aligned).
 template <typename T>
 __global__ void sweep_init_kernel(const T* __restrict__ W, int64_t ldw, int r, int k,
                                   const int32_t* __restrict__ perm,
                                   const uint8_t* __restrict__ dead, int G, int static_groups,
-                                  float* __restrict__ Wt, int32_t* __restrict__ g_idx,
+                                  int vec, float* __restrict__ Wt, int32_t* __restrict__ g_idx,
                                   double* __restrict__ loss, int32_t* __restrict__ d_status) {
   int row = blockIdx.y;
-  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < k; j += gridDim.x * blockDim.x) {
-    int c = perm[j];
-    float v = dead[c] ? 0.f : to_f32(W[(int64_t)row * ldw + c]);
-    Wt[(int64_t)row * k + j] = v;
-    // dynamic groups are runs of processing positions; static ones keep the
-    // original columns together
-    if (row == 0) g_idx[c] = (static_groups ? c : j) / G;
+  const T* wrow = W + (int64_t)row * ldw;
+  if (vec) {
+    for (int j4 = 4 * (blockIdx.x * blockDim.x + threadIdx.x); j4 < k;
+         j4 += 4 * gridDim.x * blockDim.x) {
+      const int4 c4 = *reinterpret_cast<const int4*>(perm + j4);
+      const int cc[4] = {c4.x, c4.y, c4.z, c4.w};
+      float v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[q] = dead[cc[q]] ? 0.f : to_f32(wrow[cc[q]]);
+      *reinterpret_cast<float4*>(Wt + (int64_t)row * k + j4) = make_float4(v[0], v[1], v[2], v[3]);
+      if (row == 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) g_idx[cc[q]] = (static_groups ? cc[q] : j4 + q) / G;
+      }
+    }
+  } else {
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < k; j += gridDim.x * blockDim.x) {
+      int c = perm[j];
+      float v = dead[c] ? 0.f : to_f32(wrow[c]);
+      Wt[(int64_t)row * k + j] = v;
+      // dynamic groups are runs of processing positions; static ones keep the
+      // original columns together
+      if (row == 0) g_idx[c] = (static_groups ? c : j) / G;
+    }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     if (loss != nullptr) {
@@ -683,11 +702,30 @@ __global__ void __launch_bounds__(SQ_MAX_WARPS * 32, 1) sweep_block_lane_kernel(
   if (st.nonfinite && a.d_status != nullptr) atomicCAS(a.d_status, 0, (int32_t)GPTQ_ERR_NONFINITE);
 }
 
+// Four consecutive weights as fp32 (8- or 16-byte aligned load).
+__device__ __forceinline__ void load4_f32(const float* p, float (&o)[4]) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  o[0] = v.x, o[1] = v.y, o[2] = v.z, o[3] = v.w;
+}
+__device__ __forceinline__ void load4_f32(const __half* p, float (&o)[4]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+  o[0] = a.x, o[1] = a.y, o[2] = b.x, o[3] = b.y;
+}
+__device__ __forceinline__ void load4_f32(const __nv_bfloat16* p, float (&o)[4]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+  o[0] = a.x, o[1] = a.y, o[2] = b.x, o[3] = b.y;
+}
+
 // Layer loss, second part: loss[row] -= lambda * sum_c (w0_c - q_c)^2 over the
 // original columns, q = scale * (code - zero) of the column's group (dead
-// columns count with w0 = 0).  One warp per row.
+// columns count with w0 = 0).  One warp per row; with vec (k % 4 == 0, the
+// row starts aligned) each lane takes four adjacent columns per load.
 template <typename T>
-__global__ void loss_finish_kernel(const T* __restrict__ W0, int64_t ldw, int r, int k,
+__global__ void loss_finish_kernel(const T* __restrict__ W0, int64_t ldw, int r, int k, int vec,
                                    const uint8_t* __restrict__ dead,
                                    const uint8_t* __restrict__ codes,
                                    const float* __restrict__ scales,
@@ -702,13 +740,33 @@ __global__ void loss_finish_kernel(const T* __restrict__ W0, int64_t ldw, int r,
   const T* wrow = W0 + (int64_t)row * ldw;
   const float* srow = scales + (int64_t)row * ngroups;
   const int32_t* zrow = zeros + (int64_t)row * ngroups;
+  if (vec) {
+#pragma unroll 2
+    for (int c = 4 * lane; c < k; c += 4 * kWarp) {
+      const int4 g4 = *reinterpret_cast<const int4*>(g_idx + c);
+      const uchar4 q4 = *reinterpret_cast<const uchar4*>(crow + c);
+      const uchar4 d4 = *reinterpret_cast<const uchar4*>(dead + c);
+      float w4[4];
+      load4_f32(wrow + c, w4);
+      const int gg[4] = {g4.x, g4.y, g4.z, g4.w};
+      const uint8_t qq[4] = {q4.x, q4.y, q4.z, q4.w}, de[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float q = srow[gg[i]] * ((float)qq[i] - (float)zrow[gg[i]]);
+        const float w0 = de[i] ? 0.f : w4[i];
+        const double dd = (double)w0 - (double)q;
+        acc += dd * dd;
+      }
+    }
+  } else {
 #pragma unroll 4
-  for (int c = lane; c < k; c += kWarp) {
-    const int g = g_idx[c];
-    const float q = srow[g] * ((float)crow[c] - (float)zrow[g]);
-    const float w0 = dead[c] ? 0.f : to_f32(wrow[c]);
-    const double dd = (double)w0 - (double)q;
-    acc += dd * dd;
+    for (int c = lane; c < k; c += kWarp) {
+      const int g = g_idx[c];
+      const float q = srow[g] * ((float)crow[c] - (float)zrow[g]);
+      const float w0 = dead[c] ? 0.f : to_f32(wrow[c]);
+      const double dd = (double)w0 - (double)q;
+      acc += dd * dd;
+    }
   }
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) loss[row] -= (double)(*lambda) * acc;
@@ -774,8 +832,9 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
   double* lossp = want_loss ? loss : nullptr;
   {
     dim3 grid((unsigned)cdiv(k, 1024), (unsigned)r);
+    const int ivec = (k % 4 == 0 && (uintptr_t)perm % 16 == 0) ? 1 : 0;
     sweep_init_kernel<T><<<grid, 256, 0, s>>>(W, ldw, r, k, perm, dead, G, cfg->static_groups,
-                                              sc.Wt, g_idx, lossp, d_status);
+                                              ivec, sc.Wt, g_idx, lossp, d_status);
     GPTQ_CHECK_LAUNCH();
   }
   if (stat) {
@@ -898,8 +957,13 @@ static gptq_status quantize_typed(const T* W, int64_t ldw, int r, int k, const f
     }
   }
   if (want_loss) {
+    const int lvec = (k % 4 == 0 && ldw % 4 == 0 && (uintptr_t)W % (4 * sizeof(T)) == 0 &&
+                      (uintptr_t)codes % 4 == 0 && (uintptr_t)g_idx % 16 == 0 &&
+                      (uintptr_t)dead % 4 == 0)
+                         ? 1
+                         : 0;
     loss_finish_kernel<T><<<(unsigned)cdiv((int64_t)r * kWarp, 256), 256, 0, s>>>(
-        W, ldw, r, k, dead, codes, scales, zeros, g_idx, ngroups, sc.lambda, loss);
+        W, ldw, r, k, lvec, dead, codes, scales, zeros, g_idx, ngroups, sc.lambda, loss);
     GPTQ_CHECK_LAUNCH();
     loss_total_kernel<<<1, 1024, 0, s>>>(loss, r);
     GPTQ_CHECK_LAUNCH();
