@@ -627,7 +627,9 @@ def qgemm_measure(dev, stream, peaks, seed, bits=4, G=128, reps=20):
                         f"blocks ({len(layers)} layers: 4x 4096x4096, 2x 11008x4096, "
                         f"1x 4096x11008 per block), int{bits} g{G}, f16 activations"),
            "l2": "weights larger than L2, each layer read once per pass", "bound": "hbm",
-           "peak": peaks["hbm"], "unit": "GB/s", "kernel": "qgemv_kernel (gptq_gemm)"}
+           "peak": peaks["hbm"], "unit": "GB/s", "kernel": "qgemv_kernel (gptq_gemm)",
+           "m16_kernel": "qgemm_mma_kernel (mma.sync m16n8k16, weights formed in f16)",
+           "m2048_kernel": "qgemm_tc_kernel (tcgen05)"}
     for m in (1, 16, 2048):
         xs = [torch.randn(m, k, generator=g, device=dev).half() for (_, k, *_r) in layers]
         ys = [torch.empty(m, n, dtype=torch.float16, device=dev) for (n, *_r) in layers]

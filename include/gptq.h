@@ -306,8 +306,12 @@ GPTQ_API gptq_status gptq_dequant(const int32_t* qweight, const float* scales, c
  *     group per row), X and qweight 16-byte aligned, ldx % 8 == 0: the
  *     tensor-core kernel (each weight formed in dt: the scale rounded to dt
  *     times the exact code - zero, rounded once more; fp32 accumulation);
+ *   5 <= m <= 16, 4-bit, g_idx NULL, group_size a multiple of 128 (or one
+ *     group per row), qweight 16-byte aligned: the small-batch kernel
+ *     (mma.sync, weights streamed once for all tokens and formed in dt as in
+ *     the tensor-core kernel; fp32 accumulation);
  *   else g_idx NULL, bits 2/4/8 and group_size a multiple of 128/bits (or one
- *     group per row): the decode kernel (weights streamed once per 2 tokens,
+ *     group per row): the decode kernel (weights streamed once per 8 tokens,
  *     each product x (code - zero) exact in fp32);
  *   every other case: the general kernel (fp32 weights per element).
  * Returns GPTQ_OK, GPTQ_ERR_INVALID_ARG, GPTQ_ERR_UNSUPPORTED (bits, f32 X),

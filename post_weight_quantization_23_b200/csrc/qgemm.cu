@@ -28,6 +28,10 @@ gptq_status qgemm_tc(const void* X, bool bf16, int64_t m, int64_t k, int64_t ldx
 
 // Token counts above this use the tensor-core kernel when it applies.
 constexpr int QG_TC_MIN_TOKENS = 17;
+// From this token count up to 16 the small-batch mma.sync kernel, when it applies
+// (measured on 28 7B-shaped layers per pass: 3 tokens 611 us against the decode
+// kernel's 570 at 4, 8 tokens 689 against 985, 16 tokens 808 against 1994).
+constexpr int QM_MIN_TOKENS = 5;
 
 namespace {
 
@@ -330,6 +334,227 @@ qgemm_general_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
   }
 }
 
+// Small-batch kernel (5 to 16 tokens, 4-bit codes, groups of a multiple of 128
+// columns or one group per row): the tokens are one 16-row A operand of the
+// legacy mma.sync m16n8k16 (fp32 accumulate), the weights its B operand,
+// expanded in registers from the packed words.  The weight stream, which
+// bounds these token counts as it bounds decode, is read once for all tokens.
+// CTA = 16 weight rows (two 8-row MMA tiles) x all tokens, 8 warps splitting k
+// in slabs of 256 columns as in the decode kernel (same coalesced 16-byte
+// loads, the next slab requested before the current one is computed); each
+// warp parks its slab's packed words in shared memory so that every lane can
+// pick its fragment's codes: lane (g, t) needs, for row g of a tile and k-step
+// s, codes 2t, 2t+1 of word 2s and of word 2s+1 -- one byte of each.  A code
+// pair becomes one packed pair of M + c exactly (M = 1024 for f16, 128 for
+// bf16, the nibbles put in the low mantissa bits); a packed subtract of M + z
+// leaves c - z exactly and one packed multiply by the scale (rounded to the
+// activations' type) gives the weight, rounded once: the tensor-core kernel's
+// weights.  The activations are staged per pass of QM_KC columns in shared
+// memory (tokens past m as zeros) and read as A fragments with ldmatrix.
+constexpr int QM_WARPS = 8;
+constexpr int QM_ROWS = 16;             // weight rows per CTA
+constexpr int QM_SLAB = 256;            // columns per warp-step (8 lanes x 32 codes)
+constexpr int QM_STEP = QM_WARPS * QM_SLAB;
+constexpr int QM_KC = 2048;             // columns of X staged per pass
+constexpr int QM_XLD = QM_KC + 8;       // row stride of the staged X (16-byte aligned rows)
+constexpr int QM_WLD = 36;              // words per row of a parked slab (conflict-free reads)
+constexpr size_t QM_SMEM = sizeof(uint16_t) * 16 * QM_XLD +
+                           sizeof(uint32_t) * QM_WARPS * QM_ROWS * QM_WLD +
+                           sizeof(float) * QM_WARPS * 16 * QM_ROWS;
+
+template <bool BF16> struct QmType;
+template <> struct QmType<false> {
+  using T = __half;
+  using T2 = __half2;
+  static constexpr uint32_t MAGIC = 0x64006400u;  // 1024 in both halves
+  static constexpr float BASE = 1024.f;
+  __device__ static T2 pair(float v) { return __float2half2_rn(v); }
+};
+template <> struct QmType<true> {
+  using T = __nv_bfloat16;
+  using T2 = __nv_bfloat162;
+  static constexpr uint32_t MAGIC = 0x43004300u;  // 128 in both halves
+  static constexpr float BASE = 128.f;
+  __device__ static T2 pair(float v) { return __float2bfloat162_rn(v); }
+};
+
+template <bool BF16>
+__device__ __forceinline__ void qm_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                       uint32_t b1) {
+  if (BF16)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// byte x = two codes (low nibble first) -> the weights of that pair in T
+template <bool BF16>
+__device__ __forceinline__ uint32_t qm_weights(uint32_t x, typename QmType<BF16>::T2 zb,
+                                               typename QmType<BF16>::T2 sc) {
+  using Q = QmType<BF16>;
+  const uint32_t h = (x & 0x0Fu) | ((x & 0xF0u) << 12) | Q::MAGIC;  // M + c, exactly
+  typename Q::T2 v = *reinterpret_cast<const typename Q::T2*>(&h);
+  v = __hmul2(__hsub2(v, zb), sc);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(QM_WARPS * 32, 2)
+qgemm_mma_kernel(const typename QmType<BF16>::T* __restrict__ X, int64_t ldx, int m, int k,
+                 const int32_t* __restrict__ qw, const float* __restrict__ scales,
+                 const int32_t* __restrict__ zeros, int n, int G, int ngroups, int xvec,
+                 typename QmType<BF16>::T* __restrict__ Y, int64_t ldy) {
+  using Q = QmType<BF16>;
+  using T = typename Q::T;
+  extern __shared__ __align__(16) uint8_t qm_smem[];
+  T* xs = reinterpret_cast<T*>(qm_smem);                                   // [16][QM_XLD]
+  uint32_t* wpark = reinterpret_cast<uint32_t*>(xs + 16 * QM_XLD);         // [8][16][QM_WLD]
+  float* red = reinterpret_cast<float*>(wpark + QM_WARPS * QM_ROWS * QM_WLD);  // [8][16][16]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q = lane >> 3, p = lane & 7;   // load layout: piece p of rows 4 i + q
+  const int g = lane >> 2, t = lane & 3;   // fragment layout
+  const int r0 = (int)blockIdx.x * QM_ROWS;
+  const int64_t wpr = (int64_t)k / 8;      // words per row
+  uint32_t* park = wpark + warp * QM_ROWS * QM_WLD;
+  float acc[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  const uint32_t xs_base = (uint32_t)__cvta_generic_to_shared(xs);
+  // ldmatrix row address of this lane: matrix lane / 8, row lane % 8
+  const int lm_row = (lane & 7) + ((lane >> 3) & 1) * 8, lm_col = (lane >> 4) * 8;
+
+  for (int kc0 = 0; kc0 < k; kc0 += QM_KC) {
+    const int kcw = min(QM_KC, k - kc0);
+    int sl = warp * QM_SLAB;
+    uint4 cur[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = r0 + 4 * i + q, cl = sl + p * 32;
+      cur[i] = (row < n && cl < kcw) ? ld_stream_u4(qw + (int64_t)row * wpr + (kc0 + cl) / 8)
+                                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (kc0 == 0) {
+      // X comes from the previous kernel
+      pdl_wait();
+      pdl_trigger();
+    }
+    __syncthreads();  // the previous pass is done with xs
+    if (xvec) {
+      const int nv = kcw / 8;
+      for (int e = tid; e < 16 * nv; e += blockDim.x) {
+        const int tk = e / nv, c = 8 * (e - tk * nv);
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (tk < m) u = *reinterpret_cast<const uint4*>(X + (int64_t)tk * ldx + kc0 + c);
+        *reinterpret_cast<uint4*>(xs + tk * QM_XLD + c) = u;
+      }
+    } else {
+      for (int e = tid; e < 16 * kcw; e += blockDim.x) {
+        const int tk = e / kcw, c = e - tk * kcw;
+        xs[tk * QM_XLD + c] = tk < m ? X[(int64_t)tk * ldx + kc0 + c] : Q::pair(0.f).x;
+      }
+    }
+    __syncthreads();
+    for (; sl < kcw; sl += QM_STEP) {
+      uint4 nxt[4];
+      const int sn = sl + QM_STEP;
+      if (sn < kcw) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = r0 + 4 * i + q, cl = sn + p * 32;
+          nxt[i] = (row < n && cl < kcw) ? ld_stream_u4(qw + (int64_t)row * wpr + (kc0 + cl) / 8)
+                                         : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      __syncwarp();  // the previous slab's reads of the parking rows are done
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint4*>(park + (4 * i + q) * QM_WLD + 4 * p) = cur[i];
+      __syncwarp();
+      // the group grids of this lane's two rows in the slab's two 128-column halves
+      typename Q::T2 zb[2][2], sc[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int row = r0 + 8 * nt + g;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int c = kc0 + sl + 128 * hf;
+          const int grp = min(c, k - 1) / G;
+          float sv = 0.f, zv = 0.f;
+          if (row < n) {
+            sv = scales[(int64_t)row * ngroups + grp];
+            zv = (float)zeros[(int64_t)row * ngroups + grp];
+          }
+          zb[nt][hf] = Q::pair(Q::BASE + zv);
+          sc[nt][hf] = Q::pair(sv);
+        }
+      }
+#pragma unroll 4
+      for (int s = 0; s < QM_SLAB / 16; ++s) {
+        if (sl + 16 * s >= kcw) break;  // the same for every lane
+        uint32_t a[4];
+        const uint32_t addr =
+            xs_base + (uint32_t)((lm_row * QM_XLD + sl + 16 * s + lm_col) * (int)sizeof(T));
+        asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                     : "r"(addr));
+        const int hf = s >> 3;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const uint2 w = *reinterpret_cast<const uint2*>(park + (8 * nt + g) * QM_WLD + 2 * s);
+          const uint32_t b0 = qm_weights<BF16>((w.x >> (8 * t)) & 0xFFu, zb[nt][hf], sc[nt][hf]);
+          const uint32_t b1 = qm_weights<BF16>((w.y >> (8 * t)) & 0xFFu, zb[nt][hf], sc[nt][hf]);
+          qm_mma<BF16>(acc[nt], a, b0, b1);
+        }
+      }
+      if (sn < kcw) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+      }
+    }
+  }
+  // lane (g, t) holds, per tile nt, (token g | g + 8, row 8 nt + 2 t | + 1)
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    float* rw = red + warp * 16 * QM_ROWS;
+    rw[g * QM_ROWS + 8 * nt + 2 * t] = acc[nt][0];
+    rw[g * QM_ROWS + 8 * nt + 2 * t + 1] = acc[nt][1];
+    rw[(g + 8) * QM_ROWS + 8 * nt + 2 * t] = acc[nt][2];
+    rw[(g + 8) * QM_ROWS + 8 * nt + 2 * t + 1] = acc[nt][3];
+  }
+  __syncthreads();
+  {
+    const int tk = tid / QM_ROWS, rr = tid % QM_ROWS;  // 256 threads = 16 tokens x 16 rows
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < QM_WARPS; ++w) v += red[(w * 16 + tk) * QM_ROWS + rr];
+    if (tk < m && r0 + rr < n) Y[(int64_t)tk * ldy + r0 + rr] = qg_out<T>(v);
+  }
+}
+
+template <bool BF16>
+gptq_status launch_qgemm_mma(const void* X, int64_t ldx, int m, int k, const int32_t* qw,
+                             const float* scales, const int32_t* zeros, int n, int G, int ngroups,
+                             void* Y, int64_t ldy, cudaStream_t s) {
+  using T = typename QmType<BF16>::T;
+  if (smem_optin((const void*)qgemm_mma_kernel<BF16>, QM_SMEM) != cudaSuccess) return GPTQ_ERR_CUDA;
+  const int xvec = ((uintptr_t)X % 16) == 0 && ldx % 8 == 0;
+  launch_pdl(qgemm_mma_kernel<BF16>, dim3((unsigned)cdiv(n, QM_ROWS)), dim3(QM_WARPS * 32),
+             QM_SMEM, s, (const T*)X, ldx, m, k, qw, scales, zeros, n, G, ngroups, xvec, (T*)Y,
+             ldy);
+  GPTQ_CHECK_LAUNCH();
+  return GPTQ_OK;
+}
+
 template <int BITS, int M, typename T>
 gptq_status launch_qgemv(const T* X, int64_t ldx, int m, int k, const int32_t* qw,
                          const float* scales, const int32_t* zeros, int n, int G, int ngroups,
@@ -374,6 +599,10 @@ gptq_status qgemm_typed(const T* X, int64_t ldx, int m, int k, const int32_t* qw
       qgemm_tc_supported(X, ldx, qw, bits, k, G, g_idx != nullptr))
     return qgemm_tc(X, std::is_same<T, __nv_bfloat16>::value, m, k, ldx, qw, scales, zeros, n, G,
                     ngroups, Y, ldy, s);
+  if (m >= QM_MIN_TOKENS && m <= 16 && bits == 4 && g_idx == nullptr && k > 0 && k % 32 == 0 &&
+      (G >= k || G % 128 == 0) && ((uintptr_t)qw % 16) == 0)
+    return launch_qgemm_mma<std::is_same<T, __nv_bfloat16>::value>(X, ldx, m, k, qw, scales,
+                                                                    zeros, n, G, ngroups, Y, ldy, s);
   if (pow2 && g_idx == nullptr && ((uintptr_t)qw % 16) == 0 && k > 0) {
     const int CH = 4 * (32 / bits);
     if (k % CH == 0 && (G >= k || G % CH == 0)) {

@@ -38,8 +38,14 @@ def _inputs(n, k, bits, G, m, dtype, seed, act_perm=False):
 
 
 def _tc_path(bits, G, k, m, pass_gidx):
-    """Whether gptq_gemm takes the tensor-core kernel (contiguous inputs)."""
-    return bits == 4 and not pass_gidx and k >= 64 and (G >= k or G % 32 == 0) and m >= 17
+    """Whether gptq_gemm forms each weight in the activations' 16-bit type
+    (contiguous inputs): the tensor-core kernel from 17 tokens, the
+    small-batch mma.sync kernel for 5 to 16 tokens."""
+    if bits != 4 or pass_gidx:
+        return False
+    if m >= 17:
+        return k >= 64 and (G >= k or G % 32 == 0)
+    return m >= 5 and k % 32 == 0 and (G >= k or G % 128 == 0)
 
 
 def _check(Y, X, qw, scales, zeros, g_idx, bits, k, dtype, tc=False):
@@ -84,6 +90,10 @@ CASES = [
     (64, 1024, 3, 128, 3, torch.float16, False, False),    # 3-bit codes straddle words: general
     (80, 1024, 4, 128, 9, torch.bfloat16, True, True),     # act-order g_idx: general kernel
     (48, 512, 4, 128, 17, torch.float16, True, False),     # trivial g_idx passed explicitly
+    # small-batch mma.sync kernel (5 to 16 tokens, 4-bit, groups of 128k columns or per row)
+    (272, 4096, 4, 128, 16, torch.float16, False, False),   # two passes over X
+    (50, 2112, 4, 2112, 9, torch.bfloat16, False, False),   # one group per row, a short last pass
+    (33, 1024, 4, 256, 5, torch.float16, False, False),     # groups of 256, ragged rows
     # tensor-core kernel (17 tokens and more)
     (256, 1024, 4, 128, 64, torch.float16, False, False),
     (300, 4128, 4, 128, 300, torch.bfloat16, False, False),  # ragged rows, tokens, last K stage
@@ -117,6 +127,21 @@ def test_qgemm_full_size_q_proj(m):
     Y = quant_matmul(X.cuda(), qw.cuda(), scales.cuda(), zeros.cuda(), 4, 128)
     torch.cuda.synchronize()
     _check(Y, X, qw, scales, zeros, g_idx, 4, k, torch.float16, _tc_path(4, 128, k, m, False))
+
+
+def test_qgemm_small_batch_strided():
+    # the small-batch kernel with X rows off 16-byte boundaries (scalar staging)
+    # and a padded output
+    from post_weight_quantization_23_b200 import quant_matmul
+    n, k, m = 40, 768, 6
+    codes, scales, zeros, g_idx, X, qw = _inputs(n, k, 4, 128, m, torch.bfloat16, seed=11)
+    Xo = torch.zeros(m, k + 3, dtype=torch.bfloat16, device="cuda")
+    Xo[:, :k] = X.cuda()
+    Yp = torch.full((m, n + 8), 7.0, dtype=torch.bfloat16, device="cuda")
+    quant_matmul(Xo[:, :k], qw.cuda(), scales.cuda(), zeros.cuda(), 4, 128, out=Yp[:, :n])
+    torch.cuda.synchronize()
+    _check(Yp[:, :n], X, qw, scales, zeros, g_idx, 4, k, torch.bfloat16, True)
+    assert torch.all(Yp[:, n:] == 7.0)
 
 
 def test_qgemm_strided_and_empty():
