@@ -29,8 +29,9 @@ gptq_status qgemm_tc(const void* X, bool bf16, int64_t m, int64_t k, int64_t ldx
 // Token counts above this use the tensor-core kernel when it applies.
 constexpr int QG_TC_MIN_TOKENS = 17;
 // From this token count up to 16 the small-batch mma.sync kernel, when it applies
-// (measured on 28 7B-shaped layers per pass: 3 tokens 611 us against the decode
-// kernel's 570 at 4, 8 tokens 689 against 985, 16 tokens 808 against 1994).
+// (measured on 28 7B-shaped layers per pass: 5 tokens 533 us, 8 tokens 539
+// against the decode kernel's 985, 16 tokens 573 against 1994; the decode
+// kernel takes 4 tokens in 570 us).
 constexpr int QM_MIN_TOKENS = 5;
 
 namespace {
@@ -341,16 +342,16 @@ qgemm_general_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
 // bounds these token counts as it bounds decode, is read once for all tokens.
 // CTA = 16 weight rows (two 8-row MMA tiles) x all tokens, 8 warps splitting k
 // in slabs of 256 columns as in the decode kernel (same coalesced 16-byte
-// loads, the next slab requested before the current one is computed); each
-// warp parks its slab's packed words in shared memory so that every lane can
+// loads, the next pass's slab requested before the current one is computed);
+// each warp parks its slab's packed words in shared memory so that every lane can
 // pick its fragment's codes: lane (g, t) needs, for row g of a tile and k-step
 // s, codes 2t, 2t+1 of word 2s and of word 2s+1 -- one byte of each.  A code
 // pair becomes one packed pair of M + c exactly (M = 1024 for f16, 128 for
 // bf16, the nibbles put in the low mantissa bits); a packed subtract of M + z
 // leaves c - z exactly and one packed multiply by the scale (rounded to the
 // activations' type) gives the weight, rounded once: the tensor-core kernel's
-// weights.  The activations are staged per pass of QM_KC columns in shared
-// memory (tokens past m as zeros) and read as A fragments with ldmatrix.
+// weights.  Each warp stages its own slab's columns of the activations in
+// shared memory (tokens past m as zeros) and reads A fragments with ldmatrix.
 constexpr int QM_WARPS = 8;
 constexpr int QM_ROWS = 16;             // weight rows per CTA
 constexpr int QM_SLAB = 256;            // columns per warp-step (8 lanes x 32 codes)
@@ -433,49 +434,45 @@ qgemm_mma_kernel(const typename QmType<BF16>::T* __restrict__ X, int64_t ldx, in
   // ldmatrix row address of this lane: matrix lane / 8, row lane % 8
   const int lm_row = (lane & 7) + ((lane >> 3) & 1) * 8, lm_col = (lane >> 4) * 8;
 
+  // each pass of QM_KC = 8 x 256 columns gives every warp at most one slab, and
+  // the warp stages only its own slab's activations (no CTA-wide barrier); the
+  // next pass's packed words are requested before this pass is computed
+  const int sl = warp * QM_SLAB;
+  uint4 cur[4];
+#define QM_LOAD_SLAB(d, kc0_, kcw_)                                                            \
+  _Pragma("unroll") for (int i = 0; i < 4; ++i) {                                               \
+    const int row_ = r0 + 4 * i + q, cl_ = sl + p * 32;                                          \
+    d[i] = (row_ < n && cl_ < (kcw_)) ? ld_stream_u4(qw + (int64_t)row_ * wpr + ((kc0_) + cl_) / 8) \
+                                      : make_uint4(0u, 0u, 0u, 0u);                              \
+  }
+  QM_LOAD_SLAB(cur, 0, min(QM_KC, k))
+  // X comes from the previous kernel
+  pdl_wait();
+  pdl_trigger();
   for (int kc0 = 0; kc0 < k; kc0 += QM_KC) {
     const int kcw = min(QM_KC, k - kc0);
-    int sl = warp * QM_SLAB;
-    uint4 cur[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int row = r0 + 4 * i + q, cl = sl + p * 32;
-      cur[i] = (row < n && cl < kcw) ? ld_stream_u4(qw + (int64_t)row * wpr + (kc0 + cl) / 8)
-                                     : make_uint4(0u, 0u, 0u, 0u);
+    uint4 nxt[4];
+    const bool more = kc0 + QM_KC < k;
+    if (more) {
+      QM_LOAD_SLAB(nxt, kc0 + QM_KC, min(QM_KC, k - kc0 - QM_KC))
     }
-    if (kc0 == 0) {
-      // X comes from the previous kernel
-      pdl_wait();
-      pdl_trigger();
-    }
-    __syncthreads();  // the previous pass is done with xs
-    if (xvec) {
-      const int nv = kcw / 8;
-      for (int e = tid; e < 16 * nv; e += blockDim.x) {
-        const int tk = e / nv, c = 8 * (e - tk * nv);
-        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-        if (tk < m) u = *reinterpret_cast<const uint4*>(X + (int64_t)tk * ldx + kc0 + c);
-        *reinterpret_cast<uint4*>(xs + tk * QM_XLD + c) = u;
-      }
-    } else {
-      for (int e = tid; e < 16 * kcw; e += blockDim.x) {
-        const int tk = e / kcw, c = e - tk * kcw;
-        xs[tk * QM_XLD + c] = tk < m ? X[(int64_t)tk * ldx + kc0 + c] : Q::pair(0.f).x;
-      }
-    }
-    __syncthreads();
-    for (; sl < kcw; sl += QM_STEP) {
-      uint4 nxt[4];
-      const int sn = sl + QM_STEP;
-      if (sn < kcw) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int row = r0 + 4 * i + q, cl = sn + p * 32;
-          nxt[i] = (row < n && cl < kcw) ? ld_stream_u4(qw + (int64_t)row * wpr + (kc0 + cl) / 8)
-                                         : make_uint4(0u, 0u, 0u, 0u);
+    if (sl < kcw) {
+      const int ncol = min(QM_SLAB, kcw - sl);  // a multiple of 32
+      __syncwarp();  // this warp's reads of its columns of xs and of its parking rows are done
+      if (xvec) {
+        const int nv = ncol / 8;
+        for (int e = lane; e < 16 * nv; e += 32) {
+          const int tk = e / nv, c = sl + 8 * (e - tk * nv);
+          uint4 u = make_uint4(0u, 0u, 0u, 0u);
+          if (tk < m) u = *reinterpret_cast<const uint4*>(X + (int64_t)tk * ldx + kc0 + c);
+          *reinterpret_cast<uint4*>(xs + tk * QM_XLD + c) = u;
+        }
+      } else {
+        for (int e = lane; e < 16 * ncol; e += 32) {
+          const int tk = e / ncol, c = sl + (e - tk * ncol);
+          xs[tk * QM_XLD + c] = tk < m ? X[(int64_t)tk * ldx + kc0 + c] : Q::pair(0.f).x;
         }
       }
-      __syncwarp();  // the previous slab's reads of the parking rows are done
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         *reinterpret_cast<uint4*>(park + (4 * i + q) * QM_WLD + 4 * p) = cur[i];
@@ -498,28 +495,33 @@ qgemm_mma_kernel(const typename QmType<BF16>::T* __restrict__ X, int64_t ldx, in
           sc[nt][hf] = Q::pair(sv);
         }
       }
-#pragma unroll 4
-      for (int s = 0; s < QM_SLAB / 16; ++s) {
-        if (sl + 16 * s >= kcw) break;  // the same for every lane
-        uint32_t a[4];
-        const uint32_t addr =
-            xs_base + (uint32_t)((lm_row * QM_XLD + sl + 16 * s + lm_col) * (int)sizeof(T));
-        asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
-                     : "r"(addr));
-        const int hf = s >> 3;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const uint2 w = *reinterpret_cast<const uint2*>(park + (8 * nt + g) * QM_WLD + 2 * s);
-          const uint32_t b0 = qm_weights<BF16>((w.x >> (8 * t)) & 0xFFu, zb[nt][hf], sc[nt][hf]);
-          const uint32_t b1 = qm_weights<BF16>((w.y >> (8 * t)) & 0xFFu, zb[nt][hf], sc[nt][hf]);
-          qm_mma<BF16>(acc[nt], a, b0, b1);
+      for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll 4
+        for (int s8 = 0; s8 < QM_SLAB / 32; ++s8) {
+          const int s = 8 * hf + s8;
+          if (16 * s >= ncol) break;  // the same for every lane
+          uint32_t a[4];
+          const uint32_t addr =
+              xs_base + (uint32_t)((lm_row * QM_XLD + sl + 16 * s + lm_col) * (int)sizeof(T));
+          asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                       : "r"(addr));
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const uint2 w = *reinterpret_cast<const uint2*>(park + (8 * nt + g) * QM_WLD + 2 * s);
+            const uint32_t b0 =
+                qm_weights<BF16>((w.x >> (8 * t)) & 0xFFu, zb[nt][hf], sc[nt][hf]);
+            const uint32_t b1 =
+                qm_weights<BF16>((w.y >> (8 * t)) & 0xFFu, zb[nt][hf], sc[nt][hf]);
+            qm_mma<BF16>(acc[nt], a, b0, b1);
+          }
         }
       }
-      if (sn < kcw) {
+    }
+    if (more) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
-      }
+      for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
     }
   }
   // lane (g, t) holds, per tile nt, (token g | g + 8, row 8 nt + 2 t | + 1)
@@ -540,6 +542,8 @@ qgemm_mma_kernel(const typename QmType<BF16>::T* __restrict__ X, int64_t ldx, in
     if (tk < m && r0 + rr < n) Y[(int64_t)tk * ldy + r0 + rr] = qg_out<T>(v);
   }
 }
+
+#undef QM_LOAD_SLAB
 
 template <bool BF16>
 gptq_status launch_qgemm_mma(const void* X, int64_t ldx, int m, int k, const int32_t* qw,
