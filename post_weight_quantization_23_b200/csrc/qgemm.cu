@@ -356,7 +356,8 @@ constexpr int QM_WARPS = 8;
 constexpr int QM_ROWS = 16;             // weight rows per CTA
 constexpr int QM_SLAB = 256;            // columns per warp-step (8 lanes x 32 codes)
 constexpr int QM_STEP = QM_WARPS * QM_SLAB;
-constexpr int QM_KC = 2048;             // columns of X staged per pass
+constexpr int QM_KC = 2048;             // columns of X per pass
+static_assert(QM_KC == QM_STEP, "one slab per warp and pass");
 constexpr int QM_XLD = QM_KC + 8;       // row stride of the staged X (16-byte aligned rows)
 constexpr int QM_WLD = 36;              // words per row of a parked slab (conflict-free reads)
 constexpr size_t QM_SMEM = sizeof(uint16_t) * 16 * QM_XLD +
