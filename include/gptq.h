@@ -306,7 +306,7 @@ GPTQ_API gptq_status gptq_dequant(const int32_t* qweight, const float* scales, c
  *     group per row), X and qweight 16-byte aligned, ldx % 8 == 0: the
  *     tensor-core kernel (each weight formed in dt: the scale rounded to dt
  *     times the exact code - zero, rounded once more; fp32 accumulation);
- *   5 <= m <= 16, 4-bit, g_idx NULL, group_size a multiple of 128 (or one
+ *   3 <= m <= 16, 4-bit, g_idx NULL, group_size a multiple of 128 (or one
  *     group per row), qweight 16-byte aligned: the small-batch kernel
  *     (mma.sync, weights streamed once for all tokens and formed in dt as in
  *     the tensor-core kernel; fp32 accumulation);

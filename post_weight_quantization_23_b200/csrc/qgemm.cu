@@ -29,10 +29,10 @@ gptq_status qgemm_tc(const void* X, bool bf16, int64_t m, int64_t k, int64_t ldx
 // Token counts above this use the tensor-core kernel when it applies.
 constexpr int QG_TC_MIN_TOKENS = 17;
 // From this token count up to 16 the small-batch mma.sync kernel, when it applies
-// (measured on 28 7B-shaped layers per pass: 5 tokens 533 us, 8 tokens 539
-// against the decode kernel's 985, 16 tokens 573 against 1994; the decode
-// kernel takes 4 tokens in 570 us).
-constexpr int QM_MIN_TOKENS = 5;
+// (measured on 28 7B-shaped layers per pass: 3 and 4 tokens 522 us against the
+// decode kernel's 557, 8 tokens 539 against 985, 16 tokens 573 against 1994;
+// two tokens stay on the decode kernel, 316 us).
+constexpr int QM_MIN_TOKENS = 3;
 
 namespace {
 
@@ -335,7 +335,7 @@ qgemm_general_kernel(const T* __restrict__ X, int64_t ldx, int m, int k,
   }
 }
 
-// Small-batch kernel (5 to 16 tokens, 4-bit codes, groups of a multiple of 128
+// Small-batch kernel (3 to 16 tokens, 4-bit codes, groups of a multiple of 128
 // columns or one group per row): the tokens are one 16-row A operand of the
 // legacy mma.sync m16n8k16 (fp32 accumulate), the weights its B operand,
 // expanded in registers from the packed words.  The weight stream, which

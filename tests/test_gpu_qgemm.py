@@ -40,12 +40,12 @@ def _inputs(n, k, bits, G, m, dtype, seed, act_perm=False):
 def _tc_path(bits, G, k, m, pass_gidx):
     """Whether gptq_gemm forms each weight in the activations' 16-bit type
     (contiguous inputs): the tensor-core kernel from 17 tokens, the
-    small-batch mma.sync kernel for 5 to 16 tokens."""
+    small-batch mma.sync kernel for 3 to 16 tokens."""
     if bits != 4 or pass_gidx:
         return False
     if m >= 17:
         return k >= 64 and (G >= k or G % 32 == 0)
-    return m >= 5 and k % 32 == 0 and (G >= k or G % 128 == 0)
+    return m >= 3 and k % 32 == 0 and (G >= k or G % 128 == 0)
 
 
 def _check(Y, X, qw, scales, zeros, g_idx, bits, k, dtype, tc=False):
@@ -78,7 +78,7 @@ CASES = [
     # (n, k, bits, G, m, dtype, g_idx passed, act-order g_idx)
     (256, 1024, 4, 128, 1, torch.float16, False, False),   # decode kernel, one token
     (256, 1024, 4, 128, 2, torch.float16, False, False),   # decode kernel, a token pair
-    (100, 4352, 4, 128, 3, torch.bfloat16, False, False),  # ragged rows, 2 passes over X, odd m
+    (100, 4352, 4, 128, 3, torch.bfloat16, False, False),  # small-batch kernel: ragged rows, 3 passes, odd m
     (64, 8192, 4, 32, 5, torch.float16, False, False),     # smallest 4-bit group, 2 passes
     (50, 4352, 4, 128, 8, torch.float16, False, False),    # 8 tokens per CTA, 2 passes over X
     (100, 2048, 2, 64, 12, torch.bfloat16, False, False),  # 2-bit, two 8-token groups
@@ -90,7 +90,7 @@ CASES = [
     (64, 1024, 3, 128, 3, torch.float16, False, False),    # 3-bit codes straddle words: general
     (80, 1024, 4, 128, 9, torch.bfloat16, True, True),     # act-order g_idx: general kernel
     (48, 512, 4, 128, 17, torch.float16, True, False),     # trivial g_idx passed explicitly
-    # small-batch mma.sync kernel (5 to 16 tokens, 4-bit, groups of 128k columns or per row)
+    # small-batch mma.sync kernel (3 to 16 tokens, 4-bit, groups of 128k columns or per row)
     (272, 4096, 4, 128, 16, torch.float16, False, False),   # two passes over X
     (50, 2112, 4, 2112, 9, torch.bfloat16, False, False),   # one group per row, a short last pass
     (33, 1024, 4, 256, 5, torch.float16, False, False),     # groups of 256, ragged rows
