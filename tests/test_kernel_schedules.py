@@ -11,6 +11,9 @@ definitions exactly (bit tricks) or up to fp64 rounding (butterfly order).
 * qgemm_tc_kernel: a byte permute and a mask put codes c_2i, c_2i+1 of a word
   into a half2 holding M + c (M = 1024 for f16), and (M + c) - (M + zero) is
   c - zero exactly.
+* qgemm_mma_kernel: the parked slab layout and the bytes each lane takes form
+  the m16n8k16 B fragments of every k-step exactly once, the reads of a tile's
+  8 rows are conflict-free, and a byte becomes the pair (M + c_lo, M + c_hi).
 """
 
 import numpy as np
@@ -98,3 +101,57 @@ def test_tensor_core_pair_expansion_is_exact():
                 assert float(np.float16(h) - np.float16(1024 + z)) == c - z
                 hb = np.array([(0x4300 | hv) << 16], dtype=np.uint32).view(np.float32)[0]  # bf16
                 assert float(hb) == 128 + c and 128 + z < 256  # both exact in bf16
+
+
+def test_small_batch_fragment_schedule():
+    # qgemm_mma_kernel: lane (q, p) parks the 16-byte piece p of rows 4 i + q of a
+    # 256-column slab at words 4 p .. 4 p + 3 of row 4 i + q (rows of 36 words);
+    # for k-step s, fragment lane (g, t) of tile nt reads words 2 s, 2 s + 1 of row
+    # 8 nt + g and takes byte t of each: codes 2t, 2t+1 and 2t+8, 2t+9 of the
+    # step -- the m16n8k16 B fragment of column g; its accumulators are the C
+    # entries (g | g + 8, 2t | 2t + 1), which the kernel sums as (token, row
+    # 8 nt + 2t | + 1); the byte becomes the pair (M + c_lo, M + c_hi) exactly.
+    rng = np.random.default_rng(3)
+    codes = rng.integers(0, 16, (16, 256))
+    words = np.zeros((16, 32), dtype=np.uint64)
+    for c in range(256):
+        words[:, c // 8] |= codes[:, c].astype(np.uint64) << np.uint64(4 * (c % 8))
+    park = np.zeros((16, 36), dtype=np.uint64)
+    for lane in range(32):
+        q, p = lane >> 3, lane & 7
+        for i in range(4):
+            park[4 * i + q, 4 * p:4 * p + 4] = words[4 * i + q, 4 * p:4 * p + 4]
+    for s in range(16):
+        for nt in range(2):
+            B = np.full((16, 8), -1)
+            banks = set()
+            for lane in range(32):
+                g, t = lane >> 2, lane & 3
+                R = 8 * nt + g
+                w0, w1 = int(park[R, 2 * s]), int(park[R, 2 * s + 1])
+                b = [(w0 >> (8 * t)) & 15, (w0 >> (8 * t + 4)) & 15,
+                     (w1 >> (8 * t)) & 15, (w1 >> (8 * t + 4)) & 15]
+                for kk, v in zip((2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9), b):
+                    assert B[kk, g] == -1
+                    B[kk, g] = v
+                banks.add((R * 36 + 2 * s) % 32)
+            # the B fragments of the 32 lanes are the tile's 16 x 8 operand, each
+            # entry once; the 8 rows' reads sit in distinct bank pairs
+            assert np.array_equal(B, codes[8 * nt:8 * nt + 8, 16 * s:16 * s + 16].T)
+            assert len(banks) == 8
+    # C layout: (lane, accumulator e) -> (token, column) covers the 16 x 8 tile once
+    seen = set()
+    for lane in range(32):
+        g, t = lane >> 2, lane & 3
+        for e, (tok, n) in enumerate(((g, 2 * t), (g, 2 * t + 1), (g + 8, 2 * t), (g + 8, 2 * t + 1))):
+            seen.add((tok, n))
+    assert seen == {(tok, n) for tok in range(16) for n in range(8)}
+    # byte -> pair (M + c_lo, M + c_hi) in f16 (M = 1024) and bf16 (M = 128)
+    for x in range(256):
+        h = (x & 0x0F) | ((x & 0xF0) << 12)
+        lo, hi = np.array([0x6400 | (h & 0xFFFF), 0x6400 | (h >> 16)],
+                          dtype=np.uint16).view(np.float16)
+        assert float(lo) == 1024 + (x & 15) and float(hi) == 1024 + (x >> 4)
+        blo, bhi = (np.array([(0x4300 | (h & 0xFFFF)) << 16, (0x4300 | (h >> 16)) << 16],
+                             dtype=np.uint32).view(np.float32))
+        assert float(blo) == 128 + (x & 15) and float(bhi) == 128 + (x >> 4)
